@@ -348,6 +348,37 @@ def token_output(t: int, x, dtype: str, kind: str, weights: dict, expert_indices
     return acc
 
 
+def sampled_outputs(tokens, x, dtype: str, kind: str, weights: dict, expert_indices, gates,
+                    dest) -> np.ndarray:
+    """Output rows of the listed tokens only (for sampled full-size checks).
+
+    The same definition as ``combine`` restricted to those tokens, evaluated
+    expert by expert so that only one expert's weights are widened to fp64 at
+    a time: for each expert, its kept slots among the sampled tokens are run
+    through it together, then each token adds gate * row over its slots in
+    increasing j.
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    xs = widen(np.asarray(x)[tokens], dtype)
+    idx = np.asarray(expert_indices)[tokens]
+    dst = np.asarray(dest)[tokens]
+    g = np.asarray(gates)[tokens]
+    n, k = idx.shape
+    rows = {}
+    for e in np.unique(idx[dst >= 0]):
+        sel = [(i, j) for i in range(n) for j in range(k) if idx[i, j] == e and dst[i, j] >= 0]
+        out = expert_forward(kind, xs[[i for i, _ in sel]], *expert_weights(weights, int(e), dtype))
+        for r, key in enumerate(sel):
+            rows[key] = out[r]
+    d_out = next(iter(rows.values())).shape[0] if rows else 0
+    y = np.zeros((n, d_out))
+    for i in range(n):
+        for j in range(k):
+            if dst[i, j] >= 0:
+                y[i] += float(g[i, j]) * rows[(i, j)]
+    return y
+
+
 def moe_forward_brute_force(x, W_router, weights: dict, *, top_k: int, kind: str, dtype: str,
                             capacity_factor: float = 0.0, logit_bias=None, noise=None) -> dict:
     """Independent dense formulation, for tiny inputs only.

@@ -331,6 +331,18 @@ def test_token_output_matches_layer():
         np.testing.assert_allclose(y, r["output"][t], rtol=1e-12, atol=1e-12)
 
 
+def test_sampled_outputs_match_layer():
+    """The expert-by-expert sampled path agrees with the layer's rows."""
+    w, inp = _tiny("relu", "bf16", k=3, seed=5)
+    weights = {key: inp[key] for key in ("W_in", "W_up", "W_out")}
+    r = O.moe_forward(inp["x"], inp["W_router"], weights, top_k=3, kind="relu", dtype="bf16",
+                      d_out=w.d_out, capacity_factor=0.9)
+    tokens = [0, 7, 7, 13, 39]
+    y = O.sampled_outputs(tokens, inp["x"], "bf16", "relu", weights, r["expert_indices"],
+                          r["gates"], r["dest"])
+    np.testing.assert_allclose(y, r["output"][tokens], rtol=1e-12, atol=1e-12)
+
+
 def test_idle_expert_weights_do_not_change_output():
     """PFD 'Hot shards': an expert that receives no token can have any
     weights; the output does not change (bit for bit)."""
