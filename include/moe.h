@@ -1,0 +1,204 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) forward pass of a sparsely-gated
+ * Mixture-of-Experts layer.
+ *
+ * What the layer computes (pages cited by title and section):
+ *   [MLG] "Mixture-of-Experts Routing - LLM Internals" (mlgrind.dev),
+ *         sections "Algorithm", "Inputs", "Expected Return Format",
+ *         "Edge cases and conventions", "Follow-up".
+ *   [PFD] "Mixture of Experts: the Sparsely-Gated Layer" (paperfordummies.in),
+ *         sections "The one formula", "The code",
+ *         "Switch: top-1, one loss, and a rate limit".
+ *   [EB]  "Sparsely-gated Mixture of Experts (MoE)" (Eli Bendersky's website),
+ *         section "A Minimal Numpy Implementation".
+ *
+ *   logits  = x @ W_router (+ logit_bias) (+ noise)            fp32   [MLG Algorithm 1; PFD The code]
+ *   probs   = softmax(logits) over the E experts                fp32   [MLG Algorithm 1]
+ *   indices = the top_k experts by descending logit, ties to the lower index
+ *                                                                       [MLG Algorithm 2, Edge cases]
+ *   gates   = softmax of the chosen top_k logits (rows sum to 1)      [MLG Algorithm 2]
+ *   dispatch: slots (t, j) in token order; slot position p = earlier slots
+ *             on the same expert; kept iff p < cap,
+ *             cap = ceil(((capacity_factor * T) * top_k) / E) in fp64
+ *                                                  [MLG Follow-up; PFD Switch, The code]
+ *   y_t     = sum over kept slots j of gates[t,j] * expert_{indices[t,j]}(x_t)
+ *             (a dropped slot adds 0; gates are not renormalised)   [MLG Algorithm 3; PFD Switch]
+ *   aux     = E * sum_e f_e * P_e, f_e = slots routed to e / (T*top_k)
+ *             (before capacity), P_e = mean_t probs[t,e]             [MLG Algorithm 4]
+ *
+ * Experts (weights in the pages' x @ W orientation, row-major (E, in, out)):
+ *   MOE_EXPERT_LINEAR   : x @ W_in[e]                            (fp32 only)  [MLG Inputs]
+ *   MOE_EXPERT_RELU_MLP : relu(x @ W_in[e]) @ W_out[e]           (bf16 only)  [PFD The code; EB]
+ *   MOE_EXPERT_SWIGLU   : (silu(x @ W_in[e]) * (x @ W_up[e])) @ W_out[e]
+ *                         silu(z) = z / (1 + exp(-z))            (bf16 only)  [MLG Background; PFD]
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise.
+ *     The caller allocates and owns every buffer, the workspace included;
+ *     the library never allocates or frees device memory and keeps no state
+ *     between calls other than a per-device cache of the SM count and of the
+ *     kernels' shared-memory attributes.
+ *   - All calls are asynchronous on `stream` (NULL = legacy default stream)
+ *     and never synchronise the host, except moe_device_status.
+ *   - Host-side argument checks run before any CUDA call and return
+ *     MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE.
+ *     A failed kernel launch returns MOE_ERR_CUDA.  Range errors found on the
+ *     device (an expert index outside [0, E), inconsistent offsets, a
+ *     pipeline wait that exceeded its time limit) are written to an error
+ *     word in the workspace and reported by moe_device_status.
+ *   - Row-major layouts; rows of x, x_perm, y_perm and output are contiguous.
+ *   - bf16 tensors are IEEE bfloat16 (upper half of an fp32).
+ *   - Inputs must be finite; results for NaN or Inf inputs are undefined.
+ *   - T = 0 is valid: nothing is routed, prob_mean, f and aux_loss are 0.
+ *
+ * Limits (MOE_ERR_UNSUPPORTED otherwise): 1 <= E <= 256; 1 <= top_k <=
+ * min(E, 8); 0 <= T and T * top_k < 2^31; d, d_hidden, d_out >= 8 and
+ * multiples of 8; expert_kind/act_dtype one of the three pairs above.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, top_k out of range    */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid for the method, not built here           */
+  MOE_ERR_WORKSPACE = 3,     /* workspace null, too small or misaligned        */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed    */
+  MOE_ERR_DEVICE_CHECK = 5   /* a kernel flagged a range or timeout error      */
+};
+
+enum { MOE_EXPERT_LINEAR = 0, MOE_EXPERT_RELU_MLP = 1, MOE_EXPERT_SWIGLU = 2 };
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+
+/* Shapes and options of one layer call.  [MLG Inputs] x (T, d),
+ * W_router (d, E), expert weights (E, ...), top_k; [MLG Follow-up]
+ * capacity_factor. */
+typedef struct {
+  int32_t T;               /* tokens in the batch                             */
+  int32_t d;               /* model width: router and expert input            */
+  int32_t d_hidden;        /* expert hidden width (ReLU MLP, SwiGLU)          */
+  int32_t d_out;           /* expert output width                             */
+  int32_t E;               /* experts                                         */
+  int32_t top_k;           /* experts per token                               */
+  int32_t expert_kind;     /* MOE_EXPERT_*                                    */
+  int32_t act_dtype;       /* MOE_F32 or MOE_BF16: x, expert weights, outputs */
+  float capacity_factor;   /* <= 0: no capacity limit                         */
+} moe_config_t;
+
+/* Bytes of device workspace that every entry point below needs for `cfg`
+ * (the same figure for all of them; it is sized for moe_forward, which keeps
+ * every intermediate there).  Returns 0 if `cfg` is null or invalid. */
+size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Clears the workspace's error word (first 256 bytes), asynchronously on
+ * `stream`.  Call once after allocating a workspace, before its first use.
+ * ws must be 256-byte aligned. */
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, then copies the workspace's device error word to
+ * *code_out (0 = no device-side error since the last clear) and clears it.
+ * Returns MOE_ERR_DEVICE_CHECK if the word was non-zero, MOE_OK otherwise. */
+int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t stream);
+
+/* Router: logits, softmax, top-k and renormalised gates.
+ * [MLG Algorithm 1-2; PFD The code, `router`]
+ *   x            (T, d) act_dtype
+ *   W_router     (d, E) fp32
+ *   logit_bias   (E) fp32 or NULL: added to every token's logits
+ *   noise        (T, E) fp32 or NULL: added after the bias (noisy gating;
+ *                the caller draws it)
+ *   expert_indices (T, top_k) int32 out: by descending logit, lower index first on ties
+ *   gates        (T, top_k) fp32 out, aligned with expert_indices
+ *   prob_mean    (E) fp32 out: P_e = mean over tokens of softmax(logits)[:, e]
+ *   logits_out   (T, E) fp32 out or NULL: the fp32 logits the top-k decided on
+ * The logits are fp32: the dot product is accumulated in fp32, then the
+ * bias and then the noise are each added in fp32. */
+int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
+              const float* logit_bias, const float* noise,
+              int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,
+              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Dispatch: per-expert histogram, positions in token order, capacity, the
+ * grouped (expert-major) row layout, the load-balancing loss, and the
+ * gather of token rows into that layout.
+ * [MLG Algorithm 3-4, Follow-up; PFD The code, `moe_forward`, Switch]
+ *   x            (T, d) act_dtype
+ *   expert_indices (T, top_k) int32, each in [0, E)
+ *   prob_mean    (E) fp32: P_e (from moe_route)
+ *   counts       (E) int32 out: slots routed to e, before capacity
+ *   offsets      (E+1) int32 out: exclusive scan of kept = min(counts, cap);
+ *                expert e owns grouped rows [offsets[e], offsets[e+1])
+ *   dest         (T, top_k) int32 out: grouped row of slot (t, j), or -1 if dropped
+ *   perm_token   (T * top_k) int32 out: token of each grouped row; entries
+ *                at and beyond offsets[E] are left untouched
+ *   drop_mask    (T, top_k) uint8 out: 1 where the slot was dropped
+ *   f            (E) fp32 out: counts / (T * top_k)
+ *   aux_loss     (1) fp32 out: E * sum_e f_e * P_e (f before capacity)
+ *   x_perm       (T * top_k, d) act_dtype out: x_perm[dest[t,j]] = x[t]
+ * Bit-exact and deterministic: no floating-point atomics, no order that
+ * depends on scheduling. */
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
+                 const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
+                 int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss,
+                 void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Experts on their grouped rows: rows [offsets[e], offsets[e+1]) of x_perm
+ * go through expert e and land in the same rows of y_perm.
+ * [MLG Algorithm 3, Constraints: each expert runs only on its routed tokens]
+ *   x_perm (R_max, d) act_dtype with R_max = T * top_k; offsets (E+1) int32
+ *   with 0 = offsets[0] <= ... <= offsets[E] <= R_max.
+ *   LINEAR (fp32):   W_in (E, d, d_out); W_up, W_out NULL.
+ *   RELU_MLP (bf16): W_in (E, d, d_hidden), W_out (E, d_hidden, d_out); W_up NULL.
+ *   SWIGLU (bf16):   W_in = W_gate (E, d, d_hidden), W_up (E, d, d_hidden),
+ *                    W_out = W_down (E, d_hidden, d_out).
+ *   y_perm (R_max, d_out) act_dtype out; rows at and beyond offsets[E] untouched.
+ * bf16 experts run on tcgen05 tensor cores with fp32 accumulation in tensor
+ * memory; the hidden activation is rounded to bf16 between the two
+ * projections.  The fp32 linear expert runs in fp32 FMA. */
+int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                   const void* W_in, const void* W_up, const void* W_out, void* y_perm,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine: output[t] = sum over j = 0..top_k-1 with dest[t,j] >= 0 of
+ * gates[t,j] * y_perm[dest[t,j]], accumulated in fp32 in increasing j,
+ * rounded once to act_dtype; a token with every slot dropped gets 0.
+ * No atomics.  [MLG Algorithm 3; PFD Switch]
+ *   y_perm (rows, d_out) act_dtype; dest, gates (T, top_k); output (T, d_out). */
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
+                const float* gates, void* output, moe_stream_t stream);
+
+/* The whole layer in one call: route, dispatch, experts, combine.
+ * Returns the [MLG Expected Return Format] quantities:
+ *   output (T, d_out) act_dtype, expert_indices (T, top_k) int32,
+ *   gates (T, top_k) fp32, aux_loss (1) fp32 -- all device pointers;
+ *   counts (E) int32 and drop_mask (T, top_k) uint8 are optional (NULL).
+ * Inputs as in moe_route and moe_expert_ffn.  Intermediates live in ws. */
+int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
+                const float* logit_bias, const float* noise,
+                const void* W_in, const void* W_up, const void* W_out,
+                void* output, int32_t* expert_indices, float* gates, float* aux_loss,
+                int32_t* counts, uint8_t* drop_mask,
+                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Static text for a status code. */
+const char* moe_status_string(int status);
+
+/* Text of the most recent non-OK status returned on this host thread
+ * (argument name, CUDA error string, ...).  Empty if none. */
+const char* moe_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

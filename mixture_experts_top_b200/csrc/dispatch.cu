@@ -1,0 +1,219 @@
+// dispatch.cu - deterministic MoE dispatch: per-expert histogram, positions in
+// token order, capacity, grouped layout, load-balancing loss, row gather.
+//
+// "Mixture-of-Experts Routing - LLM Internals" (mlgrind.dev), Algorithm 3-4
+// and Follow-up; "Mixture of Experts: the Sparsely-Gated Layer"
+// (paperfordummies.in), The code (`moe_forward`: tokens routed to an expert
+// in token order, truncated to the capacity, first come first served) and
+// "Switch: top-1, one loss, and a rate limit".
+//
+// Slots s = t*k + j are ranked in increasing s.  A slot's position p on its
+// expert e is the number of earlier slots on e; it is kept iff p < cap, and
+// then lands on grouped row offsets[e] + p, offsets being the exclusive scan
+// of kept_e = min(count_e, cap).
+//
+// Three launches, no atomics on data, no scheduling-dependent order:
+//   count   - one CTA per 256-token chunk; each warp ranks 32 tokens' slots
+//             with __match_any_sync (peers with the same expert) against a
+//             per-warp running histogram, then warps are offset by an
+//             exclusive scan over warps.  Writes the chunk histogram and each
+//             slot's rank inside its chunk.
+//   scan    - one CTA: per expert, exclusive scan of the chunk histograms over
+//             chunks (chunk bases) and the total count; kept, offsets, f and
+//             aux = E * sum f_e P_e (fp64, fixed-order butterfly).
+//   scatter - one warp per token: dest, drop mask, perm_token, and the copy
+//             of x[t] into every kept grouped row with 16-byte vectors.
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kCountWarps = kChunkTokens / 32;  // 8 warps, 32 tokens each
+constexpr int kMaxE = 256;
+
+__global__ void __launch_bounds__(kCountWarps * 32)
+    dispatch_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                          int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
+                          int32_t* err) {
+  __shared__ int32_t whist[kCountWarps][kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = lane; e < E; e += 32) whist[warp][e] = 0;
+  __syncwarp();
+
+  const int c = blockIdx.x;
+  const int t0 = c * kChunkTokens + warp * 32;
+  const int t1 = min(t0 + 32, T);
+  const long s_begin = (long)t0 * k, s_end = (long)max(t1, t0) * k;
+  const uint32_t lt = lanemask_lt();
+  for (long s0 = s_begin; s0 < s_end; s0 += 32) {
+    const long s = s0 + lane;
+    const bool valid = s < s_end;
+    int e = valid ? idx[s] : -1;
+    if (valid && (e < 0 || e >= E)) {
+      report_error(err, kDevBadExpertIndex);
+      e = -1;
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int r = (e >= 0) ? whist[warp][e] + __popc(peers & lt) : 0;
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0u) whist[warp][e] += __popc(peers);
+    __syncwarp();
+    if (valid) local_rank[s] = r;
+  }
+  __syncthreads();
+  // Exclusive scan over warps, per expert; the total is the chunk histogram.
+  __shared__ int32_t wbase[kCountWarps][kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kCountWarps; ++w) {
+      wbase[w][e] = run;
+      run += whist[w][e];
+    }
+    chunk_counts[(size_t)c * E + e] = run;
+  }
+  __syncthreads();
+  for (long s0 = s_begin; s0 < s_end; s0 += 32) {
+    const long s = s0 + lane;
+    if (s < s_end) {
+      const int e = idx[s];
+      if (e >= 0 && e < E) local_rank[s] += wbase[warp][e];
+    }
+  }
+}
+
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E, int T,
+                         int k, int64_t cap, const float* __restrict__ prob_mean,
+                         int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
+                         int32_t* __restrict__ offsets, float* __restrict__ f,
+                         float* __restrict__ aux) {
+  __shared__ int32_t s_counts[kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nwarps) {
+    int carry = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < nchunks ? chunk_counts[(size_t)c * E + e] : 0;
+      const int incl = warp_inclusive_scan(v);
+      if (c < nchunks) chunk_base[(size_t)c * E + e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_counts[e] = carry;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int run = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int cnt = e < E ? s_counts[e] : 0;
+      const int kept = (cap < 0 || cnt < cap) ? cnt : (int)cap;
+      const int incl = warp_inclusive_scan(kept);
+      if (e < E) {
+        offsets[e] = run + incl - kept;
+        counts[e] = cnt;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) offsets[E] = run;
+  } else if (warp == 1) {
+    const double slots = (double)T * (double)k;
+    double acc = 0.0;
+    for (int e = lane; e < E; e += 32) {
+      const double fe = slots > 0.0 ? (double)s_counts[e] / slots : 0.0;
+      f[e] = (float)fe;
+      acc += fe * (double)prob_mean[e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) aux[0] = (float)((double)E * acc);
+  }
+}
+
+template <int ELEM>
+__global__ void __launch_bounds__(256)
+    dispatch_scatter_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ idx,
+                            int T, int k, int E, int d, int64_t cap,
+                            const int32_t* __restrict__ chunk_base,
+                            const int32_t* __restrict__ local_rank,
+                            const int32_t* __restrict__ offsets, int32_t* __restrict__ dest,
+                            int32_t* __restrict__ perm_token, uint8_t* __restrict__ drop_mask,
+                            uint8_t* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int nvec = d * ELEM / 16;  // 16-byte vectors per row
+  const size_t row_bytes = (size_t)d * ELEM;
+  for (int t = gw; t < T; t += nw) {
+    int my_dest = -1;
+    if (lane < k) {
+      const size_t s = (size_t)t * k + lane;
+      const int e = idx[s];
+      if (e >= 0 && e < E) {
+        const int pos = chunk_base[(size_t)(t / kChunkTokens) * E + e] + local_rank[s];
+        if (cap < 0 || pos < cap) my_dest = offsets[e] + pos;
+      }
+      dest[s] = my_dest;
+      drop_mask[s] = my_dest < 0 ? 1 : 0;
+      if (my_dest >= 0) perm_token[my_dest] = t;
+    }
+    int dj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dj[j] = __shfl_sync(0xffffffffu, my_dest, j);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 val = __ldg(src + v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k && dj[j] >= 0)
+          reinterpret_cast<uint4*>(x_perm + (size_t)dj[j] * row_bytes)[v] = val;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* idx,
+                            const float* prob_mean, int32_t* counts, int32_t* offsets,
+                            int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
+                            float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
+                            int32_t* local_rank, int32_t* err, cudaStream_t s) {
+  const int nchunks = ceil_div(c.T, kChunkTokens);
+  const int64_t cap = capacity_slots(c.capacity_factor, c.T, c.top_k, c.E);
+  if (nchunks > 0) {
+    dispatch_count_kernel<<<nchunks, kCountWarps * 32, 0, s>>>(idx, c.T, c.top_k, c.E,
+                                                                chunk_counts, local_rank, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  dispatch_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, nchunks, c.E, c.T, c.top_k, cap,
+                                          prob_mean, chunk_base, counts, offsets, f, aux);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || c.T == 0) return e;
+  const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
+  const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
+  if (elem == 2)
+    dispatch_scatter_kernel<2><<<blocks, 256, 0, s>>>(
+        static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d, cap, chunk_base, local_rank,
+        offsets, dest, perm_token, drop_mask, static_cast<uint8_t*>(x_perm));
+  else
+    dispatch_scatter_kernel<4><<<blocks, 256, 0, s>>>(
+        static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d, cap, chunk_base, local_rank,
+        offsets, dest, perm_token, drop_mask, static_cast<uint8_t*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,438 @@
+// grouped_gemm.cu - ragged per-expert bf16 GEMM on Blackwell tensor cores
+// (tcgen05 + tensor memory), with the expert activation fused into the
+// epilogue.
+//
+// For every expert e the rows [offsets[e], offsets[e+1]) of A (the grouped
+// token rows, K-major) are multiplied by that expert's weight matrix B_e
+// (K, N), stored in the pages' x @ W orientation, i.e. N contiguous
+// ("Mixture-of-Experts Routing - LLM Internals", mlgrind.dev, Algorithm 3 and
+// Constraints: each expert runs only on its routed tokens).  Epilogues:
+//   none   : out = acc                                  (down projection)
+//   relu   : out = max(acc, 0)                          ("Mixture of Experts:
+//            the Sparsely-Gated Layer", paperfordummies.in, The code,
+//            `expert_forward`)
+//   swiglu : out[:, c] = silu(acc_gate[:, c]) * acc_up[:, c]   (the SwiGLU
+//            expert the pages name; silu(z) = z / (1 + exp(-z)))
+//
+// B200 design
+//  * One CTA per SM, persistent, 192 threads: warp 0 = TMA producer, warp 1 =
+//    MMA issuer (one elected thread) and tensor-memory owner, warps 2-5 =
+//    epilogue (each reads the 32 TMEM lanes its warp may access).
+//  * Tile = 128 rows x 256 accumulator columns; k block 64; 4-stage smem ring
+//    of 48 KiB stages (A 16 KiB + B 32 KiB), fed by TMA with 128-byte swizzle.
+//    A is K-major; B is read straight from the (E, K, N) weights as an
+//    N-major operand through a 3-D tensor map {N, K, E} (out-of-range K and N
+//    are zero-filled, so ragged K and N tails need no special case).
+//  * SwiGLU: the 256 accumulator columns are 128 gate columns followed by the
+//    128 matching up columns (two 64-column boxes from each weight), so one
+//    M128xN256xK16 instruction feeds both and the epilogue pairs them from
+//    TMEM without any weight repacking.
+//  * tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) issued by one thread;
+//    the accumulator lives in tensor memory, two buffers of 256 columns, so
+//    the epilogue of one tile overlaps the main loop of the next.
+//  * Tile order: expert-major, then output-column block, then row block, with
+//    CTAs striding through it: CTAs running together share one weight column
+//    block (read from HBM once, reused from L2) across the expert's row blocks.
+//  * A tile that straddles two experts' rows reads the next expert's rows,
+//    computes them, and masks them at the store: no padding of the grouped
+//    layout is needed.
+//  * Every mbarrier wait is bounded; on expiry the kernel records the error in
+//    the workspace error word, drains its own copies and MMAs, frees tensor
+//    memory and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;            // rows per tile (UMMA M)
+constexpr int BK = 64;             // k per stage (one 128-byte swizzle row of bf16)
+constexpr int BN = 256;            // accumulator columns per tile (UMMA N)
+constexpr int UK = 16;             // k per tcgen05.mma (kind::f16)
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;          // 16 KiB
+constexpr int B_BOX = 64 * BK * 2;            // one 64-column box: 8 KiB
+constexpr int B_STAGE = BN * BK * 2;          // 32 KiB
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;             // two accumulator buffers
+constexpr int MAX_E = 256;
+constexpr int AUX_BYTES = 4096;               // barriers, tmem address, tile table
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + AUX_BYTES;
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
+// B bf16 (10-12 = 1), A K-major (bit 15 = 0), B N-major (bit 16 = 1),
+// N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+// Shared-memory matrix descriptors (tcgen05): start address >> 4 at bits
+// 0-13, leading byte offset >> 4 at 16-29, stride byte offset >> 4 at 32-45,
+// version 1 at bit 46, swizzle mode at 61-63 (2 = 128-byte swizzle).
+// A, K-major, 128B swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart
+// (SBO); the leading offset is unused for this layout (set to 16 bytes).
+__device__ __forceinline__ uint64_t desc_a_kmajor(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// B, N-major, 128B swizzle: each 64-column box is BK rows (k) of 128 bytes;
+// 8-k-row groups are 1024 bytes apart (SBO); boxes along N are B_BOX bytes
+// apart (LBO).
+__device__ __forceinline__ uint64_t desc_b_nmajor(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(B_BOX >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+struct GemmArgs {
+  const int32_t* offsets;
+  __nv_bfloat16* out;
+  int32_t* err;
+  int E, K, N, rows_max;
+  int n_tiles;  // output-column blocks
+};
+
+struct TileCoord {
+  int e, m0, rows, n_tile;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, const int* row_off,
+                                                 int E, int n_tiles) {
+  int lo = 0, hi = E;  // prefix[lo] <= tile < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= tile) lo = mid; else hi = mid;
+  }
+  const int local = tile - prefix[lo];
+  const int mt = (prefix[lo + 1] - prefix[lo]) / n_tiles;
+  TileCoord c;
+  c.e = lo;
+  c.n_tile = local / mt;
+  c.m0 = row_off[lo] + (local % mt) * BM;
+  c.rows = min(BM, row_off[lo + 1] - c.m0);
+  return c;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+  constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;  // output columns per tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  int* tile_prefix = reinterpret_cast<int*>(tmem_holder + 4);  // MAX_E + 1
+  int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = g.E;
+
+  // ---- prologue: tile table (warp 0), tensor memory (warp 1), barriers.
+  if (warp == 0) {
+    for (int e = lane; e <= E; e += 32) row_off[e] = g.offsets[e];
+    __syncwarp();
+    bool ok = true;
+    for (int e = lane; e < E; e += 32) ok = ok && (row_off[e] <= row_off[e + 1]);
+    if (lane == 0) ok = ok && row_off[0] == 0 && row_off[E] <= g.rows_max;
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && lane == 0 && blockIdx.x == 0) report_error(g.err, kDevBadOffsets);
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int mt = (ok && e < E) ? (row_off[e + 1] - row_off[e] + BM - 1) / BM : 0;
+      int incl = mt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (e < E) tile_prefix[e + 1] = (carry + incl) * g.n_tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      tile_prefix[0] = 0;
+      tma_prefetch_map(&tmA);
+      tma_prefetch_map(&tmB0);
+      tma_prefetch_map(&tmB1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 2 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total_tiles = tile_prefix[E];
+  const int num_kb = (g.K + BK - 1) / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, last_phase = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
+      const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
+      const int n0 = c.n_tile * OUT_COLS;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+          report_error(g.err, kDevTimeoutProducer);
+          alive = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        uint8_t* sb = sa + A_STAGE;
+        const int k0 = kb * BK;
+        mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+        tma_load_2d(sa, &tmA, &full_bar[stage], k0, c.m0);
+        if (EPI == kEpiSwiglu) {
+          tma_load_3d(sb, &tmB0, &full_bar[stage], n0, k0, c.e);
+          tma_load_3d(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e);
+          tma_load_3d(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e);
+          tma_load_3d(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tma_load_3d(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e);
+        }
+        issued_mask |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Drain: every copy this thread issued must have landed before exit.
+    for (int s = 0; s < STAGES; ++s)
+      if ((issued_mask >> s) & 1u)
+        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(g.err, kDevTimeoutDrain);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
+      if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u)) {
+        report_error(g.err, kDevTimeoutMma);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase)) {
+          report_error(g.err, kDevTimeoutMma);
+          alive = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+        const uint32_t sb = sa + A_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < BK / UK; ++kk) {
+          umma_bf16_ss(d_tmem, desc_a_kmajor(sa + kk * UK * 2), desc_b_nmajor(sb + kk * UK * 128),
+                       kIdesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&empty_bar[stage]);  // frees the stage once these MMAs finish
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!alive) break;
+      umma_commit(&tfull_bar[acc]);  // accumulator ready for the epilogue
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    // Drain: all MMAs issued by this thread complete before TMEM is freed.
+    umma_commit(drain_bar);
+    if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------ epilogue
+    const int q = warp & 3;               // TMEM lane quarter of this warp
+    const int row = q * 32 + lane;        // row inside the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
+      const int n0 = c.n_tile * OUT_COLS;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase)) {
+        report_error(g.err, kDevTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const bool valid = row < c.rows;
+      __nv_bfloat16* orow = g.out + (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      if (EPI == kEpiSwiglu) {
+#pragma unroll 1
+        for (int cc = 0; cc < OUT_COLS; cc += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_ld_32x32b_x32(tacc + cc, gr);
+          tmem_ld_32x32b_x32(tacc + OUT_COLS + cc, ur);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+              const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = n0 + cc + v * 8;
+              if (col < g.N)
+                *reinterpret_cast<uint4*>(orow + col) =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < OUT_COLS; cc += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tacc + cc, r);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float v0 = __uint_as_float(r[2 * i]), v1 = __uint_as_float(r[2 * i + 1]);
+              if (EPI == kEpiRelu) {
+                v0 = fmaxf(v0, 0.f);
+                v1 = fmaxf(v1, 0.f);
+              }
+              pk[i] = pack_bf16x2(v0, v1);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = n0 + cc + v * 8;
+              if (col < g.N)
+                *reinterpret_cast<uint4*>(orow + col) =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// A: (rows, K) bf16 row-major, box 64 (k) x 128 (rows), 128B swizzle.
+bool encode_a(CUtensorMap* m, const void* ptr, int rows, int K) {
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// B: (E, K, N) bf16 row-major as a 3-D map {N, K, E}, box 64 (n) x 64 (k) x 1.
+bool encode_b(CUtensorMap* m, const void* ptr, int E, int K, int N) {
+  const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)E};
+  const cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)K * (cuuint64_t)N * 2};
+  const cuuint32_t box[3] = {64, BK, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                     const GemmArgs& g, int grid, cudaStream_t s) {
+  auto kern = grouped_gemm_kernel<EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
+                                const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
+                                const int32_t* offsets, __nv_bfloat16* out, int32_t* err,
+                                cudaStream_t s) {
+  if (rows_max == 0) return cudaSuccess;
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  CUtensorMap ta, tb0, tb1;
+  if (!encode_a(&ta, A, rows_max, K) || !encode_b(&tb0, B0, E, K, N) ||
+      !encode_b(&tb1, B1 != nullptr ? B1 : B0, E, K, N))
+    return cudaErrorInvalidValue;
+  const int out_cols = epi == kEpiSwiglu ? BN / 2 : BN;
+  GemmArgs g;
+  g.offsets = offsets;
+  g.out = out;
+  g.err = err;
+  g.E = E;
+  g.K = K;
+  g.N = N;
+  g.rows_max = rows_max;
+  g.n_tiles = ceil_div(N, out_cols);
+  const long max_tiles = (long)(ceil_div(rows_max, BM) + E) * g.n_tiles;
+  const int grid = (int)std::min<long>((long)device_sm_count(), max_tiles);
+  switch (epi) {
+    case kEpiSwiglu: return run_gemm<kEpiSwiglu>(ta, tb0, tb1, g, grid, s);
+    case kEpiRelu: return run_gemm<kEpiRelu>(ta, tb0, tb1, g, grid, s);
+    default: return run_gemm<kEpiNone>(ta, tb0, tb1, g, grid, s);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,346 @@
+// moe_api.cu - the C ABI (include/moe.h): argument checks, workspace layout,
+// and the launch sequence of each entry point.  No device memory is
+// allocated here; every buffer belongs to the caller.
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const std::string& msg) {
+  g_last_error = msg;
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return MOE_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool is_mult8(int v) { return v >= 8 && (v % 8) == 0; }
+
+// Checks the config; returns MOE_OK or an error status (message recorded).
+int check_config(const moe_config_t* c) {
+  if (c == nullptr) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (c->E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
+  if (c->top_k < 1 || c->top_k > c->E)
+    return fail(MOE_ERR_INVALID_ARG, "top_k must satisfy 1 <= top_k <= E");
+  if (c->E > 256) return fail(MOE_ERR_UNSUPPORTED, "E > 256 is not supported");
+  if (c->top_k > 8) return fail(MOE_ERR_UNSUPPORTED, "top_k > 8 is not supported");
+  if (!std::isfinite(c->capacity_factor))
+    return fail(MOE_ERR_INVALID_ARG, "capacity_factor must be finite");
+  const bool known_kind = c->expert_kind == MOE_EXPERT_LINEAR ||
+                          c->expert_kind == MOE_EXPERT_RELU_MLP ||
+                          c->expert_kind == MOE_EXPERT_SWIGLU;
+  if (!known_kind) return fail(MOE_ERR_INVALID_ARG, "unknown expert_kind");
+  if (c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "unknown act_dtype");
+  const bool pair_ok = (c->expert_kind == MOE_EXPERT_LINEAR && c->act_dtype == MOE_F32) ||
+                       (c->expert_kind != MOE_EXPERT_LINEAR && c->act_dtype == MOE_BF16);
+  if (!pair_ok)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "supported: linear experts in fp32, ReLU-MLP and SwiGLU experts in bf16");
+  if (!is_mult8(c->d)) return fail(MOE_ERR_UNSUPPORTED, "d must be a multiple of 8, >= 8");
+  if (!is_mult8(c->d_out)) return fail(MOE_ERR_UNSUPPORTED, "d_out must be a multiple of 8, >= 8");
+  if (c->expert_kind != MOE_EXPERT_LINEAR && !is_mult8(c->d_hidden))
+    return fail(MOE_ERR_UNSUPPORTED, "d_hidden must be a multiple of 8, >= 8");
+  if ((int64_t)c->T * c->top_k >= (int64_t)1 << 31)
+    return fail(MOE_ERR_UNSUPPORTED, "T * top_k must be < 2^31");
+  return MOE_OK;
+}
+
+int check_ws(const moe_config_t& c, void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const size_t need = workspace_layout(c).total;
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) + " bytes");
+  return MOE_OK;
+}
+
+#define MOE_REQUIRE(ptr)                                                      \
+  do {                                                                        \
+    if ((ptr) == nullptr) return fail(MOE_ERR_INVALID_ARG, #ptr " is NULL"); \
+  } while (0)
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int act_bytes(const moe_config_t& c) { return c.act_dtype == MOE_BF16 ? 2 : 4; }
+
+// Up and down projections (or the linear expert) on grouped rows.
+cudaError_t run_experts(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
+                        const void* W_in, const void* W_up, const void* W_out, void* y_perm,
+                        void* ws, cudaStream_t s) {
+  const WsLayout L = workspace_layout(c);
+  int32_t* err = at<int32_t>(ws, L.ctrl);
+  const int rows_max = c.T * c.top_k;
+  if (c.expert_kind == MOE_EXPERT_LINEAR)
+    return launch_linear_expert(c, static_cast<const float*>(x_perm), offsets,
+                                static_cast<const float*>(W_in), static_cast<float*>(y_perm), err,
+                                s);
+  __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
+  const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
+  cudaError_t e = launch_grouped_gemm(
+      epi, static_cast<const __nv_bfloat16*>(x_perm), rows_max, c.d,
+      static_cast<const __nv_bfloat16*>(W_in),
+      epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
+      offsets, hidden, err, s);
+  if (e != cudaSuccess) return e;
+  return launch_grouped_gemm(kEpiNone, hidden, rows_max, c.d_hidden,
+                             static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
+                             offsets, static_cast<__nv_bfloat16*>(y_perm), err, s);
+}
+
+}  // namespace
+
+WsLayout workspace_layout(const moe_config_t& c) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  const size_t Tk = (size_t)c.T * (size_t)c.top_k;
+  const size_t E = (size_t)c.E;
+  const size_t s = (size_t)act_bytes(c);
+  const size_t n_router = (size_t)std::max(1, ceil_div(c.T, kRouterTokens));
+  const size_t n_chunks = (size_t)std::max(1, ceil_div(c.T, kChunkTokens));
+  L.ctrl = take(256);
+  L.router_part = take(n_router * E * 4);
+  L.prob_mean = take(E * 4);
+  L.chunk_counts = take(n_chunks * E * 4);
+  L.chunk_base = take(n_chunks * E * 4);
+  L.local_rank = take(Tk * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.dest = take(Tk * 4);
+  L.perm_token = take(Tk * 4);
+  L.drop_mask = take(Tk);
+  L.f = take(E * 4);
+  L.x_perm = take(Tk * (size_t)c.d * s);
+  L.hidden = take(c.expert_kind == MOE_EXPERT_LINEAR ? 0 : Tk * (size_t)c.d_hidden * 2);
+  L.y_perm = take(Tk * (size_t)c.d_out * s);
+  L.total = off;
+  return L;
+}
+
+int64_t capacity_slots(float capacity_factor, int T, int k, int E) {
+  const double cf = (double)capacity_factor;
+  if (!(cf > 0.0)) return -1;
+  return (int64_t)std::ceil(((cf * (double)T) * (double)k) / (double)E);
+}
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return workspace_layout(*cfg).total;
+}
+
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace NULL or < 256 bytes");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const cudaError_t e = cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
+}
+
+int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace NULL or < 256 bytes");
+  MOE_REQUIRE(code_out);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t code = 0;
+  cudaError_t e = cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_device_status");
+  *code_out = code;
+  if (code != 0) {
+    e = cudaMemsetAsync(ws, 0, sizeof(code), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_device_status");
+    return fail(MOE_ERR_DEVICE_CHECK, "device error code " + std::to_string(code));
+  }
+  return MOE_OK;
+}
+
+int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
+              const float* logit_bias, const float* noise, int32_t* expert_indices, float* gates,
+              float* prob_mean, float* logits_out, void* ws, size_t ws_bytes,
+              moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(gates);
+  }
+  MOE_REQUIRE(W_router);
+  MOE_REQUIRE(prob_mean);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates,
+                                     prob_mean, logits_out, at<float>(ws, L.router_part),
+                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
+}
+
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
+                 const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
+                 int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss, void* x_perm,
+                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(dest);
+    MOE_REQUIRE(perm_token);
+    MOE_REQUIRE(drop_mask);
+    MOE_REQUIRE(x_perm);
+  }
+  MOE_REQUIRE(prob_mean);
+  MOE_REQUIRE(counts);
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(f);
+  MOE_REQUIRE(aux_loss);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_dispatch(
+      c, x, expert_indices, prob_mean, counts, offsets, dest, perm_token, drop_mask, f, aux_loss,
+      x_perm, at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
+      at<int32_t>(ws, L.local_rank), at<int32_t>(ws, L.ctrl),
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch");
+}
+
+int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                   const void* W_in, const void* W_up, const void* W_out, void* y_perm, void* ws,
+                   size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(W_in);
+  if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
+  if (c.expert_kind != MOE_EXPERT_LINEAR) MOE_REQUIRE(W_out);
+  if (c.T > 0) {
+    MOE_REQUIRE(x_perm);
+    MOE_REQUIRE(y_perm);
+  }
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const cudaError_t e = run_experts(c, x_perm, offsets, W_in, W_up, W_out, y_perm, ws,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn");
+}
+
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
+                const float* gates, void* output, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(y_perm);
+    MOE_REQUIRE(dest);
+    MOE_REQUIRE(gates);
+    MOE_REQUIRE(output);
+  }
+  const cudaError_t e = launch_combine(c, y_perm, dest, gates, output,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine");
+}
+
+int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
+                const float* logit_bias, const float* noise, const void* W_in, const void* W_up,
+                const void* W_out, void* output, int32_t* expert_indices, float* gates,
+                float* aux_loss, int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(output);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(gates);
+  }
+  MOE_REQUIRE(W_router);
+  MOE_REQUIRE(W_in);
+  if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
+  if (c.expert_kind != MOE_EXPERT_LINEAR) MOE_REQUIRE(W_out);
+  MOE_REQUIRE(aux_loss);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* P = at<float>(ws, L.prob_mean);
+  int32_t* cnt = counts != nullptr ? counts : at<int32_t>(ws, L.counts);
+  uint8_t* drop = drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask);
+  int32_t* offs = at<int32_t>(ws, L.offsets);
+  int32_t* dest = at<int32_t>(ws, L.dest);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, P,
+                               nullptr, at<float>(ws, L.router_part), s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/route");
+  e = launch_dispatch(c, x, expert_indices, P, cnt, offs, dest, at<int32_t>(ws, L.perm_token),
+                      drop, at<float>(ws, L.f), aux_loss, x_perm, at<int32_t>(ws, L.chunk_counts),
+                      at<int32_t>(ws, L.chunk_base), at<int32_t>(ws, L.local_rank),
+                      at<int32_t>(ws, L.ctrl), s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/dispatch");
+  e = run_experts(c, x_perm, offs, W_in, W_up, W_out, y_perm, ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts");
+  e = launch_combine(c, y_perm, dest, gates, output, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/combine");
+  return MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: configuration not supported";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA runtime or launch failure";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a kernel reported an error";
+    default: return "unknown status";
+  }
+}
+
+const char* moe_last_error_message(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

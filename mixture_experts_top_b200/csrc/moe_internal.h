@@ -1,0 +1,79 @@
+// moe_internal.h - host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include <algorithm>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Tokens handled by one router CTA and by one dispatch chunk.
+constexpr int kRouterTokens = 64;
+constexpr int kChunkTokens = 256;
+
+// Workspace regions, byte offsets from the workspace base (each 256-aligned).
+struct WsLayout {
+  size_t ctrl;           // int32 error word (+ padding)
+  size_t router_part;    // (router CTAs, E) fp32 per-CTA column sums of probs
+  size_t prob_mean;      // (E) fp32, moe_forward only
+  size_t chunk_counts;   // (chunks, E) int32
+  size_t chunk_base;     // (chunks, E) int32
+  size_t local_rank;     // (T*k) int32 position of a slot inside its chunk
+  size_t counts;         // (E) int32           -- moe_forward intermediates
+  size_t offsets;        // (E+1) int32
+  size_t dest;           // (T*k) int32
+  size_t perm_token;     // (T*k) int32
+  size_t drop_mask;      // (T*k) uint8
+  size_t f;              // (E) fp32
+  size_t x_perm;         // (T*k, d) act
+  size_t hidden;         // (T*k, d_hidden) bf16
+  size_t y_perm;         // (T*k, d_out) act
+  size_t total;
+};
+
+WsLayout workspace_layout(const moe_config_t& c);
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Per-device properties cached on first use.
+int device_sm_count();
+
+// Launchers; each returns cudaSuccess or the launch error.
+cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,
+                         const float* bias, const float* noise, int32_t* idx, float* gates,
+                         float* prob_mean, float* logits_out, float* router_part,
+                         cudaStream_t s);
+
+cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* idx,
+                            const float* prob_mean, int32_t* counts, int32_t* offsets,
+                            int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
+                            float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
+                            int32_t* local_rank, int32_t* err, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* dest,
+                           const float* gates, void* out, cudaStream_t s);
+
+cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
+                                 const int32_t* offsets, const float* W, float* y_perm,
+                                 int32_t* err, cudaStream_t s);
+
+// Grouped bf16 GEMM on tcgen05: for every expert e, rows [offsets[e],
+// offsets[e+1]) of A (rows_max, K) times B_e (K, N) -> out rows, with a fused
+// epilogue.  epi: 0 = none, 1 = ReLU, 2 = SwiGLU (B0 = gate, B1 = up; the
+// output has N columns, each from one gate and one up column).
+enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2 };
+
+cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
+                                const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
+                                const int32_t* offsets, __nv_bfloat16* out, int32_t* err,
+                                cudaStream_t s);
+
+// Host-side capacity: ceil(((cf * T) * k) / E) in fp64, or -1 for no limit.
+int64_t capacity_slots(float capacity_factor, int T, int k, int E);
+
+}  // namespace moe

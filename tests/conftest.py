@@ -16,3 +16,11 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="session")
+def moe_lib():
+    """The built library (compiled here if it is missing or stale)."""
+    from mixture_experts_top_b200 import api, build
+    build.build()
+    return api.load_library()

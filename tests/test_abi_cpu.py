@@ -1,0 +1,130 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host -- all without a GPU (no call here reaches CUDA:
+each one fails an argument check first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_top_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(moe_lib):
+    names = declared_functions()
+    assert len(names) == 10
+    for n in names:
+        assert hasattr(moe_lib, n), n
+    assert sorted(api.exported_symbols()) == names
+
+
+def _cfg(**kw):
+    base = dict(T=64, d=32, d_hidden=0, d_out=32, E=8, top_k=2, kind="linear", dtype="f32",
+                capacity_factor=0.0)
+    base.update(kw)
+    return api.make_config(**base)
+
+
+FAKE = 0x7F0000000000          # 256-aligned, never dereferenced
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(top_k=0), api.MOE_ERR_INVALID_ARG),
+    (dict(top_k=9, E=16), api.MOE_ERR_UNSUPPORTED),
+    (dict(top_k=9), api.MOE_ERR_INVALID_ARG),            # k > E
+    (dict(E=0), api.MOE_ERR_INVALID_ARG),
+    (dict(E=257, top_k=2), api.MOE_ERR_UNSUPPORTED),
+    (dict(T=-1), api.MOE_ERR_INVALID_ARG),
+    (dict(d=12), api.MOE_ERR_UNSUPPORTED),
+    (dict(d_out=4), api.MOE_ERR_UNSUPPORTED),
+    (dict(dtype="bf16"), api.MOE_ERR_UNSUPPORTED),       # linear experts are fp32 only
+    (dict(kind="swiglu", d_hidden=64), api.MOE_ERR_UNSUPPORTED),  # SwiGLU is bf16 only
+    (dict(kind="relu", dtype="bf16", d_hidden=12), api.MOE_ERR_UNSUPPORTED),
+    (dict(capacity_factor=float("nan")), api.MOE_ERR_INVALID_ARG),
+    (dict(T=1 << 29, top_k=4), api.MOE_ERR_UNSUPPORTED),  # T*k >= 2^31
+])
+def test_config_checks(moe_lib, kw, status):
+    cfg = _cfg(**kw)
+    assert moe_lib.moe_workspace_size(ctypes.byref(cfg)) == 0
+    st = moe_lib.moe_forward(ctypes.byref(cfg), *([FAKE] * 7), FAKE, FAKE, FAKE, FAKE, None,
+                             None, FAKE, 1 << 40, None)
+    assert st == status, moe_lib.moe_last_error_message()
+
+
+def test_unknown_enum_values(moe_lib):
+    cfg = _cfg()
+    cfg.expert_kind = 7
+    assert moe_lib.moe_workspace_size(ctypes.byref(cfg)) == 0
+    cfg = _cfg()
+    cfg.act_dtype = 5
+    assert moe_lib.moe_workspace_size(ctypes.byref(cfg)) == 0
+
+
+def test_null_config(moe_lib):
+    assert moe_lib.moe_workspace_size(None) == 0
+    assert moe_lib.moe_combine(None, FAKE, FAKE, FAKE, FAKE, None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_size_grows_with_tokens(moe_lib):
+    small = moe_lib.moe_workspace_size(ctypes.byref(_cfg(T=64)))
+    big = moe_lib.moe_workspace_size(ctypes.byref(_cfg(T=6400)))
+    assert 0 < small < big and small % 256 == 0 and big % 256 == 0
+    cfg = api.make_config(8192, 4096, 14336, 4096, 8, 2, "swiglu", "bf16")
+    n = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    # grouped copies of x, the hidden activation and the expert outputs dominate
+    rows = 8192 * 2
+    assert n >= rows * (4096 + 14336 + 4096) * 2
+
+
+def test_null_pointers_and_workspace(moe_lib):
+    cfg = _cfg()
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    # x, W_router, bias, noise, W_in, W_up, W_out | output, indices, gates, aux | counts, drops
+    args = [FAKE] * 7 + [FAKE, FAKE, FAKE, FAKE] + [None, None]
+    # x is NULL
+    st = moe_lib.moe_forward(ctypes.byref(cfg), None, *args[1:], FAKE, ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    assert "x" in moe_lib.moe_last_error_message().decode()
+    # W_up may be NULL for linear experts, but the workspace may not
+    st = moe_lib.moe_forward(ctypes.byref(cfg), *args, None, ws, None)
+    assert st == api.MOE_ERR_WORKSPACE
+    st = moe_lib.moe_forward(ctypes.byref(cfg), *args, FAKE + 16, ws, None)   # misaligned
+    assert st == api.MOE_ERR_WORKSPACE
+    st = moe_lib.moe_forward(ctypes.byref(cfg), *args, FAKE, ws - 1, None)    # too small
+    assert st == api.MOE_ERR_WORKSPACE
+    assert moe_lib.moe_workspace_init(None, 1024, None) == api.MOE_ERR_WORKSPACE
+    code = ctypes.c_int32()
+    assert moe_lib.moe_device_status(None, 1024, ctypes.byref(code), None) == api.MOE_ERR_WORKSPACE
+
+
+def test_swiglu_needs_three_matrices(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    st = moe_lib.moe_expert_ffn(ctypes.byref(cfg), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, ws,
+                                None)
+    assert st == api.MOE_ERR_INVALID_ARG and "W_up" in moe_lib.moe_last_error_message().decode()
+
+
+def test_status_strings(moe_lib):
+    for s in range(6):
+        assert moe_lib.moe_status_string(s).startswith(b"MOE_")
+    assert moe_lib.moe_status_string(99) == b"unknown status"
+
+
+def test_binding_refuses_missing_library(tmp_path):
+    """No fallback: without the library every call raises."""
+    saved = api._lib
+    api._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="not found"):
+            api.load_library(str(tmp_path / "none.so"))
+    finally:
+        api._lib = saved

@@ -1,0 +1,67 @@
+"""GPU combine (moe_combine) against the oracle's combine on the same expert
+rows, destinations and gates: within one bf16 ulp of the correctly rounded
+fp64 sum (the kernel sums k fp32 products, then rounds once)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import bf16_to_f64, bf16_ulp, dev, host
+from mixture_experts_top_b200 import api
+from oracle import moe_oracle as O
+from workloads.generate import f32_to_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def run_combine(cfg, y_perm, dest, gates):
+    act = torch.bfloat16 if cfg.act_dtype == 1 else torch.float32
+    out = torch.full((cfg.T, cfg.d_out), 99.0, dtype=act, device="cuda")
+    api.moe_combine(cfg, dev(y_perm), dev(dest.astype(np.int32)), dev(gates.astype(np.float32)), out)
+    torch.cuda.synchronize()
+    return host(out)
+
+
+def _case(T, k, d_out, drop_frac, rng):
+    R = T * k
+    perm = rng.permutation(R)
+    dest = perm.reshape(T, k).astype(np.int32)
+    dest[rng.random((T, k)) < drop_frac] = -1
+    g = rng.random((T, k)).astype(np.float32)
+    g /= g.sum(axis=1, keepdims=True)
+    return dest, g.astype(np.float32)
+
+
+@pytest.mark.parametrize("T,k,d_out,drop", [(1, 1, 8, 0.0), (100, 2, 4096, 0.0), (999, 6, 2048, 0.3),
+                                            (64, 8, 768, 0.5), (300, 1, 264, 0.2)])
+def test_combine_bf16(T, k, d_out, drop):
+    rng = np.random.default_rng(T + k)
+    dest, gates = _case(T, k, d_out, drop, rng)
+    y_perm = f32_to_bf16_bits(rng.standard_normal((T * k, d_out)).astype(np.float32))
+    cfg = api.make_config(T, 64, 64, d_out, 8, k, "relu", "bf16")
+    got = bf16_to_f64(run_combine(cfg, y_perm, dest, gates))
+    ref = O.combine(bf16_to_f64(y_perm), dest, gates)
+    assert np.all(np.abs(got - ref) <= bf16_ulp(ref))
+    dropped_all = (dest < 0).all(axis=1)
+    assert (got[dropped_all] == 0).all()
+
+
+def test_combine_f32():
+    rng = np.random.default_rng(3)
+    T, k, d_out = 64, 2, 32
+    dest, gates = _case(T, k, d_out, 0.1, rng)
+    y_perm = rng.standard_normal((T * k, d_out)).astype(np.float32)
+    cfg = api.make_config(T, 32, 0, d_out, 8, k, "linear", "f32")
+    got = run_combine(cfg, y_perm, dest, gates).astype(np.float64)
+    ref = O.combine(y_perm.astype(np.float64), dest, gates)
+    assert np.all(np.abs(got - ref) <= 1e-6 * np.maximum(np.abs(ref), 1e-6))
+
+
+def test_combine_top1_gate_one_copies_row():
+    """top_k = 1 with gate 1.0: the output row is the expert row, bit for bit."""
+    rng = np.random.default_rng(4)
+    T, d_out = 50, 512
+    dest = rng.permutation(T).reshape(T, 1).astype(np.int32)
+    y_perm = f32_to_bf16_bits(rng.standard_normal((T, d_out)).astype(np.float32))
+    cfg = api.make_config(T, 64, 64, d_out, 4, 1, "relu", "bf16")
+    got = run_combine(cfg, y_perm, dest, np.ones((T, 1), np.float32))
+    assert np.array_equal(got, y_perm[dest[:, 0]])

@@ -10,6 +10,7 @@ from .generate import (  # noqa: F401
     Workload,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
+    make_expert_weights,
     make_inputs,
     make_exact_router_inputs,
 )
