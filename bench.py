@@ -224,7 +224,7 @@ def run_ours(args, rank, world):
     perm = torch.empty(R, **i32)
     f = torch.empty(E, dtype=torch.float32, device="cuda")
     x_perm = torch.empty((R, w.d), dtype=torch.bfloat16, device="cuda")
-    y_perm = torch.empty((R, w.d_out), dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.empty((R, w.d_out), dtype=torch.float32, device="cuda")
     ws = layer.ws
     stream = torch.cuda.current_stream()
 

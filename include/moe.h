@@ -36,8 +36,7 @@
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise.
  *     The caller allocates and owns every buffer, the workspace included;
  *     the library never allocates or frees device memory and keeps no state
- *     between calls other than a per-device cache of the SM count and of the
- *     kernels' shared-memory attributes.
+ *     between calls other than a per-device cache of the SM count.
  *   - All calls are asynchronous on `stream` (NULL = legacy default stream)
  *     and never synchronise the host, except moe_device_status.
  *   - Host-side argument checks run before any CUDA call and return
@@ -161,10 +160,13 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
  *   RELU_MLP (bf16): W_in (E, d, d_hidden), W_out (E, d_hidden, d_out); W_up NULL.
  *   SWIGLU (bf16):   W_in = W_gate (E, d, d_hidden), W_up (E, d, d_hidden),
  *                    W_out = W_down (E, d_hidden, d_out).
- *   y_perm (R_max, d_out) act_dtype out; rows at and beyond offsets[E] untouched.
+ *   y_perm (R_max, d_out) fp32 out (for every expert kind): each expert's
+ *   output, unrounded; rows at and beyond offsets[E] are left untouched.
  * bf16 experts run on tcgen05 tensor cores with fp32 accumulation in tensor
  * memory; the hidden activation is rounded to bf16 between the two
- * projections.  The fp32 linear expert runs in fp32 FMA. */
+ * projections (it is the second projection's tensor-core operand); the
+ * output stays fp32 until the combine rounds the layer output once.
+ * The fp32 linear expert runs in fp32 FMA. */
 int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
                    const void* W_in, const void* W_up, const void* W_out, void* y_perm,
                    void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -173,7 +175,8 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* o
  * gates[t,j] * y_perm[dest[t,j]], accumulated in fp32 in increasing j,
  * rounded once to act_dtype; a token with every slot dropped gets 0.
  * No atomics.  [MLG Algorithm 3; PFD Switch]
- *   y_perm (rows, d_out) act_dtype; dest, gates (T, top_k); output (T, d_out). */
+ *   y_perm (rows, d_out) fp32 (moe_expert_ffn's output); dest, gates
+ *   (T, top_k); output (T, d_out) act_dtype. */
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
                 const float* gates, void* output, moe_stream_t stream);
 

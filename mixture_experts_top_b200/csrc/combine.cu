@@ -5,65 +5,37 @@
 // "Mixture of Experts: the Sparsely-Gated Layer" (paperfordummies.in),
 // "Switch: top-1, one loss, and a rate limit": a dropped slot contributes 0.
 //
-// One warp per token, 16-byte vectors along the row; each output element is
-// an fp32 fused multiply-add chain over j = 0..k-1 in that order (no atomics,
-// so the result does not depend on scheduling), rounded once to the output
-// dtype.  HBM bound: reads k rows, writes one.
+// The expert rows arrive in fp32 (the experts' unrounded outputs).  One warp
+// per token, 8 columns per lane step (two 16-byte loads per expert row); each
+// output element is an fp32 fused multiply-add chain over j = 0..k-1 in that
+// order (no atomics, so the result does not depend on scheduling), rounded
+// once to the layer's dtype.  HBM bound: reads k rows, writes one.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
-template <typename XT>
-struct Vec16;
+// Stores 8 fp32 accumulators as 8 output elements.
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&a)[8]) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                                            pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+}
+__device__ __forceinline__ void store8(float* p, const float (&a)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(a[0], a[1], a[2], a[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(a[4], a[5], a[6], a[7]);
+}
 
-template <>
-struct Vec16<__nv_bfloat16> {
-  static constexpr int kN = 8;
-  __device__ static void fma_row(const void* p, float g, float (&acc)[8]) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), acc[2 * i]);
-      acc[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
-    }
-  }
-  __device__ static void store(void* p, const float (&acc)[8]) {
-    uint4 q;
-    q.x = pack_bf16x2(acc[0], acc[1]);
-    q.y = pack_bf16x2(acc[2], acc[3]);
-    q.z = pack_bf16x2(acc[4], acc[5]);
-    q.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(p) = q;
-  }
-};
-
-template <>
-struct Vec16<float> {
-  static constexpr int kN = 4;
-  __device__ static void fma_row(const void* p, float g, float (&acc)[4]) {
-    const float4 q = __ldg(reinterpret_cast<const float4*>(p));
-    acc[0] = fmaf(g, q.x, acc[0]);
-    acc[1] = fmaf(g, q.y, acc[1]);
-    acc[2] = fmaf(g, q.z, acc[2]);
-    acc[3] = fmaf(g, q.w, acc[3]);
-  }
-  __device__ static void store(void* p, const float (&acc)[4]) {
-    *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  }
-};
-
-template <typename XT>
+// y_perm rows are the experts' fp32 outputs; OutT is the layer's dtype.
+template <typename OutT>
 __global__ void __launch_bounds__(256)
-    combine_kernel(const XT* __restrict__ y_perm, const int32_t* __restrict__ dest,
-                   const float* __restrict__ gates, XT* __restrict__ out, int T, int k, int d_out) {
-  constexpr int V = Vec16<XT>::kN;
+    combine_kernel(const float* __restrict__ y_perm, const int32_t* __restrict__ dest,
+                   const float* __restrict__ gates, OutT* __restrict__ out, int T, int k,
+                   int d_out) {
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int nvec = d_out / V;
+  const int nvec = d_out / 8;  // 8 columns per lane step
   for (int t = gw; t < T; t += nw) {
     int dl = -1;
     float gl = 0.f;
@@ -78,34 +50,44 @@ __global__ void __launch_bounds__(256)
       dj[j] = __shfl_sync(0xffffffffu, dl, j);
       gj[j] = __shfl_sync(0xffffffffu, gl, j);
     }
-    XT* orow = out + (size_t)t * d_out;
+    OutT* orow = out + (size_t)t * d_out;
 #pragma unroll 2
     for (int v = lane; v < nvec; v += 32) {
-      float acc[V];
+      float acc[8];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < k && dj[j] >= 0)
-          Vec16<XT>::fma_row(y_perm + (size_t)dj[j] * d_out + (size_t)v * V, gj[j], acc);
-      Vec16<XT>::store(orow + (size_t)v * V, acc);
+      for (int j = 0; j < 8; ++j) {
+        if (j < k && dj[j] >= 0) {
+          const float4* src = reinterpret_cast<const float4*>(y_perm + (size_t)dj[j] * d_out) + 2 * v;
+          const float4 a = __ldg(src), b = __ldg(src + 1);
+          acc[0] = fmaf(gj[j], a.x, acc[0]);
+          acc[1] = fmaf(gj[j], a.y, acc[1]);
+          acc[2] = fmaf(gj[j], a.z, acc[2]);
+          acc[3] = fmaf(gj[j], a.w, acc[3]);
+          acc[4] = fmaf(gj[j], b.x, acc[4]);
+          acc[5] = fmaf(gj[j], b.y, acc[5]);
+          acc[6] = fmaf(gj[j], b.z, acc[6]);
+          acc[7] = fmaf(gj[j], b.w, acc[7]);
+        }
+      }
+      store8(orow + (size_t)v * 8, acc);
     }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* dest,
+cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int32_t* dest,
                            const float* gates, void* out, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
   if (c.act_dtype == MOE_BF16)
     combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(y_perm), dest, gates, static_cast<__nv_bfloat16*>(out),
-        c.T, c.top_k, c.d_out);
+        y_perm, dest, gates, static_cast<__nv_bfloat16*>(out), c.T, c.top_k, c.d_out);
   else
-    combine_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(y_perm), dest, gates,
-                                                 static_cast<float*>(out), c.T, c.top_k, c.d_out);
+    combine_kernel<float><<<blocks, 256, 0, s>>>(y_perm, dest, gates, static_cast<float*>(out),
+                                                 c.T, c.top_k, c.d_out);
   return cudaGetLastError();
 }
 

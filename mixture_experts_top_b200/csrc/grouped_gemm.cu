@@ -7,7 +7,8 @@
 // (K, N), stored in the pages' x @ W orientation, i.e. N contiguous
 // ("Mixture-of-Experts Routing - LLM Internals", mlgrind.dev, Algorithm 3 and
 // Constraints: each expert runs only on its routed tokens).  Epilogues:
-//   none   : out = acc                                  (down projection)
+//   none   : out = acc, kept in fp32                    (down projection: the
+//            expert output stays unrounded until the combine)
 //   relu   : out = max(acc, 0)                          ("Mixture of Experts:
 //            the Sparsely-Gated Layer", paperfordummies.in, The code,
 //            `expert_forward`)
@@ -89,7 +90,7 @@ __device__ __forceinline__ uint64_t desc_b_nmajor(uint32_t saddr) {
 
 struct GemmArgs {
   const int32_t* offsets;
-  __nv_bfloat16* out;
+  void* out;  // bf16 for kEpiRelu / kEpiSwiglu, fp32 for kEpiNone
   int32_t* err;
   int E, K, N, rows_max;
   int n_tiles;  // output-column blocks
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
-      __nv_bfloat16* orow = g.out + (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      const size_t orow_off = (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       if (EPI == kEpiSwiglu) {
 #pragma unroll 1
         for (int cc = 0; cc < OUT_COLS; cc += 32) {
@@ -305,12 +306,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const int col = n0 + cc + v * 8;
               if (col < g.N)
                 *reinterpret_cast<uint4*>(orow + col) =
                     make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+      } else if (EPI == kEpiNone) {
+#pragma unroll 1
+        for (int cc = 0; cc < OUT_COLS; cc += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tacc + cc, r);
+          tmem_ld_wait();
+          if (valid) {
+            float* orow = static_cast<float*>(g.out) + orow_off;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int col = n0 + cc + v * 4;
+              if (col < g.N)
+                *reinterpret_cast<uint4*>(orow + col) =
+                    make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
             }
           }
         }
@@ -324,13 +343,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float v0 = __uint_as_float(r[2 * i]), v1 = __uint_as_float(r[2 * i + 1]);
-              if (EPI == kEpiRelu) {
-                v0 = fmaxf(v0, 0.f);
-                v1 = fmaxf(v1, 0.f);
-              }
+              const float v0 = fmaxf(__uint_as_float(r[2 * i]), 0.f);
+              const float v1 = fmaxf(__uint_as_float(r[2 * i + 1]), 0.f);
               pk[i] = pack_bf16x2(v0, v1);
             }
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const int col = n0 + cc + v * 8;
@@ -408,7 +425,7 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, __nv_bfloat16* out, int32_t* err,
+                                const int32_t* offsets, void* out, int32_t* err,
                                 cudaStream_t s) {
   if (rows_max == 0) return cudaSuccess;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;

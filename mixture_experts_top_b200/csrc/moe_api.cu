@@ -102,7 +102,7 @@ cudaError_t run_experts(const moe_config_t& c, const void* x_perm, const int32_t
   if (e != cudaSuccess) return e;
   return launch_grouped_gemm(kEpiNone, hidden, rows_max, c.d_hidden,
                              static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
-                             offsets, static_cast<__nv_bfloat16*>(y_perm), err, s);
+                             offsets, y_perm, err, s);
 }
 
 }  // namespace
@@ -134,7 +134,7 @@ WsLayout workspace_layout(const moe_config_t& c) {
   L.f = take(E * 4);
   L.x_perm = take(Tk * (size_t)c.d * s);
   L.hidden = take(c.expert_kind == MOE_EXPERT_LINEAR ? 0 : Tk * (size_t)c.d_hidden * 2);
-  L.y_perm = take(Tk * (size_t)c.d_out * s);
+  L.y_perm = take(Tk * (size_t)c.d_out * 4);
   L.total = off;
   return L;
 }
@@ -280,7 +280,7 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest
     MOE_REQUIRE(gates);
     MOE_REQUIRE(output);
   }
-  const cudaError_t e = launch_combine(c, y_perm, dest, gates, output,
+  const cudaError_t e = launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output,
                                        reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine");
 }
@@ -324,7 +324,7 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/dispatch");
   e = run_experts(c, x_perm, offs, W_in, W_up, W_out, y_perm, ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts");
-  e = launch_combine(c, y_perm, dest, gates, output, s);
+  e = launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output, s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/combine");
   return MOE_OK;
 }

@@ -32,7 +32,7 @@ struct WsLayout {
   size_t f;              // (E) fp32
   size_t x_perm;         // (T*k, d) act
   size_t hidden;         // (T*k, d_hidden) bf16
-  size_t y_perm;         // (T*k, d_out) act
+  size_t y_perm;         // (T*k, d_out) fp32
   size_t total;
 };
 
@@ -55,7 +55,7 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
                             int32_t* local_rank, int32_t* err, cudaStream_t s);
 
-cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* dest,
+cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int32_t* dest,
                            const float* gates, void* out, cudaStream_t s);
 
 cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
@@ -64,13 +64,14 @@ cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
 
 // Grouped bf16 GEMM on tcgen05: for every expert e, rows [offsets[e],
 // offsets[e+1]) of A (rows_max, K) times B_e (K, N) -> out rows, with a fused
-// epilogue.  epi: 0 = none, 1 = ReLU, 2 = SwiGLU (B0 = gate, B1 = up; the
-// output has N columns, each from one gate and one up column).
+// epilogue.  epi: 0 = none (fp32 output), 1 = ReLU (bf16 output), 2 = SwiGLU
+// (bf16 output; B0 = gate, B1 = up; each output column pairs one gate and
+// one up column).
 enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2 };
 
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, __nv_bfloat16* out, int32_t* err,
+                                const int32_t* offsets, void* out, int32_t* err,
                                 cudaStream_t s);
 
 // Host-side capacity: ceil(((cf * T) * k) / E) in fp64, or -1 for no limit.

@@ -349,14 +349,15 @@ def token_output(t: int, x, dtype: str, kind: str, weights: dict, expert_indices
 
 
 def sampled_outputs(tokens, x, dtype: str, kind: str, weights: dict, expert_indices, gates,
-                    dest) -> np.ndarray:
+                    dest, return_rows: bool = False):
     """Output rows of the listed tokens only (for sampled full-size checks).
 
     The same definition as ``combine`` restricted to those tokens, evaluated
     expert by expert so that only one expert's weights are widened to fp64 at
     a time: for each expert, its kept slots among the sampled tokens are run
     through it together, then each token adds gate * row over its slots in
-    increasing j.
+    increasing j.  With ``return_rows`` the kept slots' expert output rows
+    are returned as well, stacked in (token, j) order.
     """
     tokens = np.asarray(tokens, dtype=np.int64)
     xs = widen(np.asarray(x)[tokens], dtype)
@@ -376,6 +377,8 @@ def sampled_outputs(tokens, x, dtype: str, kind: str, weights: dict, expert_indi
         for j in range(k):
             if dst[i, j] >= 0:
                 y[i] += float(g[i, j]) * rows[(i, j)]
+    if return_rows:
+        return y, np.array([rows[key] for key in sorted(rows)])
     return y
 
 
