@@ -127,6 +127,30 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
               int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,
               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route without a workspace.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- for
+ * example a plugin running inside a host program whose memory pool owns the
+ * whole GPU and hands out no scratch, or a service that forbids allocation
+ * once it is serving.  Arguments, outputs and results are those of
+ * moe_route; the caller still passes every input and output buffer.
+ *   Scratch: the per-CTA column sums of the probabilities go to one fixed
+ *   array inside the library, 65536 floats (256 KiB), which every GPU that
+ *   loads the library keeps until the process exits.  A call needs
+ *   ceil(T / 64) * E floats of it; larger calls return MOE_ERR_UNSUPPORTED
+ *   (use moe_route with a workspace instead).  The array is overwritten in
+ *   full by each call before it is read, so nothing needs clearing.
+ *   Sharing: every call on a device uses the same array and it keeps the
+ *   last call's contents, so calls whose kernels overlap on the GPU (on
+ *   different streams, or from different host threads without ordering)
+ *   race on it; order such calls on one stream.
+ *   Set-up: the first call on each device looks up the array's device
+ *   address (with that device current) and caches it; make that first call
+ *   before any stream capture.  No call allocates or frees memory. */
+int moe_route_noalloc(const moe_config_t* cfg, const void* x, const float* W_router,
+                      const float* logit_bias, const float* noise,
+                      int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,
+                      moe_stream_t stream);
+
 /* Dispatch: per-expert histogram, positions in token order, capacity, the
  * grouped (expert-major) row layout, the load-balancing loss, and the
  * gather of token rows into that layout.

@@ -30,6 +30,7 @@ _SIGNATURES = {
     "moe_workspace_init": (ctypes.c_int, [_c_p, ctypes.c_size_t, _c_p]),
     "moe_device_status": (ctypes.c_int, [_c_p, ctypes.c_size_t, _c_p, _c_p]),
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
+    "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
     "moe_dispatch": (ctypes.c_int, [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn": (ctypes.c_int, [_c_p] * 8 + [ctypes.c_size_t, _c_p]),
     "moe_combine": (ctypes.c_int, [_c_p] * 6),
@@ -141,6 +142,16 @@ def moe_route(cfg, x, W_router, logit_bias, noise, expert_indices, gates, prob_m
         ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
         _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _ptr(ws),
         ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_noalloc(cfg, x, W_router, logit_bias, noise, expert_indices, gates, prob_mean,
+                      logits_out, stream=None) -> None:
+    """moe_route for callers that cannot allocate: no workspace argument;
+    the library's fixed scratch array is used (see include/moe.h)."""
+    _check(load_library().moe_route_noalloc(
+        ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
+        _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _stream(stream)),
+        "moe_route_noalloc")
 
 
 def moe_dispatch(cfg, x, expert_indices, prob_mean, counts, offsets, dest, perm_token, drop_mask,

@@ -344,3 +344,69 @@ const char* moe_status_string(int status) {
 const char* moe_last_error_message(void) { return g_last_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_route_noalloc: the router for callers that cannot allocate device
+// memory.  Its only scratch, the per-CTA column sums of the probabilities,
+// lives in a fixed file-scope device array instead of a caller workspace.
+// ---------------------------------------------------------------------------
+
+namespace moe {
+namespace {
+
+// Fixed scratch of the allocation-free router: 65536 floats (256 KiB),
+// reserved on every GPU that loads this library until the process exits.
+constexpr size_t kNoAllocScratchFloats = 65536;
+static __device__ __align__(256) float g_route_scratch[kNoAllocScratchFloats];
+
+// Device address of g_route_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is asked of
+// the runtime once per device (with that device current) and cached.
+cudaError_t route_scratch_address(float** out) {
+  static std::mutex mu;
+  static float* cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = static_cast<float*>(p);
+  }
+  *out = cached[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_route_noalloc(const moe_config_t* cfg, const void* x, const float* W_router,
+                                 const float* logit_bias, const float* noise,
+                                 int32_t* expert_indices, float* gates, float* prob_mean,
+                                 float* logits_out, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(gates);
+  }
+  MOE_REQUIRE(W_router);
+  MOE_REQUIRE(prob_mean);
+  const size_t need = (size_t)std::max(1, ceil_div(c.T, kRouterTokens)) * (size_t)c.E;
+  if (need > kNoAllocScratchFloats)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_route_noalloc: ceil(T/64) * E = " + std::to_string(need) +
+                    " exceeds its fixed scratch of " + std::to_string(kNoAllocScratchFloats) +
+                    " floats; use moe_route with a workspace");
+  float* scratch = nullptr;
+  cudaError_t e = route_scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_route_noalloc: cudaGetSymbolAddress");
+  e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, prob_mean,
+                   logits_out, scratch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_noalloc");
+}
