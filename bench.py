@@ -191,6 +191,8 @@ def run_ours(args, rank, world):
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_tokens(args.tokens)
     peaks, peak_src = load_peaks()
 
     # inputs: weights identical on every rank, tokens drawn per rank
@@ -374,6 +376,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for profiling; not a bench line)")
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
