@@ -113,6 +113,30 @@ def profiled_traffic(kernel_file: str, summary: str):
     return float(m_b.group(1))
 
 
+# ------------------------------------------------------------- ranks (N>1) --
+
+def rank_token_seed(rank: int) -> int:
+    """Seed of a rank's token batch: rank 0 uses the workload's own batch,
+    other ranks independent batches; the weights (seed 0) are replicated."""
+    return 0 if rank == 0 else 1000 + rank
+
+
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise max over ranks of a list of floats (the step time of the
+    slowest rank decides)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------- reference arm --
 
 def blas_threads():
@@ -199,7 +223,8 @@ def run_ours(args, rank, world):
     t0 = time.time()
     inp = make_inputs(w, seed=0)
     if rank > 0:
-        inp.update({k: v for k, v in make_inputs(w, seed=1000 + rank, with_experts=False).items()
+        inp.update({k: v for k, v in make_inputs(w, seed=rank_token_seed(rank),
+                                                 with_experts=False).items()
                     if k in ("x", "noise")})
     log(f"[rank {rank}] inputs generated in {time.time() - t0:.1f}s")
 
@@ -306,19 +331,16 @@ def run_ours(args, rank, world):
         raise RuntimeError(f"device error word {status} after the benchmark")
 
     # max over ranks
-    t = torch.tensor([elapsed_ms, e2e_ms] + stage_ms, dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(t[0]), float(t[1])
-    stage_ms = [float(v) for v in t[2:]]
+    red = max_over_ranks([elapsed_ms, e2e_ms] + stage_ms, world, device="cuda")
+    elapsed_ms, e2e_ms, stage_ms = red[0], red[1], red[2:]
     if rank != 0:
         return 0
 
     counts = o.counts.cpu().numpy()
-    rows = int(min(counts.sum(), R))
+    rows = A.kept_rows(counts, w.capacity_factor, T, k)
     used = int((counts > 0).sum())
     ms_step = elapsed_ms / args.steps
-    value = world * T / (ms_step / 1e3)
+    value = job_value(world, T, ms_step)
     flops = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
     t_exp = stage_ms[2] / 1e3
     tensor_peak = peaks["bf16_tflops"]
@@ -347,7 +369,7 @@ def run_ours(args, rank, world):
         "config": workload_config(w, world),
         "roofline": gemm,
         "stages": stages,
-        "e2e": {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_value(world, T, e2e_ms / args.steps), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "moe_forward via the Python binding; x copied from pinned host memory, "
                        "output and aux_loss copied back, every step"},

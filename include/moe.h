@@ -136,7 +136,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
  *   Scratch: the per-CTA column sums of the probabilities go to one fixed
  *   array inside the library, 65536 floats (256 KiB), which every GPU that
  *   loads the library keeps until the process exits.  A call needs
- *   ceil(T / 64) * E floats of it; larger calls return MOE_ERR_UNSUPPORTED
+ *   ceil(T / 32) * E floats of it; larger calls return MOE_ERR_UNSUPPORTED
  *   (use moe_route with a workspace instead).  The array is overwritten in
  *   full by each call before it is read, so nothing needs clearing.
  *   Sharing: every call on a device uses the same array and it keeps the

@@ -54,6 +54,19 @@ def expert_weight_bytes(used_experts: int, d: int, d_hidden: int, d_out: int, ki
     return used_experts * per * elem
 
 
+def capacity_slots(capacity_factor: float, T: int, k: int, E: int):
+    """ceil(((cf * T) * k) / E) slots per expert, or None without a limit."""
+    import math
+    cf = float(capacity_factor)
+    return None if cf <= 0 else int(math.ceil(((cf * T) * k) / E))
+
+
+def kept_rows(counts, capacity_factor: float, T: int, k: int) -> int:
+    """Rows the experts process: per expert min(count, capacity), summed."""
+    cap = capacity_slots(capacity_factor, T, k, len(counts))
+    return int(sum(c if cap is None else min(int(c), cap) for c in counts))
+
+
 def router_bytes(T: int, d: int, E: int, k: int, elem: int, noise: bool) -> int:
     """x read once, W_router read once, indices and gates written."""
     return T * d * elem + d * E * 4 + (T * E * 4 if noise else 0) + T * k * 8
@@ -68,9 +81,9 @@ def permute_bytes(T: int, rows: int, d: int, elem: int) -> int:
     return T * d * elem + rows * d * elem
 
 
-def combine_bytes(T: int, rows: int, d_out: int, k: int, elem: int) -> int:
-    """Each kept expert-output row read once, dest+gates read, y written."""
-    return rows * d_out * elem + T * k * 8 + T * d_out * elem
+def combine_bytes(T: int, rows: int, d_out: int, k: int, out_elem: int, row_elem: int = 4) -> int:
+    """Each kept expert-output row (fp32) read once, dest+gates read, y written."""
+    return rows * d_out * row_elem + T * k * 8 + T * d_out * out_elem
 
 
 def gemm_roofline_seconds(flops: float, weight_bytes: float, act_bytes: float,

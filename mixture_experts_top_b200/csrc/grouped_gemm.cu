@@ -415,7 +415,7 @@ template <int EPI>
 cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                      const GemmArgs& g, int grid, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, g);
   return cudaGetLastError();

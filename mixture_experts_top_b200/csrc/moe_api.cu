@@ -4,6 +4,8 @@
 #include <cmath>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "moe_device.cuh"
 #include "moe_internal.h"
@@ -158,6 +160,20 @@ int device_sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& p : done)
+    if (p.first == dev && p.second == kernel) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(dev, kernel);
+  return e;
 }
 
 }  // namespace moe
@@ -400,7 +416,7 @@ extern "C" int moe_route_noalloc(const moe_config_t* cfg, const void* x, const f
   const size_t need = (size_t)std::max(1, ceil_div(c.T, kRouterTokens)) * (size_t)c.E;
   if (need > kNoAllocScratchFloats)
     return fail(MOE_ERR_UNSUPPORTED,
-                "moe_route_noalloc: ceil(T/64) * E = " + std::to_string(need) +
+                "moe_route_noalloc: ceil(T/32) * E = " + std::to_string(need) +
                     " exceeds its fixed scratch of " + std::to_string(kNoAllocScratchFloats) +
                     " floats; use moe_route with a workspace");
   float* scratch = nullptr;

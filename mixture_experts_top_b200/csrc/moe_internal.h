@@ -12,8 +12,11 @@
 
 namespace moe {
 
-// Tokens handled by one router CTA and by one dispatch chunk.
-constexpr int kRouterTokens = 64;
+// Smallest number of tokens a router CTA owns (every router configuration
+// uses a whole multiple of it, so ceil(T / kRouterTokens) bounds the number
+// of router CTAs and sizes the per-CTA partial sums), and the tokens of one
+// dispatch chunk.
+constexpr int kRouterTokens = 32;
 constexpr int kChunkTokens = 256;
 
 // Workspace regions, byte offsets from the workspace base (each 256-aligned).
@@ -42,6 +45,9 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Per-device properties cached on first use.
 int device_sm_count();
+
+// Sets a kernel's dynamic shared-memory limit once per (device, kernel).
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,

@@ -9,46 +9,58 @@
 // code, `router`: an optional per-expert bias, then optional noise, are added
 // to the logits before the softmax and the top-k.
 //
-// Design (B200): a CTA owns 64 tokens.  The contraction x (64, d) @ W (d, E)
-// runs on the fp32 pipes (fp32 results are required, so no tensor cores):
-// x and W stream through shared memory in 64-wide k chunks with cp.async
-// double buffering; each lane owns two tokens and TN experts, so W values
-// are warp-wide broadcasts and x rows are read as conflict-free 16-byte
-// vectors (rows padded by 16 bytes).  Warps split experts (WN) and the k
-// range (KS); the KS partial sums are added in a fixed order in shared
-// memory.  Then one warp per token finishes the row in registers: bias and
-// noise, max-subtracted softmax, k rounds of a warp-wide max over 64-bit
-// keys (order-preserving logit bits, then the complemented expert index so
-// the lower index wins ties), the gates, and a running per-lane sum of the
-// probabilities.  Column sums are combined across warps in a fixed order and
-// written per CTA; a second tiny kernel adds the CTA partials in fp64.
+// Design (B200): a thread-block cluster of S CTAs (S = 1..8) owns a tile of
+// 32 or 64 tokens; each CTA of the cluster takes 1/S of the contraction
+// range d.  The contraction x (tile, d/S) @ W (d/S, E) runs on the fp32 pipes
+// (fp32 logits are required, so no tensor cores): x and W stream through
+// shared memory in k chunks with a multi-stage cp.async pipeline; each lane
+// owns TM tokens and TN experts, so W values are warp-wide broadcasts and x
+// rows are read as conflict-free 16-byte vectors (rows padded by 16 bytes).
+// k is consumed in pairs with packed fp32 FMAs (fma.rn.f32x2): unpacking a
+// 32-bit word of bf16 x gives the pair {x_k, x_k+1}, and W is stored
+// interleaved by k pairs so one broadcast load feeds two experts.
+// Warps split experts (WN) and the chunk (KS); the KS partial sums are added
+// in a fixed order in shared memory.  Splitting d over the cluster keeps the
+// serial chain of chunk loads per CTA short, so the kernel is not bound by
+// one CTA's load latency when there are few tokens.  The S partial logit
+// tiles are then added in rank order through distributed shared memory, and
+// the cluster's warps finish one token each: bias and noise, max-subtracted
+// softmax, k rounds of a warp-wide max over 64-bit keys (order-preserving
+// logit bits, then the complemented expert index so the lower index wins
+// ties), the gates, and a running per-lane sum of the probabilities.  The
+// column sums are added across warps and CTAs in a fixed order into one row
+// per token tile; a second small kernel adds the rows in fp64.
+#include <cooperative_groups.h>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 namespace {
 
+// 16 bytes of x -> VEC/2 pairs {x_k, x_k+1} (fp32).
 template <typename XT>
 struct XVec;
 template <>
 struct XVec<float> {
   static constexpr int kN = 4;  // elements per 16 bytes
-  __device__ static void load(const float* p, float (&v)[4]) {
+  __device__ static void load(const float* p, float2 (&v)[2]) {
     const float4 q = *reinterpret_cast<const float4*>(p);
-    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    v[0] = make_float2(q.x, q.y);
+    v[1] = make_float2(q.z, q.w);
   }
 };
 template <>
 struct XVec<__nv_bfloat16> {
   static constexpr int kN = 8;
-  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+  __device__ static void load(const __nv_bfloat16* p, float2 (&v)[4]) {
     const uint4 q = *reinterpret_cast<const uint4*>(p);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+    for (int i = 0; i < 4; ++i)
+      v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
   }
 };
 
@@ -83,149 +95,158 @@ struct RouterArgs {
   int T, d, E, k;
 };
 
-constexpr int kBM = kRouterTokens;   // tokens per CTA (two per lane)
-constexpr int kStages = 2;
 constexpr int kMaxK = 8;
 
-template <typename XT, int TN, int WN, int KS, int BK>
+// TM tokens per lane (a CTA owns BM = 32 * TM tokens), TN experts per lane,
+// WN warps across experts, KS warps across the k chunk, BK k per chunk,
+// ST cp.async pipeline stages.
+template <typename XT, int TM, int TN, int WN, int KS, int BK, int ST>
 struct RouterShape {
   static constexpr int VEC = XVec<XT>::kN;
+  static constexpr int BM = 32 * TM;
   static constexpr int EP = TN * WN;            // experts covered (padded E)
   static constexpr int THREADS = 32 * WN * KS;
   static constexpr int XROW = BK + VEC;         // padded x row, elements
-  static constexpr int X_STAGE = kBM * XROW;    // elements
+  static constexpr int X_STAGE = BM * XROW;     // elements
   static constexpr int W_STAGE = BK * EP;       // floats
-  static constexpr int PIPE_BYTES = kStages * (X_STAGE * (int)sizeof(XT) + W_STAGE * 4);
-  static constexpr int PART_BYTES = KS * kBM * EP * 4;
+  static constexpr int PIPE_BYTES = ST * (X_STAGE * (int)sizeof(XT) + W_STAGE * 4);
+  static constexpr int PART_BYTES = KS * BM * EP * 4;
   static constexpr int CS_BYTES = WN * KS * EP * 4;
   static constexpr int MAIN_BYTES = PIPE_BYTES > PART_BYTES ? PIPE_BYTES : PART_BYTES;
   static constexpr int SMEM = MAIN_BYTES + CS_BYTES;
   static_assert((BK / KS) % VEC == 0, "k split must hold whole vectors");
   static_assert(TN % 4 == 0, "experts per lane must be a multiple of 4");
+  static_assert(BK % 2 == 0, "k is consumed in pairs");
+  static_assert(BM % kRouterTokens == 0, "CTA tiles are whole multiples of the sizing unit");
 };
 
-template <typename XT, int TN, int WN, int KS, int BK>
+template <typename XT, int TM, int TN, int WN, int KS, int BK, int ST>
 __global__ void __launch_bounds__(32 * WN * KS)
     router_kernel(const RouterArgs<XT> a) {
-  using S = RouterShape<XT, TN, WN, KS, BK>;
-  constexpr int VEC = S::VEC, EP = S::EP, NT = S::THREADS, XROW = S::XROW;
+  using S = RouterShape<XT, TM, TN, WN, KS, BK, ST>;
+  constexpr int VEC = S::VEC, EP = S::EP, NT = S::THREADS, XROW = S::XROW, BM = S::BM;
   constexpr int QMAX = (EP + 31) / 32;  // experts per lane in the finishing pass
   extern __shared__ __align__(16) unsigned char smem[];
   XT* xs = reinterpret_cast<XT*>(smem);
-  float* wsm = reinterpret_cast<float*>(smem + kStages * S::X_STAGE * sizeof(XT));
+  float* wsm = reinterpret_cast<float*>(smem + ST * S::X_STAGE * sizeof(XT));
   float* lg = reinterpret_cast<float*>(smem);                       // after the k loop
   float* cs = reinterpret_cast<float*>(smem + S::MAIN_BYTES);
 
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int nsplit = (int)cluster.num_blocks();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wn = warp % WN, kg = warp / WN;
   const int T = a.T, d = a.d, E = a.E;
-  const int t_base = blockIdx.x * kBM;
-  const int nchunks = (d + BK - 1) / BK;
+  const int tile = blockIdx.x / nsplit;
+  const int t_base = tile * BM;
+  // This CTA's share of the k chunks.
+  const int total_chunks = (d + BK - 1) / BK;
+  const int per = (total_chunks + nsplit - 1) / nsplit;
+  const int c_begin = min(rank * per, total_chunks);
+  const int nchunks = min(per, total_chunks - c_begin);
 
   // Padding columns e >= E of the W tiles are never loaded: zero them once.
   if (E < EP) {
-    for (int i = tid; i < kStages * S::W_STAGE; i += NT)
-      if (i % EP >= E) wsm[i] = 0.f;
+    for (int i = tid; i < ST * S::W_STAGE; i += NT)
+      if ((i >> 1) % EP >= E) wsm[i] = 0.f;
   }
 
   auto load_stage = [&](int chunk, int stage) {
-    const int k0 = chunk * BK;
+    const int k0 = (c_begin + chunk) * BK;
     XT* xd = xs + stage * S::X_STAGE;
     constexpr int XV = BK / VEC;
-    for (int v = tid; v < kBM * XV; v += NT) {
+    for (int v = tid; v < BM * XV; v += NT) {
       const int r = v / XV, cv = v % XV;
       const int t = t_base + r, kk = k0 + cv * VEC;
       const bool ok = (t < T) && (kk < d);
       cp_async_16(xd + r * XROW + cv * VEC, ok ? (const void*)(a.x + (size_t)t * d + kk) : (const void*)a.x, ok);
     }
+    // W chunk rows k0..k0+BK-1, stored as [k/2][e][k%2] so that one 16-byte
+    // broadcast load gives {W[k][e], W[k+1][e], W[k][e+1], W[k+1][e+1]}.
     float* wd = wsm + stage * S::W_STAGE;
-    if ((E & 3) == 0) {
-      const int EV = E >> 2;
-      for (int v = tid; v < BK * EV; v += NT) {
-        const int r = v / EV, cv = v % EV, kk = k0 + r;
-        const bool ok = kk < d;
-        cp_async_16(wd + r * EP + cv * 4, ok ? (const void*)(a.W + (size_t)kk * E + cv * 4) : (const void*)a.W, ok);
-      }
-    } else {
-      for (int v = tid; v < BK * E; v += NT) {
-        const int r = v / E, c = v % E, kk = k0 + r;
-        const bool ok = kk < d;
-        cp_async_4(wd + r * EP + c, ok ? (const void*)(a.W + (size_t)kk * E + c) : (const void*)a.W, ok);
-      }
+    for (int v = tid; v < BK * E; v += NT) {
+      const int r = v / E, c = v % E, kk = k0 + r;
+      const bool ok = kk < d;
+      cp_async_4(wd + ((r >> 1) * EP + c) * 2 + (r & 1),
+                 ok ? (const void*)(a.W + (size_t)kk * E + c) : (const void*)a.W, ok);
     }
-    cp_async_commit();
   };
 
-  float acc0[TN], acc1[TN];
+  // acc[m][n] holds the even-k and odd-k partial sums of token m, expert n.
+  float2 acc[TM][TN];
 #pragma unroll
-  for (int n = 0; n < TN; ++n) acc0[n] = acc1[n] = 0.f;
+  for (int m = 0; m < TM; ++m)
+#pragma unroll
+    for (int n = 0; n < TN; ++n) acc[m][n] = make_float2(0.f, 0.f);
 
-  if (nchunks > 0) load_stage(0, 0);
+  // Prologue: ST - 1 chunks in flight (one commit group per chunk; empty
+  // groups past the end keep the group count uniform).
+#pragma unroll
+  for (int st = 0; st < ST - 1; ++st) {
+    if (st < nchunks) load_stage(st, st);
+    cp_async_commit();
+  }
   for (int chunk = 0; chunk < nchunks; ++chunk) {
-    if (chunk + 1 < nchunks) {
-      load_stage(chunk + 1, (chunk + 1) % kStages);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int stage = chunk % kStages;
+    cp_async_wait<ST - 2>();   // chunk `chunk` has landed
+    __syncthreads();           // ... for every thread; stage (chunk-1)%ST is free
+    const int nxt = chunk + ST - 1;
+    if (nxt < nchunks) load_stage(nxt, nxt % ST);
+    cp_async_commit();
+    const int stage = chunk % ST;
     const XT* xa = xs + stage * S::X_STAGE + lane * XROW;
-    const XT* xb = xa + 32 * XROW;
-    const float* wb = wsm + stage * S::W_STAGE + wn * TN;
+    const float* wb = wsm + stage * S::W_STAGE + wn * TN * 2;
 #pragma unroll
     for (int kv = kg * (BK / KS); kv < (kg + 1) * (BK / KS); kv += VEC) {
-      float x0[VEC], x1[VEC];
-      XVec<XT>::load(xa + kv, x0);
-      XVec<XT>::load(xb + kv, x1);
+      float2 xp[TM][VEC / 2];
 #pragma unroll
-      for (int u = 0; u < VEC; ++u) {
-        const float4* wr = reinterpret_cast<const float4*>(wb + (kv + u) * EP);
+      for (int m = 0; m < TM; ++m) XVec<XT>::load(xa + m * 32 * XROW + kv, xp[m]);
 #pragma unroll
-        for (int q = 0; q < TN / 4; ++q) {
+      for (int pi = 0; pi < VEC / 2; ++pi) {
+        const float4* wr = reinterpret_cast<const float4*>(wb + ((kv >> 1) + pi) * EP * 2);
+#pragma unroll
+        for (int q = 0; q < TN / 2; ++q) {
           const float4 w = wr[q];
-          acc0[4 * q + 0] = fmaf(x0[u], w.x, acc0[4 * q + 0]);
-          acc0[4 * q + 1] = fmaf(x0[u], w.y, acc0[4 * q + 1]);
-          acc0[4 * q + 2] = fmaf(x0[u], w.z, acc0[4 * q + 2]);
-          acc0[4 * q + 3] = fmaf(x0[u], w.w, acc0[4 * q + 3]);
-          acc1[4 * q + 0] = fmaf(x1[u], w.x, acc1[4 * q + 0]);
-          acc1[4 * q + 1] = fmaf(x1[u], w.y, acc1[4 * q + 1]);
-          acc1[4 * q + 2] = fmaf(x1[u], w.z, acc1[4 * q + 2]);
-          acc1[4 * q + 3] = fmaf(x1[u], w.w, acc1[4 * q + 3]);
+          const float2 w0 = make_float2(w.x, w.y), w1 = make_float2(w.z, w.w);
+#pragma unroll
+          for (int m = 0; m < TM; ++m) {
+            acc[m][2 * q] = __ffma2_rn(xp[m][pi], w0, acc[m][2 * q]);
+            acc[m][2 * q + 1] = __ffma2_rn(xp[m][pi], w1, acc[m][2 * q + 1]);
+          }
         }
       }
     }
-    __syncthreads();
   }
+  cp_async_wait<0>();
+  __syncthreads();
 
-  // Partial logits of each k group -> shared memory, then a fixed-order sum.
-  {
-    float* p0 = lg + (kg * kBM + lane) * EP + wn * TN;
-    float* p1 = p0 + 32 * EP;
+  // This CTA's partial logits: per k group to shared memory, then a
+  // fixed-order sum over the groups into lg[BM][EP].
 #pragma unroll
-    for (int n = 0; n < TN; ++n) {
-      p0[n] = acc0[n];
-      p1[n] = acc1[n];
-    }
+  for (int m = 0; m < TM; ++m) {
+    float* p = lg + (kg * BM + m * 32 + lane) * EP + wn * TN;
+#pragma unroll
+    for (int n = 0; n < TN; ++n) p[n] = acc[m][n].x + acc[m][n].y;
   }
   __syncthreads();
   if (KS > 1) {
-    for (int i = tid; i < kBM * EP; i += NT) {
-      float s = lg[i];
+    for (int i = tid; i < BM * EP; i += NT) {
+      float v = lg[i];
 #pragma unroll
-      for (int g = 1; g < KS; ++g) s += lg[g * kBM * EP + i];
-      lg[i] = s;
+      for (int g = 1; g < KS; ++g) v += lg[g * BM * EP + i];
+      lg[i] = v;
     }
-    __syncthreads();
   }
+  cluster.sync();  // every CTA's partial tile is complete and visible
 
-  // One warp per token: bias, noise, softmax, top-k, gates, column sums.
+  // Finishing pass: token r of the tile is finished by CTA r % nsplit, one
+  // warp per token; the logits are the rank-ordered sum of the partials.
   constexpr int NW = WN * KS;
   float colsum[QMAX];
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) colsum[q] = 0.f;
   const int k = a.k;
-  for (int r = warp; r < kBM; r += NW) {
+  for (int r = rank + nsplit * warp; r < BM; r += nsplit * NW) {
     const int t = t_base + r;
     if (t >= T) break;
     float L[QMAX];
@@ -235,7 +256,8 @@ __global__ void __launch_bounds__(32 * WN * KS)
       const int e = lane + 32 * q;
       float v = -INFINITY;
       if (e < E) {
-        v = lg[r * EP + e];
+        v = 0.f;
+        for (int sp = 0; sp < nsplit; ++sp) v += cluster.map_shared_rank(lg, sp)[r * EP + e];
         if (a.bias != nullptr) v = __fadd_rn(v, a.bias[e]);
         if (a.noise != nullptr) v = __fadd_rn(v, a.noise[(size_t)t * E + e]);
         if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = v;
@@ -246,16 +268,16 @@ __global__ void __launch_bounds__(32 * WN * KS)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float p[QMAX];
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
     for (int q = 0; q < QMAX; ++q) {
       p[q] = (lane + 32 * q < E) ? expf(L[q] - m) : 0.f;
-      s += p[q];
+      sum += p[q];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
 #pragma unroll
-    for (int q = 0; q < QMAX; ++q) colsum[q] += p[q] / s;
+    for (int q = 0; q < QMAX; ++q) colsum[q] += p[q] / sum;
 
     // Top-k over packed keys: (order-preserving logit bits) << 32 | ~e.
     uint64_t key[QMAX];
@@ -304,48 +326,93 @@ __global__ void __launch_bounds__(32 * WN * KS)
     }
   }
 
-  // Column sums of probs: per warp -> shared -> fixed-order sum over warps.
+  // Column sums of probs: per warp -> own shared memory; then CTA 0 adds
+  // them over ranks and warps in a fixed order into this tile's row.
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int e = lane + 32 * q;
     if (e < EP) cs[warp * EP + e] = colsum[q];
   }
+  cluster.sync();
+  if (rank == 0) {
+    for (int e = tid; e < E; e += NT) {
+      float v = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float* pcs = cluster.map_shared_rank(cs, sp);
+        for (int w = 0; w < NW; ++w) v += pcs[w * EP + e];
+      }
+      a.part[(size_t)tile * E + e] = v;
+    }
+  }
+  cluster.sync();  // peers keep their shared memory until CTA 0 has read it
+}
+
+// P_e = (sum over token tiles of the column-sum rows, in fp64) / T.  Each
+// thread adds a fixed strided subset of rows in increasing order, then the
+// subsets are added in increasing order.
+__global__ void __launch_bounds__(256)
+    prob_mean_kernel(const float* __restrict__ part, int nrows, int E, int T,
+                     float* __restrict__ prob_mean) {
+  __shared__ double acc[256];
+  const int groups = max(1, (int)blockDim.x / E);   // threads per expert
+  const int e = threadIdx.x % E, g = threadIdx.x / E;
+  double v = 0.0;
+  if (g < groups)
+    for (int b = g; b < nrows; b += groups) v += (double)part[(size_t)b * E + e];
+  acc[threadIdx.x] = v;
   __syncthreads();
-  for (int e = tid; e < E; e += NT) {
-    float s = 0.f;
-    for (int w = 0; w < NW; ++w) s += cs[w * EP + e];
-    a.part[(size_t)blockIdx.x * E + e] = s;
-  }
-}
-
-// P_e = (sum over router CTAs of the partial column sums, in fp64) / T.
-__global__ void prob_mean_kernel(const float* __restrict__ part, int nblocks, int E, int T,
-                                 float* __restrict__ prob_mean) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  for (int ee = threadIdx.x; ee < E; ee += blockDim.x) {
     double s = 0.0;
-    for (int b = 0; b < nblocks; ++b) s += (double)part[(size_t)b * E + e];
-    prob_mean[e] = T > 0 ? (float)(s / (double)T) : 0.f;
+    for (int gg = 0; gg < groups; ++gg)
+      if (gg * E + ee < (int)blockDim.x) s += acc[gg * E + ee];
+    prob_mean[ee] = T > 0 ? (float)(s / (double)T) : 0.f;
   }
 }
 
-template <typename XT, int TN, int WN, int KS, int BK>
-cudaError_t run_router(const RouterArgs<XT>& a, int nblocks, cudaStream_t s) {
-  using S = RouterShape<XT, TN, WN, KS, BK>;
-  auto kern = router_kernel<XT, TN, WN, KS, BK>;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
-  if (e != cudaSuccess) return e;
-  kern<<<nblocks, S::THREADS, S::SMEM, s>>>(a);
-  return cudaGetLastError();
+// Clusters of nsplit CTAs per token tile: enough CTAs to fill the GPU about
+// four times over, at most 8 per cluster and at most one k chunk each.
+int router_splits(int tiles, int chunks) {
+  const int target = 4 * device_sm_count();
+  int s = 1;
+  while (s < 8 && tiles * s < target && s * 2 <= chunks) s *= 2;
+  return s;
 }
 
+template <typename XT, int TM, int TN, int WN, int KS, int BK, int ST>
+cudaError_t run_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles_out) {
+  using S = RouterShape<XT, TM, TN, WN, KS, BK, ST>;
+  auto kern = router_kernel<XT, TM, TN, WN, KS, BK, ST>;
+  const int tiles = ceil_div(a.T, S::BM);
+  const int nsplit = router_splits(tiles, ceil_div(a.d, BK));
+  *tiles_out = tiles;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), S::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * nsplit), 1, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)nsplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Two tokens per lane everywhere (each W broadcast feeds two packed FMAs);
+// small E keeps 3 chunks in flight to stream x, large E narrows the chunk to
+// bound shared memory.
 template <typename XT>
-cudaError_t dispatch_router(const RouterArgs<XT>& a, int nblocks, cudaStream_t s) {
-  if (a.E <= 8) return run_router<XT, 8, 1, 4, 64>(a, nblocks, s);
-  if (a.E <= 16) return run_router<XT, 16, 1, 4, 64>(a, nblocks, s);
-  if (a.E <= 32) return run_router<XT, 16, 2, 2, 64>(a, nblocks, s);
-  if (a.E <= 64) return run_router<XT, 16, 4, 2, 64>(a, nblocks, s);
-  if (a.E <= 128) return run_router<XT, 16, 8, 1, 32>(a, nblocks, s);
-  return run_router<XT, 16, 16, 1, 32>(a, nblocks, s);
+cudaError_t dispatch_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles) {
+  if (a.E <= 8) return run_router<XT, 2, 8, 1, 4, 64, 4>(a, s, tiles);
+  if (a.E <= 16) return run_router<XT, 2, 16, 1, 4, 64, 4>(a, s, tiles);
+  if (a.E <= 32) return run_router<XT, 2, 16, 2, 2, 64, 3>(a, s, tiles);
+  if (a.E <= 64) return run_router<XT, 2, 16, 4, 2, 64, 3>(a, s, tiles);
+  if (a.E <= 128) return run_router<XT, 2, 16, 8, 1, 32, 2>(a, s, tiles);
+  return run_router<XT, 1, 16, 16, 1, 32, 2>(a, s, tiles);  // 512 threads: 128 regs each
 }
 
 }  // namespace
@@ -354,21 +421,21 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_ro
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
                          cudaStream_t s) {
-  const int nblocks = ceil_div(c.T, kRouterTokens);
-  if (nblocks > 0) {
+  int tiles = 0;  // token tiles; each writes one row of router_part
+  if (c.T > 0) {
     cudaError_t e;
     if (c.act_dtype == MOE_BF16) {
       RouterArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
                                   gates, logits_out, router_part, c.T, c.d, c.E, c.top_k};
-      e = dispatch_router(a, nblocks, s);
+      e = dispatch_router(a, s, &tiles);
     } else {
       RouterArgs<float> a{static_cast<const float*>(x), W_router, bias, noise, idx,
                           gates, logits_out, router_part, c.T, c.d, c.E, c.top_k};
-      e = dispatch_router(a, nblocks, s);
+      e = dispatch_router(a, s, &tiles);
     }
     if (e != cudaSuccess) return e;
   }
-  prob_mean_kernel<<<1, 256, 0, s>>>(router_part, nblocks, c.E, c.T, prob_mean);
+  prob_mean_kernel<<<1, 256, 0, s>>>(router_part, tiles, c.E, c.T, prob_mean);
   return cudaGetLastError();
 }
 

@@ -30,3 +30,12 @@ def test_pfd_mixtral_expert_params(golden_dir):
     assert one * g["top_k"] * g["layers"] == g["active_expert_params"]
     # bytes of one layer's bf16 expert weights (all 8 used)
     assert A.expert_weight_bytes(8, 4096, 14336, 4096, "swiglu", 2) == 8 * one * 2
+
+
+def test_kept_rows_apply_the_capacity():
+    """The capacity table of 'Switch: top-1, one loss, and a rate limit':
+    64 tokens, 8 experts, top-1, counts 12,6,1,10,8,11,14,2 -> 15/7/0 dropped."""
+    counts = [12, 6, 1, 10, 8, 11, 14, 2]
+    for cf, dropped in ((1.0, 15), (1.25, 7), (2.0, 0)):
+        assert A.kept_rows(counts, cf, 64, 1) == 64 - dropped
+    assert A.kept_rows(counts, 0.0, 64, 1) == 64

@@ -52,8 +52,8 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
 
 
 def test_route_noalloc_rejects_calls_beyond_its_scratch():
-    # ceil(T/64) * E = 1025 * 64 floats > 65536
-    cfg = api.make_config(1025 * 64, 64, 64, 64, 64, 2, "swiglu", "bf16")
+    # ceil(T/32) * E = 1025 * 64 floats > 65536
+    cfg = api.make_config(1025 * 32, 64, 64, 64, 64, 2, "swiglu", "bf16")
     lib = api.load_library()
     buf = torch.empty(16, device="cuda")
     p = buf.data_ptr()
