@@ -100,6 +100,7 @@ struct TileCoord {
   int e, m0, rows, n_tile;
 };
 
+template <int TILE_M = BM>
 __device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, const int* row_off,
                                                  int E, int n_tiles) {
   int lo = 0, hi = E;  // prefix[lo] <= tile < prefix[hi]
@@ -112,12 +113,90 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, co
   TileCoord c;
   c.e = lo;
   c.n_tile = local / mt;
-  c.m0 = row_off[lo] + (local % mt) * BM;
-  c.rows = min(BM, row_off[lo + 1] - c.m0);
+  c.m0 = row_off[lo] + (local % mt) * TILE_M;
+  c.rows = min(TILE_M, row_off[lo + 1] - c.m0);
   return c;
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+// Epilogue of one accumulator row held by this thread (TMEM lane = tile row):
+// reads the 256 accumulator columns in chunks of 32 and writes the row's
+// output columns [n0, n0 + OUT_COLS) of `out` (row offset orow_off), masked to
+// N.  Every lane of the warp executes the tensor-memory loads (they are
+// warp-collective); only rows with `valid` store.
+template <int EPI>
+__device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
+                                                const GemmArgs& g) {
+  constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  if (EPI == kEpiSwiglu) {
+#pragma unroll 1
+    for (int cc = 0; cc < OUT_COLS; cc += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_ld_32x32b_x32(tacc + cc, gr);
+      tmem_ld_32x32b_x32(tacc + OUT_COLS + cc, ur);
+      tmem_ld_wait();
+      if (valid) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+          const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+          pk[i] = pack_bf16x2(h0, h1);
+        }
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int col = n0 + cc + v * 8;
+          if (col < g.N)
+            *reinterpret_cast<uint4*>(orow + col) =
+                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  } else if (EPI == kEpiNone) {
+#pragma unroll 1
+    for (int cc = 0; cc < OUT_COLS; cc += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tacc + cc, r);
+      tmem_ld_wait();
+      if (valid) {
+        float* orow = static_cast<float*>(g.out) + orow_off;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int col = n0 + cc + v * 4;
+          if (col < g.N)
+            *reinterpret_cast<uint4*>(orow + col) =
+                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int cc = 0; cc < OUT_COLS; cc += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tacc + cc, r);
+      tmem_ld_wait();
+      if (valid) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float v0 = fmaxf(__uint_as_float(r[2 * i]), 0.f);
+          const float v1 = fmaxf(__uint_as_float(r[2 * i + 1]), 0.f);
+          pk[i] = pack_bf16x2(v0, v1);
+        }
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int col = n0 + cc + v * 8;
+          if (col < g.N)
+            *reinterpret_cast<uint4*>(orow + col) =
+                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  }
+}
 
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -291,73 +370,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
       const size_t orow_off = (size_t)(c.m0 + (valid ? row : 0)) * g.N;
-      if (EPI == kEpiSwiglu) {
-#pragma unroll 1
-        for (int cc = 0; cc < OUT_COLS; cc += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld_32x32b_x32(tacc + cc, gr);
-          tmem_ld_32x32b_x32(tacc + OUT_COLS + cc, ur);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
-              const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
-            }
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = n0 + cc + v * 8;
-              if (col < g.N)
-                *reinterpret_cast<uint4*>(orow + col) =
-                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-            }
-          }
-        }
-      } else if (EPI == kEpiNone) {
-#pragma unroll 1
-        for (int cc = 0; cc < OUT_COLS; cc += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tacc + cc, r);
-          tmem_ld_wait();
-          if (valid) {
-            float* orow = static_cast<float*>(g.out) + orow_off;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const int col = n0 + cc + v * 4;
-              if (col < g.N)
-                *reinterpret_cast<uint4*>(orow + col) =
-                    make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int cc = 0; cc < OUT_COLS; cc += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tacc + cc, r);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float v0 = fmaxf(__uint_as_float(r[2 * i]), 0.f);
-              const float v1 = fmaxf(__uint_as_float(r[2 * i + 1]), 0.f);
-              pk[i] = pack_bf16x2(v0, v1);
-            }
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = n0 + cc + v * 8;
-              if (col < g.N)
-                *reinterpret_cast<uint4*>(orow + col) =
-                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-            }
-          }
-        }
-      }
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[acc]);
       acc ^= 1;
@@ -371,6 +384,218 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2): a cluster of two CTAs computes a tile of
+// 256 rows x 256 accumulator columns.  Each CTA stages its own 128 rows of A
+// and one half of B (128 columns: the gate half and the up half for SwiGLU,
+// or the two column halves otherwise) per 64-wide k block, 32 KiB per stage
+// and 6 stages; the leader CTA's single MMA thread issues
+// tcgen05.mma.cta_group::2 (M256 N256 K16), which reads both CTAs' shared
+// memory and writes each CTA's 128 accumulator rows into its own tensor
+// memory.  Per CTA this moves two thirds of the bytes of the single-CTA tile
+// for the same FLOPs.  Both CTAs' copies count their bytes on the leader's
+// full barrier; the leader's commits are multicast to both CTAs' empty and
+// accumulator-full barriers; both CTAs' epilogue warps release an
+// accumulator by arriving on the leader's barrier.  No load is multicast.
+// ---------------------------------------------------------------------------
+
+constexpr int PBM = 2 * BM;                       // rows per pair tile
+constexpr int P_STAGES = 6;
+constexpr int P_STAGE_BYTES = A_STAGE + B_STAGE / 2;  // 32 KiB
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES;
+constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+  constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + P_STAGES;
+  uint64_t* tfull_bar = empty_bar + P_STAGES;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  int* tile_prefix = reinterpret_cast<int*>(tmem_holder + 4);  // MAX_E + 1
+  int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = g.E;
+  const uint32_t rank = cluster_cta_rank();   // 0 = leader, 1 = peer
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    for (int e = lane; e <= E; e += 32) row_off[e] = g.offsets[e];
+    __syncwarp();
+    bool ok = true;
+    for (int e = lane; e < E; e += 32) ok = ok && (row_off[e] <= row_off[e + 1]);
+    if (lane == 0) ok = ok && row_off[0] == 0 && row_off[E] <= g.rows_max;
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && lane == 0 && blockIdx.x == 0) report_error(g.err, kDevBadOffsets);
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int mt = (ok && e < E) ? (row_off[e + 1] - row_off[e] + PBM - 1) / PBM : 0;
+      int incl = mt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (e < E) tile_prefix[e + 1] = (carry + incl) * g.n_tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      tile_prefix[0] = 0;
+      tma_prefetch_map(&tmA);
+      tma_prefetch_map(&tmB0);
+      tma_prefetch_map(&tmB1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  } else if (warp == 2 && lane == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 8);  // one arrive per epilogue warp of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before_sync();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total_tiles = tile_prefix[E];
+  const int num_kb = (g.K + BK - 1) / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer (both)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, last_phase = 0;
+    bool alive = true;
+    const CUtensorMap* bmap = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
+    for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
+      const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
+      const int n0 = c.n_tile * OUT_COLS;
+      // this CTA's B half: gate / up for SwiGLU, else the column halves
+      const int nb = (EPI == kEpiSwiglu) ? n0 : n0 + (int)rank * (BN / 2);
+      const int my_m = c.m0 + (int)rank * BM;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+          report_error(g.err, kDevTimeoutProducer);
+          alive = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * P_STAGE_BYTES;
+        uint8_t* sb = sa + A_STAGE;
+        const int k0 = kb * BK;
+        if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
+        tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m);
+        tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e);
+        tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e);
+        issued_mask |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Drain: the leader's full barriers count both CTAs' copies.
+    if (rank == 0)
+      for (int s = 0; s < P_STAGES; ++s)
+        if ((issued_mask >> s) & 1u)
+          if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(g.err, kDevTimeoutDrain);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ MMA issuer (leader)
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool alive = true;
+    for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
+      if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u)) {
+        report_error(g.err, kDevTimeoutMma);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase)) {
+          report_error(g.err, kDevTimeoutMma);
+          alive = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sa = smem_u32(smem + stage * P_STAGE_BYTES);
+        const uint32_t sb = sa + A_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < BK / UK; ++kk) {
+          umma_bf16_ss_pair(d_tmem, desc_a_kmajor(sa + kk * UK * 2),
+                            desc_b_nmajor(sb + kk * UK * 128), kIdescPair,
+                            (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!alive) break;
+      umma_commit_pair(&tfull_bar[acc], 0x3);  // accumulator ready in both CTAs
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    umma_commit_pair(drain_bar, 0x1);
+    if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
+  } else if (warp >= 2) {
+    // ------------------------------------------------ epilogue (both)
+    const int q = warp & 3;
+    const int row = (int)rank * BM + q * 32 + lane;  // row inside the pair tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs) {
+      const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
+      const int n0 = c.n_tile * OUT_COLS;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase)) {
+        report_error(g.err, kDevTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const bool valid = row < c.rows;
+      const size_t orow_off = (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // ---- teardown: both CTAs done with tensor memory and shared memory
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -421,6 +646,27 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
   return cudaGetLastError();
 }
 
+template <int EPI>
+cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                          const GemmArgs& g, int pairs, cudaStream_t s) {
+  auto kern = grouped_gemm_pair_kernel<EPI>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), P_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, g);
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
@@ -443,6 +689,18 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   g.N = N;
   g.rows_max = rows_max;
   g.n_tiles = ceil_div(N, out_cols);
+  // Expert groups of 1024 rows or more on average: CTA pairs (M = 256 tiles,
+  // a third less traffic per CTA); smaller groups: single CTAs (M = 128
+  // tiles waste fewer rows at group edges).
+  if (rows_max >= 1024 * E) {
+    const long max_pairs = (long)(ceil_div(rows_max, PBM) + E) * g.n_tiles;
+    const int pairs = (int)std::min<long>((long)(device_sm_count() / 2), max_pairs);
+    switch (epi) {
+      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu>(ta, tb0, tb1, g, pairs, s);
+      case kEpiRelu: return run_gemm_pair<kEpiRelu>(ta, tb0, tb1, g, pairs, s);
+      default: return run_gemm_pair<kEpiNone>(ta, tb0, tb1, g, pairs, s);
+    }
+  }
   const long max_tiles = (long)(ceil_div(rows_max, BM) + E) * g.n_tiles;
   const int grid = (int)std::min<long>((long)device_sm_count(), max_tiles);
   switch (epi) {

@@ -138,3 +138,37 @@ def test_bad_offsets_are_reported_not_used():
     torch.cuda.synchronize()
     assert api.moe_device_status(ws) == 2            # kDevBadOffsets
     assert (host(y) == 0).all()
+
+
+# Groups averaging 1024 rows or more run on CTA pairs (cta_group::2, 256-row
+# tiles); these shapes put the pair kernel through ragged groups, 1-row
+# groups, and ragged K and N.
+PAIR_CASES = [([1500, 700], 2200, 256, 384, 200),
+              ([0, 1, 2049, 2050], 4100, 200, 256, 256),
+              ([2048], 2048, 512, 1024, 512)]
+
+
+@pytest.mark.parametrize("kind", ["relu", "swiglu"])
+@pytest.mark.parametrize("sizes,T_k,d,h,d_out", PAIR_CASES)
+def test_grouped_ffn_bf16_cta_pairs(kind, sizes, T_k, d, h, d_out):
+    cfg, x_perm, offsets, weights = make_case(kind, "bf16", d, h, d_out, sizes, T_k, seed=T_k + d)
+    assert cfg.T * cfg.top_k >= 1024 * cfg.E
+    y = run_ffn(cfg, x_perm, offsets, weights["W_in"], weights["W_up"], weights["W_out"])
+    compare_bf16(y, oracle_rows(kind, "bf16", x_perm, offsets, weights), offsets)
+    assert np.isnan(y[int(offsets[-1]):]).all()
+
+
+def test_grouped_ffn_cta_pairs_exact_small_integers():
+    """The exact-arithmetic check of the operand layouts, on the pair kernel."""
+    d, h, d_out, R = 128, 512, 256, 2100
+    rng = np.random.default_rng(1)
+    x = rng.integers(-2, 3, size=(R, d)).astype(np.float32)
+    W1 = rng.integers(-1, 2, size=(1, d, h)).astype(np.float32)
+    W2 = rng.integers(-1, 2, size=(1, h, d_out)).astype(np.float32) / 8
+    cfg = api.make_config(R, d, h, d_out, 1, 1, "relu", "bf16")
+    offsets = np.array([0, R], np.int32)
+    y = run_ffn(cfg, f32_to_bf16_bits(x), offsets, f32_to_bf16_bits(W1), None,
+                f32_to_bf16_bits(W2))
+    ref = O.expert_forward("relu", x.astype(np.float64), W1[0].astype(np.float64), None,
+                           W2[0].astype(np.float64))
+    assert np.array_equal(y[:R].astype(np.float64), ref)
