@@ -347,6 +347,7 @@ def run_ours(args, rank, world):
     gemm = {"bound": "tensor", "achieved": flops / t_exp / 1e12, "peak": tensor_peak,
             "unit": "TFLOP/s", "frac": flops / t_exp / 1e12 / tensor_peak,
             "traffic": profiled_traffic("grouped_gemm.cu", "grouped_gemm_mixtral.md"),
+            "traffic_note": "DRAM bytes of both launches of one step (ncu), same unit as achieved",
             "kernel": "grouped_gemm_kernel (2 launches per step: up-projection with fused SwiGLU, "
                       "down-projection); achieved = algorithmic FLOPs of both / their summed time",
             "peak_source": f"{peak_src} burst bf16 (cuBLAS)"}

@@ -34,6 +34,9 @@
 //  * Tile order: expert-major, then output-column block, then row block, with
 //    CTAs striding through it: CTAs running together share one weight column
 //    block (read from HBM once, reused from L2) across the expert's row blocks.
+//    Row tiles are re-read for every column block, so they are loaded with an
+//    evict-last L2 policy; weights keep the normal policy (an evict-first
+//    policy on them made CTAs that share a weight block re-read it from HBM).
 //  * A tile that straddles two experts' rows reads the next expert's rows,
 //    computes them, and masks them at the store: no padding of the grouped
 //    layout is needed.
@@ -275,6 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
+    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal();
     for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
       const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
@@ -288,16 +292,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint8_t* sb = sa + A_STAGE;
         const int k0 = kb * BK;
         mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-        tma_load_2d(sa, &tmA, &full_bar[stage], k0, c.m0);
+        tma_load_2d_hint(sa, &tmA, &full_bar[stage], k0, c.m0, keep);
         if (EPI == kEpiSwiglu) {
-          tma_load_3d(sb, &tmB0, &full_bar[stage], n0, k0, c.e);
-          tma_load_3d(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e);
-          tma_load_3d(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e);
-          tma_load_3d(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e);
+          tma_load_3d_hint(sb, &tmB0, &full_bar[stage], n0, k0, c.e, stream);
+          tma_load_3d_hint(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e, stream);
+          tma_load_3d_hint(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e, stream);
+          tma_load_3d_hint(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e, stream);
         } else {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            tma_load_3d(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e);
+            tma_load_3d_hint(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e, stream);
         }
         issued_mask |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -489,6 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
     const CUtensorMap* bmap = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
+    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal();
     for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
       const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
@@ -505,9 +510,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint8_t* sb = sa + A_STAGE;
         const int k0 = kb * BK;
         if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-        tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m);
-        tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e);
-        tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e);
+        tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, keep);
+        tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, stream);
+        tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, stream);
         issued_mask |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == P_STAGES) {
