@@ -117,6 +117,7 @@ struct RouterShape {
   static_assert((BK / KS) % VEC == 0, "k split must hold whole vectors");
   static_assert(TN % 4 == 0, "experts per lane must be a multiple of 4");
   static_assert(BK % 2 == 0, "k is consumed in pairs");
+  static_assert((EP & (EP - 1)) == 0, "the padded expert width is a power of two");
   static_assert(BM % kRouterTokens == 0, "CTA tiles are whole multiples of the sizing unit");
 };
 
@@ -164,12 +165,18 @@ __global__ void __launch_bounds__(32 * WN * KS)
     }
     // W chunk rows k0..k0+BK-1, stored as [k/2][e][k%2] so that one 16-byte
     // broadcast load gives {W[k][e], W[k+1][e], W[k][e+1], W[k+1][e+1]}.
+    // Indexed by the compile-time padded width EP (a power of two), so no
+    // integer division by the runtime E; columns e >= E are skipped and keep
+    // their zeros.
     float* wd = wsm + stage * S::W_STAGE;
-    for (int v = tid; v < BK * E; v += NT) {
-      const int r = v / E, c = v % E, kk = k0 + r;
-      const bool ok = kk < d;
-      cp_async_4(wd + ((r >> 1) * EP + c) * 2 + (r & 1),
-                 ok ? (const void*)(a.W + (size_t)kk * E + c) : (const void*)a.W, ok);
+#pragma unroll 4
+    for (int v = tid; v < BK * EP; v += NT) {
+      const int r = v / EP, c = v % EP, kk = k0 + r;
+      if (c < E) {
+        const bool ok = kk < d;
+        cp_async_4(wd + ((r >> 1) * EP + c) * 2 + (r & 1),
+                   ok ? (const void*)(a.W + (size_t)kk * E + c) : (const void*)a.W, ok);
+      }
     }
   };
 
@@ -408,10 +415,10 @@ cudaError_t run_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles_out) 
 template <typename XT>
 cudaError_t dispatch_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles) {
   if (a.E <= 8) return run_router<XT, 2, 8, 1, 4, 64, 4>(a, s, tiles);
-  if (a.E <= 16) return run_router<XT, 2, 16, 1, 4, 64, 4>(a, s, tiles);
-  if (a.E <= 32) return run_router<XT, 2, 16, 2, 2, 64, 3>(a, s, tiles);
-  if (a.E <= 64) return run_router<XT, 2, 16, 4, 2, 64, 3>(a, s, tiles);
-  if (a.E <= 128) return run_router<XT, 2, 16, 8, 1, 32, 2>(a, s, tiles);
+  if (a.E <= 16) return run_router<XT, 2, 8, 2, 2, 64, 4>(a, s, tiles);
+  if (a.E <= 32) return run_router<XT, 2, 8, 4, 2, 64, 3>(a, s, tiles);
+  if (a.E <= 64) return run_router<XT, 2, 8, 8, 1, 64, 2>(a, s, tiles);
+  if (a.E <= 128) return run_router<XT, 2, 8, 16, 1, 32, 2>(a, s, tiles);
   return run_router<XT, 1, 16, 16, 1, 32, 2>(a, s, tiles);  // 512 threads: 128 regs each
 }
 
