@@ -255,22 +255,25 @@ def run_ours(args, rank, world):
     ws = layer.ws
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def step(ev=None, marks=(0, 1, 2, 3, 4)):
+        # ev[j] is recorded before stage j (route, dispatch, experts, combine)
+        # and ev[4] after the last, for the stage indices listed in `marks`.
+        # Every recorded event separates two launches that could otherwise
+        # overlap (each kernel is launched as a programmatic dependent of the
+        # one before), so the timed loop marks only the expert stage.
+        def mark(j):
+            if ev is not None and j in marks:
+                ev[j].record(stream)
+        mark(0)
         api.moe_route(cfg, x, Wr, bias, noise, o.expert_indices, o.gates, P, None, ws)
-        if ev is not None:
-            ev[1].record(stream)
+        mark(1)
         api.moe_dispatch(cfg, x, o.expert_indices, P, o.counts, offsets, dest, perm, o.drop_mask,
                          f, o.aux_loss, x_perm, ws)
-        if ev is not None:
-            ev[2].record(stream)
+        mark(2)
         api.moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws)
-        if ev is not None:
-            ev[3].record(stream)
+        mark(3)
         api.moe_combine(cfg, y_perm, dest, o.gates, o.output)
-        if ev is not None:
-            ev[4].record(stream)
+        mark(4)
 
     def barrier():
         if world > 1:
@@ -292,11 +295,19 @@ def run_ours(args, rank, world):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(evs[i], marks=(2, 3))
     end.record(stream)
     barrier()
     elapsed_ms = start.elapsed_time(end)
+    expert_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+
+    # Stage breakdown (diagnostic, outside the timed region): the same steps
+    # again with an event between every two stages.
+    for i in range(args.steps):
+        step(evs[i])
+    barrier()
     stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(4)]
+    stage_ms[2] = expert_ms
 
     # End to end through the public call (moe_forward): every step copies its
     # tokens from pinned host memory and its output and aux_loss back to pinned
@@ -367,14 +378,21 @@ def run_ours(args, rank, world):
     value = job_value(world, T, ms_step)
     flops = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
     t_exp = stage_ms[2] / 1e3
-    tensor_peak = peaks["bf16_tflops"]
+    # The GEMMs run back to back for the whole timed loop (seconds at the power
+    # cap), so the sustained cuBLAS figure is the denominator; the burst
+    # fraction is given beside it.
+    tensor_peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    burst_peak = peaks["bf16_tflops"]
     gemm = {"bound": "tensor", "achieved": flops / t_exp / 1e12, "peak": tensor_peak,
             "unit": "TFLOP/s", "frac": flops / t_exp / 1e12 / tensor_peak,
+            "frac_of_burst": flops / t_exp / 1e12 / burst_peak,
             "traffic": profiled_traffic("grouped_gemm.cu", "grouped_gemm_mixtral.md"),
             "traffic_note": "DRAM bytes of both launches of one step (ncu), same unit as achieved",
             "kernel": "grouped_gemm_kernel (2 launches per step: up-projection with fused SwiGLU, "
                       "down-projection); achieved = algorithmic FLOPs of both / their summed time",
-            "peak_source": f"{peak_src} burst bf16 (cuBLAS)"}
+            "peak_source": (f"{peak_src} sustained bf16 (cuBLAS back to back for 4 s)"
+                            if peaks.get("bf16_tflops_sustained") else
+                            f"{peak_src} burst bf16 (cuBLAS)")}
     hbm = peaks["hbm_gbs"]
     rb = A.router_bytes(T, w.d, E, k, 2, w.noise)
     pb = A.permute_bytes(T, rows, w.d, 2)
@@ -385,6 +403,8 @@ def run_ours(args, rank, world):
         "experts": {"ms": stage_ms[2], "TFLOP/s": flops / t_exp / 1e12,
                     "frac_tensor": flops / t_exp / 1e12 / tensor_peak},
         "combine": {"ms": stage_ms[3], "GB/s": cb / stage_ms[3] / 1e6, "frac_hbm": cb / stage_ms[3] / 1e6 / hbm},
+        "note": "experts: events inside the timed loop; route, dispatch, combine: a second "
+                "pass of the same steps with an event between every two stages",
     }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,

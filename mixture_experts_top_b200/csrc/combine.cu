@@ -32,6 +32,7 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ y_perm, const int32_t* __restrict__ dest,
                    const float* __restrict__ gates, OutT* __restrict__ out, int T, int k,
                    int d_out) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -83,12 +84,10 @@ cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int
   if (c.T == 0) return cudaSuccess;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
   if (c.act_dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        y_perm, dest, gates, static_cast<__nv_bfloat16*>(out), c.T, c.top_k, c.d_out);
-  else
-    combine_kernel<float><<<blocks, 256, 0, s>>>(y_perm, dest, gates, static_cast<float*>(out),
-                                                 c.T, c.top_k, c.d_out);
-  return cudaGetLastError();
+    return launch_kernel(combine_kernel<__nv_bfloat16>, blocks, 256, 0, s, 0, y_perm, dest, gates,
+                         static_cast<__nv_bfloat16*>(out), c.T, c.top_k, c.d_out);
+  return launch_kernel(combine_kernel<float>, blocks, 256, 0, s, 0, y_perm, dest, gates,
+                       static_cast<float*>(out), c.T, c.top_k, c.d_out);
 }
 
 }  // namespace moe

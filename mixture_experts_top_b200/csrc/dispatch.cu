@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kCountWarps * 32)
     dispatch_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                           int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
                           int32_t* err) {
+  pdl_wait_and_release();
   __shared__ int32_t whist[kCountWarps][kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = lane; e < E; e += 32) whist[warp][e] = 0;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(1024)
                          int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, float* __restrict__ f,
                          float* __restrict__ aux) {
+  pdl_wait_and_release();
   __shared__ int32_t s_counts[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int e = warp; e < E; e += nwarps) {
@@ -150,6 +152,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ dest,
                             int32_t* __restrict__ perm_token, uint8_t* __restrict__ drop_mask,
                             uint8_t* __restrict__ x_perm) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -194,26 +197,20 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
   const int nchunks = ceil_div(c.T, kChunkTokens);
   const int64_t cap = capacity_slots(c.capacity_factor, c.T, c.top_k, c.E);
   if (nchunks > 0) {
-    dispatch_count_kernel<<<nchunks, kCountWarps * 32, 0, s>>>(idx, c.T, c.top_k, c.E,
-                                                                chunk_counts, local_rank, err);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
+                                  c.T, c.top_k, c.E, chunk_counts, local_rank, err);
     if (e != cudaSuccess) return e;
   }
-  dispatch_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, nchunks, c.E, c.T, c.top_k, cap,
-                                          prob_mean, chunk_base, counts, offsets, f, aux);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(dispatch_scan_kernel, 1, 1024, 0, s, 0, chunk_counts, nchunks,
+                                c.E, c.T, c.top_k, cap, prob_mean, chunk_base, counts, offsets,
+                                f, aux);
   if (e != cudaSuccess || c.T == 0) return e;
   const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
-  if (elem == 2)
-    dispatch_scatter_kernel<2><<<blocks, 256, 0, s>>>(
-        static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d, cap, chunk_base, local_rank,
-        offsets, dest, perm_token, drop_mask, static_cast<uint8_t*>(x_perm));
-  else
-    dispatch_scatter_kernel<4><<<blocks, 256, 0, s>>>(
-        static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d, cap, chunk_base, local_rank,
-        offsets, dest, perm_token, drop_mask, static_cast<uint8_t*>(x_perm));
-  return cudaGetLastError();
+  return launch_kernel(elem == 2 ? dispatch_scatter_kernel<2> : dispatch_scatter_kernel<4>, blocks,
+                       256, 0, s, 0, static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d,
+                       cap, chunk_base, local_rank, offsets, dest, perm_token, drop_mask,
+                       static_cast<uint8_t*>(x_perm));
 }
 
 }  // namespace moe

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256)
     linear_expert_kernel(const float* __restrict__ x_perm, const int32_t* __restrict__ offsets,
                          const float* __restrict__ W, float* __restrict__ y_perm, int rows_max,
                          int E, int d, int d_out, int32_t* err) {
+  pdl_wait_and_release();
   __shared__ int32_t off[kMaxE + 1];
   __shared__ int ok;
   if (threadIdx.x == 0 && threadIdx.y == 0) ok = 1;
@@ -62,9 +63,8 @@ cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
   if (rows_max == 0) return cudaSuccess;
   const dim3 block(32, 8);
   const dim3 grid(ceil_div(c.d_out, 32), min(ceil_div(rows_max, 8), 8192));
-  linear_expert_kernel<<<grid, block, 0, s>>>(x_perm, offsets, W, y_perm, rows_max, c.E, c.d,
-                                               c.d_out, err);
-  return cudaGetLastError();
+  return launch_kernel(linear_expert_kernel, grid, block, 0, s, 0, x_perm, offsets, W, y_perm,
+                       rows_max, c.E, c.d, c.d_out, err);
 }
 
 }  // namespace moe

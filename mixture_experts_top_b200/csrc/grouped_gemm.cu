@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+  pdl_wait_and_release();
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;  // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -419,6 +420,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+  pdl_wait_and_release();
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -647,8 +649,7 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
   auto kern = grouped_gemm_kernel<EPI>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, g);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, NUM_THREADS, SMEM_BYTES, s, 0, a, b0, b1, g);
 }
 
 template <int EPI>
@@ -657,19 +658,7 @@ cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUt
   auto kern = grouped_gemm_pair_kernel<EPI>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), P_SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = P_SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, g);
+  return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, g);
 }
 
 }  // namespace

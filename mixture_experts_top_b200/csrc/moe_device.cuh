@@ -307,6 +307,16 @@ __device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
                : "memory");
 }
 
+// --------------------------------------------- programmatic dependent launch --
+// Every kernel of the library is launched so that it may be scheduled while
+// the kernel before it in the stream is still draining.  Each kernel first
+// waits for that predecessor to complete (and its memory to be visible)
+// before it touches global memory, then lets its own successor be scheduled.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- small utils --
 
 __device__ __forceinline__ uint32_t lanemask_lt() {

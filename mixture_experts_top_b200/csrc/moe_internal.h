@@ -6,6 +6,7 @@
 #include <stddef.h>
 
 #include <algorithm>
+#include <utility>
 #include <stdint.h>
 
 #include "../../include/moe.h"
@@ -48,6 +49,34 @@ int device_sm_count();
 
 // Sets a kernel's dynamic shared-memory limit once per (device, kernel).
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+
+// Launches `kern` with programmatic stream serialization (the kernel may be
+// scheduled while its predecessor drains; it waits for it in-kernel) and, if
+// cluster > 0, an explicit 1-D cluster of that many CTAs (0: no cluster
+// attribute).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,

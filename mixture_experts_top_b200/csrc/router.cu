@@ -124,6 +124,7 @@ struct RouterShape {
 template <typename XT, int TM, int TN, int WN, int KS, int BK, int ST>
 __global__ void __launch_bounds__(32 * WN * KS)
     router_kernel(const RouterArgs<XT> a) {
+  pdl_wait_and_release();
   using S = RouterShape<XT, TM, TN, WN, KS, BK, ST>;
   constexpr int VEC = S::VEC, EP = S::EP, NT = S::THREADS, XROW = S::XROW, BM = S::BM;
   constexpr int QMAX = (EP + 31) / 32;  // experts per lane in the finishing pass
@@ -360,6 +361,7 @@ __global__ void __launch_bounds__(32 * WN * KS)
 __global__ void __launch_bounds__(256)
     prob_mean_kernel(const float* __restrict__ part, int nrows, int E, int T,
                      float* __restrict__ prob_mean) {
+  pdl_wait_and_release();
   __shared__ double acc[256];
   const int groups = max(1, (int)blockDim.x / E);   // threads per expert
   const int e = threadIdx.x % E, g = threadIdx.x / E;
@@ -394,19 +396,7 @@ cudaError_t run_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles_out) 
   *tiles_out = tiles;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), S::SMEM);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(tiles * nsplit), 1, 1);
-  cfg.blockDim = dim3(S::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = S::SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)nsplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return launch_kernel(kern, tiles * nsplit, S::THREADS, S::SMEM, s, nsplit, a);
 }
 
 // Two tokens per lane everywhere (each W broadcast feeds two packed FMAs);
@@ -442,8 +432,8 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_ro
     }
     if (e != cudaSuccess) return e;
   }
-  prob_mean_kernel<<<1, 256, 0, s>>>(router_part, tiles, c.E, c.T, prob_mean);
-  return cudaGetLastError();
+  return launch_kernel(prob_mean_kernel, 1, 256, 0, s, 0, router_part, tiles, c.E, c.T,
+                       prob_mean);
 }
 
 }  // namespace moe
