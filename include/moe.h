@@ -46,6 +46,9 @@
  *     pipeline wait that exceeded its time limit) are written to an error
  *     word in the workspace and reported by moe_device_status.
  *   - Row-major layouts; rows of x, x_perm, y_perm and output are contiguous.
+ *   - x, x_perm, y_perm, output, W_in, W_up and W_out start on a 16-byte
+ *     boundary (they are moved with 16-byte vectors and TMA); a misaligned
+ *     one is rejected with MOE_ERR_INVALID_ARG.
  *   - bf16 tensors are IEEE bfloat16 (upper half of an fp32).
  *   - Inputs must be finite; results for NaN or Inf inputs are undefined.
  *   - T = 0 is valid: nothing is routed, prob_mean, f and aux_loss are 0.
@@ -121,7 +124,12 @@ int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t
  *   prob_mean    (E) fp32 out: P_e = mean over tokens of softmax(logits)[:, e]
  *   logits_out   (T, E) fp32 out or NULL: the fp32 logits the top-k decided on
  * The logits are fp32: the dot product is accumulated in fp32, then the
- * bias and then the noise are each added in fp32. */
+ * bias and then the noise are each added in fp32.  With bf16 x and E <= 64
+ * the dot product runs on the tensor cores: W_router is split exactly into
+ * three bf16 terms (hi + mid + lo), so every product x_i * W_part is exact in
+ * fp32 and the tensor core's fp32 accumulator adds them; the workspace holds
+ * the split (3 * EP * d bf16, EP = E rounded up to 16, 32 or 64).  Otherwise
+ * the fp32 pipes compute it. */
 int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
               const float* logit_bias, const float* noise,
               int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,
@@ -145,7 +153,11 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
  *   race on it; order such calls on one stream.
  *   Set-up: the first call on each device looks up the array's device
  *   address (with that device current) and caches it; make that first call
- *   before any stream capture.  No call allocates or frees memory. */
+ *   before any stream capture.  No call allocates or frees memory.
+ *   Arithmetic: this entry point always computes the logits on the fp32
+ *   pipes (it has no room for moe_route's split copy of W_router), so its
+ *   logits may differ from moe_route's in the last bits; both are fp32 dot
+ *   products of the same inputs. */
 int moe_route_noalloc(const moe_config_t* cfg, const void* x, const float* W_router,
                       const float* logit_bias, const float* noise,
                       int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,

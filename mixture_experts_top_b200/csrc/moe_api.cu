@@ -76,6 +76,13 @@ int check_ws(const moe_config_t& c, void* ws, size_t ws_bytes) {
     if ((ptr) == nullptr) return fail(MOE_ERR_INVALID_ARG, #ptr " is NULL"); \
   } while (0)
 
+// Row tensors and expert weights are moved with 16-byte vectors and TMA.
+#define MOE_ALIGNED16(ptr)                                                     \
+  do {                                                                         \
+    if ((reinterpret_cast<uintptr_t>(ptr) & 15u) != 0)                         \
+      return fail(MOE_ERR_INVALID_ARG, #ptr " must be 16-byte aligned");       \
+  } while (0)
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -124,6 +131,7 @@ WsLayout workspace_layout(const moe_config_t& c) {
   const size_t n_chunks = (size_t)std::max(1, ceil_div(c.T, kChunkTokens));
   L.ctrl = take(256);
   L.router_part = take(n_router * E * 4);
+  L.w_split = take((size_t)3 * (size_t)router_tc_width(c) * (size_t)c.d * 2);
   L.prob_mean = take(E * 4);
   L.chunk_counts = take(n_chunks * E * 4);
   L.chunk_base = take(n_chunks * E * 4);
@@ -225,12 +233,14 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
     MOE_REQUIRE(expert_indices);
     MOE_REQUIRE(gates);
   }
+  MOE_ALIGNED16(x);
   MOE_REQUIRE(W_router);
   MOE_REQUIRE(prob_mean);
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = workspace_layout(c);
   const cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates,
                                      prob_mean, logits_out, at<float>(ws, L.router_part),
+                                     at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl),
                                      reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
 }
@@ -250,6 +260,8 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
     MOE_REQUIRE(drop_mask);
     MOE_REQUIRE(x_perm);
   }
+  MOE_ALIGNED16(x);
+  MOE_ALIGNED16(x_perm);
   MOE_REQUIRE(prob_mean);
   MOE_REQUIRE(counts);
   MOE_REQUIRE(offsets);
@@ -279,6 +291,11 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* o
     MOE_REQUIRE(x_perm);
     MOE_REQUIRE(y_perm);
   }
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
+  MOE_ALIGNED16(x_perm);
+  MOE_ALIGNED16(y_perm);
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
   const cudaError_t e = run_experts(c, x_perm, offsets, W_in, W_up, W_out, y_perm, ws,
                                     reinterpret_cast<cudaStream_t>(stream));
@@ -296,6 +313,8 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest
     MOE_REQUIRE(gates);
     MOE_REQUIRE(output);
   }
+  MOE_ALIGNED16(y_perm);
+  MOE_ALIGNED16(output);
   const cudaError_t e = launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output,
                                        reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine");
@@ -320,6 +339,11 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
   if (c.expert_kind != MOE_EXPERT_LINEAR) MOE_REQUIRE(W_out);
   MOE_REQUIRE(aux_loss);
+  MOE_ALIGNED16(x);
+  MOE_ALIGNED16(output);
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = workspace_layout(c);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -331,7 +355,8 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, P,
-                               nullptr, at<float>(ws, L.router_part), s);
+                               nullptr, at<float>(ws, L.router_part),
+                               at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl), s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/route");
   e = launch_dispatch(c, x, expert_indices, P, cnt, offs, dest, at<int32_t>(ws, L.perm_token),
                       drop, at<float>(ws, L.f), aux_loss, x_perm, at<int32_t>(ws, L.chunk_counts),
@@ -411,6 +436,7 @@ extern "C" int moe_route_noalloc(const moe_config_t* cfg, const void* x, const f
     MOE_REQUIRE(expert_indices);
     MOE_REQUIRE(gates);
   }
+  MOE_ALIGNED16(x);
   MOE_REQUIRE(W_router);
   MOE_REQUIRE(prob_mean);
   const size_t need = (size_t)std::max(1, ceil_div(c.T, kRouterTokens)) * (size_t)c.E;
@@ -423,6 +449,6 @@ extern "C" int moe_route_noalloc(const moe_config_t* cfg, const void* x, const f
   cudaError_t e = route_scratch_address(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "moe_route_noalloc: cudaGetSymbolAddress");
   e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, prob_mean,
-                   logits_out, scratch, reinterpret_cast<cudaStream_t>(stream));
+                   logits_out, scratch, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_noalloc");
 }

@@ -1,6 +1,7 @@
 // moe_internal.h - host-side declarations shared by the library's .cu files.
 #pragma once
 
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -24,6 +25,7 @@ constexpr int kChunkTokens = 256;
 struct WsLayout {
   size_t ctrl;           // int32 error word (+ padding)
   size_t router_part;    // (router CTAs, E) fp32 per-CTA column sums of probs
+  size_t w_split;        // (3, EP, d) bf16: W_router split for the tensor-core router
   size_t prob_mean;      // (E) fp32, moe_forward only
   size_t chunk_counts;   // (chunks, E) int32
   size_t chunk_base;     // (chunks, E) int32
@@ -46,6 +48,17 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Per-device properties cached on first use.
 int device_sm_count();
+
+// The driver's cuTensorMapEncodeTiled, looked up once (nullptr if missing).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Expert columns of the tensor-core router for this configuration (E padded
+// to 16, 32 or 64), or 0 where the fp32 SIMT router runs instead (fp32
+// activations, or E > 64).
+inline int router_tc_width(const moe_config_t& c) {
+  if (c.act_dtype != MOE_BF16 || c.E > 64) return 0;
+  return c.E <= 16 ? 16 : (c.E <= 32 ? 32 : 64);
+}
 
 // Sets a kernel's dynamic shared-memory limit once per (device, kernel).
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
@@ -79,10 +92,19 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 }
 
 // Launchers; each returns cudaSuccess or the launch error.
+// w_split (3 * router_tc_width(c) * d bf16) selects the tensor-core router
+// where router_tc_width(c) > 0; nullptr always runs the SIMT router.  err is
+// the workspace error word (may be nullptr with w_split == nullptr).
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
-                         cudaStream_t s);
+                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s);
+// Tensor-core router (router_tc.cu): logits, softmax, top-k, gates and one
+// row of probability column sums per 128-token tile; *tiles_out = rows.
+cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W_router,
+                            const float* bias, const float* noise, int32_t* idx, float* gates,
+                            float* logits_out, float* router_part, __nv_bfloat16* w_split,
+                            int32_t* err, cudaStream_t s, int* tiles_out);
 
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* idx,
                             const float* prob_mean, int32_t* counts, int32_t* offsets,

@@ -417,11 +417,14 @@ cudaError_t dispatch_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles)
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
-                         cudaStream_t s) {
+                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s) {
   int tiles = 0;  // token tiles; each writes one row of router_part
   if (c.T > 0) {
     cudaError_t e;
-    if (c.act_dtype == MOE_BF16) {
+    if (w_split != nullptr && router_tc_width(c) > 0) {
+      e = launch_route_tc(c, static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
+                          gates, logits_out, router_part, w_split, err, s, &tiles);
+    } else if (c.act_dtype == MOE_BF16) {
       RouterArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
                                   gates, logits_out, router_part, c.T, c.d, c.E, c.top_k};
       e = dispatch_router(a, s, &tiles);

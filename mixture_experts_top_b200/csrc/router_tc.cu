@@ -1,0 +1,450 @@
+// router_tc.cu - the router on the tensor cores for bf16 tokens: fp32
+// logits, softmax, top-k, renormalised gates and the column sums of the
+// probabilities, in one kernel.
+//
+// What it computes is the router of router.cu:
+// "Mixture-of-Experts Routing - LLM Internals" (mlgrind.dev), Algorithm 1-2:
+//   logits = x @ W_router; probs = softmax(logits); indices = the k largest
+//   logits by descending value, lower index first on ties; gates = softmax
+//   over the chosen k logits.
+// "Mixture of Experts: the Sparsely-Gated Layer" (paperfordummies.in), The
+// code, `router`: an optional per-expert bias, then optional noise, are added
+// to the logits before the softmax and the top-k.
+//
+// fp32 logits from bf16 tensor cores.  x is bf16, so every x_i is exact.
+// W_router (fp32) is split exactly into three bf16 terms, W = W_hi + W_mid +
+// W_lo, each taking the next 8 significant bits of the fp32 value (the
+// remainders w - W_hi and (w - W_hi) - W_mid are exact in fp32).  Every
+// product x_i * W_part has at most 16 significant bits and is exact in fp32,
+// and tcgen05.mma (kind::f16: bf16 in, fp32 accumulate) adds them in fp32.
+// The tensor core's accumulator does not round to nearest (its errors lean
+// towards zero, measured on B200), so it only sums one 64-wide block of d
+// (4 x 3 MMAs); the blocks' sums are added in round-to-nearest fp32 in
+// registers, in block order.  The result is an fp32 dot product like the
+// scalar router's, in another summation order, and the contraction is bound
+// by reading x from HBM instead of by the fp32 pipes.
+//
+// Design (B200)
+//  * A split kernel writes (W_hi, W_mid, W_lo) as one (3, EP, d) bf16 array,
+//    d contiguous (a K-major operand), rows E..EP-1 zero; EP = E padded to
+//    16, 32 or 64 (the MMA's N).
+//  * A thread-block cluster of S CTAs (S = 1..8) owns a tile of 128 tokens;
+//    CTA r of the cluster takes 1/S of the contraction range d.  192 threads:
+//    warp 0 lane 0 issues TMA copies (x box 64 (d) x 128 (tokens) and the
+//    three W boxes 64 (d) x EP, 128-byte swizzle) into a ring of stages;
+//    warp 1 lane 0 issues, per 64-wide d block, 4 x 3 tcgen05.mma
+//    M128 x N=EP x K16 into a fresh fp32 accumulator in tensor memory (for
+//    each 16-wide slice: the hi, mid and lo terms), alternating between two
+//    accumulators; warps 2-5 (warp w reads TMEM lanes 32 (w mod 4) ..) add
+//    each block's accumulator row into their token's fp32 registers and
+//    release it.  Out-of-range tokens and d are zero-filled by TMA.
+//  * Epilogue: each token's partial logits go to shared memory; after a
+//    cluster barrier, the CTA of rank r finishes tokens
+//    [r 128/S, (r+1) 128/S) of the tile, one thread per token: the S partial
+//    logit rows added in rank order through distributed shared memory, bias,
+//    noise, top-k by k scans in expert order (strictly greater wins, so the
+//    lower index wins ties), the softmax (its maximum is the first top-k
+//    logit) and the gates.  Each CTA then adds its tokens' probabilities per
+//    expert in token order, and rank 0 adds the S sums in rank order into the
+//    tile's row of column sums (the fp64 mean over rows is router.cu's).
+//  * Every mbarrier wait is bounded; on expiry the error word is set, the
+//    copies in flight are drained and tensor memory is freed.
+#include <cooperative_groups.h>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace moe {
+namespace {
+
+constexpr int TBM = 128;       // tokens per CTA (UMMA M)
+constexpr int TBK = 64;        // d per stage: one 128-byte swizzle row of bf16
+constexpr int TUK = 16;        // d per tcgen05.mma (kind::f16)
+constexpr int TTHREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 accumulate and finish
+constexpr int kTopKMax = 8;
+
+template <int EP>
+struct TcShape {
+  static_assert(EP == 16 || EP == 32 || EP == 64, "EP is 16, 32 or 64");
+  static constexpr int ST = EP == 16 ? 4 : (EP == 32 ? 3 : 2);   // two CTAs per SM
+  static constexpr int X_BYTES = TBM * TBK * 2;                  // 16 KiB
+  static constexpr int W_PART = EP * TBK * 2;                    // one term's box
+  static constexpr int STAGE = X_BYTES + 3 * W_PART;
+  static constexpr int LGS = EP + 4;                             // padded logit row (floats)
+  static constexpr int PIPE = ST * STAGE;
+  static constexpr int LG_BYTES = TBM * LGS * 4;
+  static constexpr int MAIN = PIPE > LG_BYTES ? PIPE : LG_BYTES;
+  static constexpr int AUX = 256;                                // barriers, TMEM address
+  static constexpr int SMEM = 1024 + MAIN + EP * 4 + AUX;
+  static constexpr uint32_t TMEM_COLS = 2 * EP < 32 ? 32u : (uint32_t)(2 * EP);  // two accumulators
+  // kind::f16: D fp32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 =
+  // 1), A and B K-major (bits 15, 16 = 0), N >> 3 at 17, M >> 4 at 24.
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(TBM >> 4) << 24);
+  static_assert((2 * ST + 5) * 8 + 4 <= AUX, "barriers fit");
+};
+
+// K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024
+// bytes apart (stride byte offset); the leading byte offset is unused for
+// this layout (16 bytes); descriptor version 1 (bit 46); swizzle mode 2.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+struct TcArgs {
+  const float* bias;
+  const float* noise;
+  int32_t* idx;
+  float* gates;
+  float* logits_out;
+  float* part;
+  int32_t* err;
+  int T, d, E, k;
+};
+
+// (d, E) fp32 -> (3, EP, d) bf16 terms hi, mid, lo with w = hi + mid + lo.
+// One block per 64 rows of d, transposed through shared memory.
+__global__ void __launch_bounds__(256)
+    split_router_weights_kernel(const float* __restrict__ W, int d, int E, int EP,
+                                __nv_bfloat16* __restrict__ out) {
+  pdl_wait_and_release();
+  __shared__ float tile[TBK][65];
+  const int k0 = blockIdx.x * TBK;
+  for (int i = threadIdx.x; i < TBK * E; i += blockDim.x) {
+    const int kk = i / E, e = i - kk * E;
+    tile[kk][e] = (k0 + kk < d) ? W[(size_t)(k0 + kk) * E + e] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < EP * TBK; i += blockDim.x) {
+    const int e = i / TBK, kk = i % TBK;
+    if (k0 + kk >= d) continue;
+    const float w = e < E ? tile[kk][e] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = __fsub_rn(w, __bfloat162float(hi));      // exact
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(mid));    // exact, <= 8 bits
+    const size_t o = (size_t)e * d + k0 + kk;
+    out[o] = hi;
+    out[(size_t)EP * d + o] = mid;
+    out[(size_t)2 * EP * d + o] = __float2bfloat16_rn(r2);
+  }
+}
+
+template <int EP>
+__global__ void __launch_bounds__(TTHREADS, 2)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const TcArgs a) {
+  pdl_wait_and_release();
+  using S = TcShape<EP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* lg = reinterpret_cast<float*>(smem);                  // after the main loop
+  float* csum = reinterpret_cast<float*>(smem + S::MAIN);      // EP floats
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S::MAIN + EP * 4);
+  uint64_t* empty_bar = full_bar + S::ST;
+  uint64_t* tfull_bar = empty_bar + S::ST;   // [2] accumulator written
+  uint64_t* tempty_bar = tfull_bar + 2;      // [2] accumulator read
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int nsplit = (int)cluster.num_blocks();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = a.T, E = a.E;
+  const int tile = blockIdx.x / nsplit;
+  const int t_base = tile * TBM;
+  const int total_chunks = (a.d + TBK - 1) / TBK;
+  const int per = (total_chunks + nsplit - 1) / nsplit;
+  const int c_begin = min(rank * per, total_chunks);
+  const int nchunks = min(per, total_chunks - c_begin);
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmX);
+    tma_prefetch_map(&tmW);
+  } else if (warp == 1) {
+    tmem_alloc(tmem_holder, S::TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 2 && lane == 0) {
+    for (int s = 0; s < S::ST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, last_phase = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
+        report_error(a.err, kDevTimeoutProducer);
+        break;
+      }
+      uint8_t* sx = smem + stage * S::STAGE;
+      const int k0 = (c_begin + c) * TBK;
+      mbar_arrive_expect_tx(&full_bar[stage], S::STAGE);
+      tma_load_2d(sx, &tmX, &full_bar[stage], k0, t_base);
+      tma_load_3d(sx + S::X_BYTES, &tmW, &full_bar[stage], k0, 0, 0);
+      issued |= 1u << stage;
+      last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+      if (++stage == S::ST) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    for (int s = 0; s < S::ST; ++s)
+      if ((issued >> s) & 1u)
+        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(a.err, kDevTimeoutDrain);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      if (!mbar_wait(&tempty_bar[b], ((uint32_t)(c >> 1) & 1u) ^ 1u) ||
+          !mbar_wait(&full_bar[stage], phase)) {
+        report_error(a.err, kDevTimeoutMma);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t sx = smem_u32(smem + stage * S::STAGE);
+      const uint32_t sw = sx + S::X_BYTES;
+      const uint32_t acc = tmem + (uint32_t)(b * EP);
+#pragma unroll
+      for (int kk = 0; kk < TBK / TUK; ++kk) {
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          umma_bf16_ss(acc, desc_kmajor_sw128(sx + kk * TUK * 2),
+                       desc_kmajor_sw128(sw + p * S::W_PART + kk * TUK * 2), S::IDESC,
+                       (kk | p) != 0 ? 1u : 0u);
+      }
+      umma_commit(&empty_bar[stage]);   // frees the stage once these MMAs finish
+      umma_commit(&tfull_bar[b]);       // this block's sums are ready
+      if (++stage == S::ST) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    umma_commit(drain_bar);  // every MMA issued above completes before TMEM is freed
+    if (!mbar_wait(drain_bar, 0)) report_error(a.err, kDevTimeoutDrain);
+  } else if (warp >= 2) {
+    // ------------------------------- per-block sums -> fp32 registers -> smem
+    const int q = warp & 3;                 // TMEM lanes 32q .. 32q + 31
+    float acc[EP];
+#pragma unroll
+    for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      const bool ready = mbar_wait(&tfull_bar[b], (uint32_t)(c >> 1) & 1u);
+      if (!__all_sync(0xffffffffu, ready)) {
+        if (lane == 0) report_error(a.err, kDevTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * EP);
+      if (EP == 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] += __uint_as_float(r[j]);
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < EP; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + (uint32_t)c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[(c0 + j) % EP] += __uint_as_float(r[j]);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&tempty_bar[b]);
+    }
+    float* my = lg + (q * 32 + lane) * S::LGS;
+#pragma unroll
+    for (int e = 0; e < EP; e += 4)
+      *reinterpret_cast<float4*>(my + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+  }
+  __syncwarp();
+  cluster.sync();  // every CTA's partial logits are complete and visible
+
+  // ---------------------------------------------- finishing, one thread a token
+  const int rpc = TBM / nsplit;  // tokens finished by each CTA of the cluster
+  const int r0 = rank * rpc;
+  const int ft = (int)threadIdx.x - 64;  // warps 2-5 finish the tokens
+  if (ft >= 0 && ft < rpc) {
+    const int r = r0 + ft;
+    const int t = t_base + r;
+    if (t < T) {
+      float L[EP];
+#pragma unroll
+      for (int e = 0; e < EP; ++e) L[e] = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float* src = cluster.map_shared_rank(lg, sp) + r * S::LGS;
+#pragma unroll
+        for (int e = 0; e < EP; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src + e);
+          L[e] += v.x;
+          L[e + 1] += v.y;
+          L[e + 2] += v.z;
+          L[e + 3] += v.w;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          if (a.bias != nullptr) L[e] = __fadd_rn(L[e], a.bias[e]);
+          if (a.noise != nullptr) L[e] = __fadd_rn(L[e], a.noise[(size_t)t * E + e]);
+          if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = L[e];
+        }
+      }
+      // Top-k: k scans in expert order; strictly greater replaces, so the
+      // lower index wins ties (-0 and +0 compare equal).
+      uint64_t taken = 0ull;
+      float vals[kTopKMax];
+      int ids[kTopKMax];
+      const int k = a.k;
+#pragma unroll
+      for (int j = 0; j < kTopKMax; ++j) {
+        float best = 0.f;
+        int bi = -1;
+        if (j < k) {
+#pragma unroll
+          for (int e = 0; e < EP; ++e)
+            if (e < E && !((taken >> e) & 1ull) && (bi < 0 || L[e] > best)) {
+              best = L[e];
+              bi = e;
+            }
+          taken |= 1ull << bi;
+        }
+        vals[j] = best;
+        ids[j] = bi;
+      }
+      // Softmax over the E logits; vals[0] is their maximum.
+      const float m = vals[0];
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        L[e] = e < E ? expf(L[e] - m) : 0.f;
+        sum += L[e];
+      }
+      float* pr = lg + r * S::LGS;  // this CTA's own row: no other CTA reads it
+#pragma unroll
+      for (int e = 0; e < EP; e += 4)
+        *reinterpret_cast<float4*>(pr + e) =
+            make_float4(L[e] / sum, L[e + 1] / sum, L[e + 2] / sum, L[e + 3] / sum);
+      float ex[kTopKMax];
+      float sk = 0.f;
+#pragma unroll
+      for (int j = 0; j < kTopKMax; ++j) {
+        ex[j] = j < k ? expf(vals[j] - vals[0]) : 0.f;
+        sk += ex[j];
+      }
+#pragma unroll
+      for (int j = 0; j < kTopKMax; ++j)
+        if (j < k) {
+          a.idx[(size_t)t * k + j] = ids[j];
+          a.gates[(size_t)t * k + j] = ex[j] / sk;
+        }
+    }
+  }
+  __syncthreads();
+  // Column sums of the probabilities over this CTA's tokens, in token order.
+  if ((int)threadIdx.x < EP) {
+    const int nvalid = min(rpc, T - (t_base + r0));
+    float v = 0.f;
+    for (int i = 0; i < nvalid; ++i) v += lg[(r0 + i) * S::LGS + threadIdx.x];
+    csum[threadIdx.x] = v;
+  }
+  cluster.sync();
+  if (rank == 0 && (int)threadIdx.x < E) {
+    float v = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) v += cluster.map_shared_rank(csum, sp)[threadIdx.x];
+    a.part[(size_t)tile * E + threadIdx.x] = v;
+  }
+  cluster.sync();  // peers keep their shared memory until rank 0 has read it
+
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, S::TMEM_COLS);
+  }
+}
+
+// Token tiles x splits: about one wave at two CTAs per SM, at most 8 CTAs per
+// cluster and at least one 64-wide d block per CTA.
+int tc_splits(int tiles, int chunks) {
+  const int slots = 2 * device_sm_count();
+  int s = 1;
+  while (s < 8 && tiles * s * 2 <= slots && s * 2 <= chunks) s *= 2;
+  return s;
+}
+
+bool encode_bf16(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                              const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EP>
+cudaError_t run_router_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W,
+                          const TcArgs& a, __nv_bfloat16* w_split, cudaStream_t s, int* tiles_out) {
+  using S = TcShape<EP>;
+  const int chunks = ceil_div(c.d, TBK);
+  cudaError_t e = launch_kernel(split_router_weights_kernel, chunks, 256, 0, s, 0, W, c.d, c.E,
+                                EP, w_split);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tx, tw;
+  const cuuint64_t xd[2] = {(cuuint64_t)c.d, (cuuint64_t)c.T};
+  const cuuint64_t xs[1] = {(cuuint64_t)c.d * 2};
+  const cuuint32_t xb[2] = {TBK, TBM};
+  const cuuint64_t wd[3] = {(cuuint64_t)c.d, (cuuint64_t)EP, 3};
+  const cuuint64_t wstr[2] = {(cuuint64_t)c.d * 2, (cuuint64_t)EP * (cuuint64_t)c.d * 2};
+  const cuuint32_t wb[3] = {TBK, EP, 3};
+  if (!encode_bf16(&tx, x, 2, xd, xs, xb) || !encode_bf16(&tw, w_split, 3, wd, wstr, wb))
+    return cudaErrorInvalidValue;
+  const int tiles = ceil_div(c.T, TBM);
+  const int nsplit = tc_splits(tiles, chunks);
+  *tiles_out = tiles;
+  auto kern = router_tc_kernel<EP>;
+  e = ensure_smem_limit(reinterpret_cast<const void*>(kern), S::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(kern, tiles * nsplit, TTHREADS, S::SMEM, s, nsplit, tx, tw, a);
+}
+
+}  // namespace
+
+cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W_router,
+                            const float* bias, const float* noise, int32_t* idx, float* gates,
+                            float* logits_out, float* router_part, __nv_bfloat16* w_split,
+                            int32_t* err, cudaStream_t s, int* tiles_out) {
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  const TcArgs a{bias, noise, idx, gates, logits_out, router_part, err, c.T, c.d, c.E, c.top_k};
+  switch (router_tc_width(c)) {
+    case 16: return run_router_tc<16>(c, x, W_router, a, w_split, s, tiles_out);
+    case 32: return run_router_tc<32>(c, x, W_router, a, w_split, s, tiles_out);
+    case 64: return run_router_tc<64>(c, x, W_router, a, w_split, s, tiles_out);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

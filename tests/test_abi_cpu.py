@@ -105,6 +105,32 @@ def test_null_pointers_and_workspace(moe_lib):
     assert moe_lib.moe_device_status(None, 1024, ctypes.byref(code), None) == api.MOE_ERR_WORKSPACE
 
 
+def test_row_tensors_must_be_16_byte_aligned(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    st = moe_lib.moe_route(ctypes.byref(cfg), FAKE + 8, FAKE, None, None, FAKE, FAKE, FAKE, None,
+                           FAKE, ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    assert "x must be 16-byte aligned" in moe_lib.moe_last_error_message().decode()
+    st = moe_lib.moe_expert_ffn(ctypes.byref(cfg), FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, FAKE,
+                                ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    assert "W_up must be 16-byte aligned" in moe_lib.moe_last_error_message().decode()
+    st = moe_lib.moe_combine(ctypes.byref(cfg), FAKE, FAKE, FAKE, FAKE + 4, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_holds_the_split_router_weights(moe_lib):
+    """bf16 with E <= 64 adds 3 * EP * d bf16 for the tensor-core router."""
+    a = api.make_config(64, 4096, 128, 64, 8, 2, "swiglu", "bf16")
+    b = api.make_config(64, 4096, 128, 64, 100, 2, "swiglu", "bf16")   # E > 64: SIMT router
+    c = api.make_config(64, 4096, 128, 64, 16, 2, "swiglu", "bf16")
+    na, nb, nc = (moe_lib.moe_workspace_size(ctypes.byref(x)) for x in (a, b, c))
+    assert nc - na == 0                                  # E = 8 and 16 both pad to 16
+    assert na >= 3 * 16 * 4096 * 2
+    assert nb > 0
+
+
 def test_swiglu_needs_three_matrices(moe_lib):
     cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
     ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))

@@ -46,6 +46,7 @@ EXACT_CASES = [
     (77, 128, 256, 8, "f32"),
     (1, 8, 1, 1, "bf16"),
     (5, 16, 4, 4, "f32"),          # k = E
+    (20000, 256, 16, 2, "bf16"),   # > 2 tiles per SM: one CTA per token tile, no split of d
 ]
 
 
@@ -62,6 +63,30 @@ def test_route_exact_logits_bit_exact(T, d, E, k, dtype, extras):
     cfg = cfg_of(_wl(T, d, E, k, dtype))
     g = run_route(cfg, inp["x"], inp["W_router"], bias, noise)
     o = O.moe_route(inp["x"], inp["W_router"], k, dtype, bias, noise)
+    assert np.array_equal(g["L"], o["logits"]), "fp32 logits must be bit-identical"
+    assert np.array_equal(g["idx"], o["expert_indices"])
+    assert rel_close(g["gates"], o["gates"], REL_ROUTE)
+    assert rel_close(g["P"], o["P"], REL_ROUTE)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(300, 64, 8, 2), (129, 200, 64, 6), (64, 4096, 32, 4)])
+def test_route_full_precision_router_weights(T, d, E, k):
+    """bf16 tokens that are one-hot (one entry +-2^j, the rest 0) make every
+    logit one fp32 router weight times a power of two, exactly: the logits
+    must equal the oracle's bit for bit, whatever the 24-bit mantissas of
+    W_router.  This checks that no bit of the fp32 weights is lost by the
+    bf16 tensor-core router, which splits each weight into three bf16 terms."""
+    rng = np.random.default_rng(T * 7 + E)
+    xf = np.zeros((T, d), np.float32)
+    t = np.arange(T)
+    xf[t, rng.integers(0, d, size=T)] = (rng.choice([-1.0, 1.0], size=T) *
+                                          2.0 ** rng.integers(-3, 4, size=T)).astype(np.float32)
+    x = (xf.view(np.uint32) >> 16).astype(np.uint16)        # exact in bf16
+    Wr = rng.standard_normal((d, E)).astype(np.float32) * np.float32(0.37)
+    bias = rng.standard_normal(E).astype(np.float32)
+    cfg = cfg_of(_wl(T, d, E, k, "bf16"))
+    g = run_route(cfg, x, Wr, bias)
+    o = O.moe_route(x, Wr, k, "bf16", bias, None)
     assert np.array_equal(g["L"], o["logits"]), "fp32 logits must be bit-identical"
     assert np.array_equal(g["idx"], o["expert_indices"])
     assert rel_close(g["gates"], o["gates"], REL_ROUTE)
