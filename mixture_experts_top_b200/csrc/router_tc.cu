@@ -19,7 +19,7 @@
 // and tcgen05.mma (kind::f16: bf16 in, fp32 accumulate) adds them in fp32.
 // The tensor core's accumulator does not round to nearest (its errors lean
 // towards zero, measured on B200), so it only sums one 64-wide block of d
-// (4 x 3 MMAs); the blocks' sums are added in round-to-nearest fp32 in
+// (4 MMAs); the blocks' sums are added in round-to-nearest fp32 in
 // registers, in block order.  The result is an fp32 dot product like the
 // scalar router's, in another summation order, and the contraction is bound
 // by reading x from HBM instead of by the fp32 pipes.
@@ -32,12 +32,14 @@
 //    CTA r of the cluster takes 1/S of the contraction range d.  192 threads:
 //    warp 0 lane 0 issues TMA copies (x box 64 (d) x 128 (tokens) and the
 //    three W boxes 64 (d) x EP, 128-byte swizzle) into a ring of stages;
-//    warp 1 lane 0 issues, per 64-wide d block, 4 x 3 tcgen05.mma
-//    M128 x N=EP x K16 into a fresh fp32 accumulator in tensor memory (for
-//    each 16-wide slice: the hi, mid and lo terms), alternating between two
-//    accumulators; warps 2-5 (warp w reads TMEM lanes 32 (w mod 4) ..) add
-//    each block's accumulator row into their token's fp32 registers and
-//    release it.  Out-of-range tokens and d are zero-filled by TMA.
+//    warp 1 lane 0 issues, per 64-wide d block, 4 tcgen05.mma M128 x N x K16
+//    into a fresh fp32 accumulator in tensor memory, N = 3 EP: the three W
+//    boxes lie one after another in shared memory, so one MMA forms the hi,
+//    mid and lo products in three column groups (two accumulators alternate
+//    for EP <= 32); warps 2-5 (warp w reads TMEM lanes 32 (w mod 4) ..) add
+//    each block's hi + (mid + lo) into their token's fp32 registers and
+//    release the accumulator.  Out-of-range tokens and d are zero-filled by
+//    TMA.
 //  * Epilogue: each token's partial logits go to shared memory; after a
 //    cluster barrier, the CTA of rank r finishes tokens
 //    [r 128/S, (r+1) 128/S) of the tile, one thread per token: the S partial
@@ -78,11 +80,19 @@ struct TcShape {
   static constexpr int MAIN = PIPE > LG_BYTES ? PIPE : LG_BYTES;
   static constexpr int AUX = 256;                                // barriers, TMEM address
   static constexpr int SMEM = 1024 + MAIN + EP * 4 + AUX;
-  static constexpr uint32_t TMEM_COLS = 2 * EP < 32 ? 32u : (uint32_t)(2 * EP);  // two accumulators
+  // One MMA covers the three terms: B is the 3 EP rows (hi, mid, lo) of the
+  // stage, so an accumulator is 3 EP columns.  Two accumulators alternate
+  // (one when 2 x 3 EP columns would not leave room for a second CTA).
+  static constexpr int N = 3 * EP;
+  static constexpr int NBUF = EP <= 32 ? 2 : 1;
+  static constexpr int G = 1;   // 64-wide d blocks summed per accumulator before it is read
+  static constexpr uint32_t TMEM_COLS = NBUF * N <= 32 ? 32u : NBUF * N <= 64 ? 64u
+                                        : NBUF * N <= 128 ? 128u : 256u;
   // kind::f16: D fp32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 =
   // 1), A and B K-major (bits 15, 16 = 0), N >> 3 at 17, M >> 4 at 24.
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(TBM >> 4) << 24);
+                                    ((uint32_t)(N >> 3) << 17) | ((uint32_t)(TBM >> 4) << 24);
+  static_assert(NBUF * N <= 256 && N % 16 == 0, "accumulators fit half of tensor memory");
   static_assert((2 * ST + 5) * 8 + 4 <= AUX, "barriers fit");
 };
 
@@ -146,8 +156,8 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   float* csum = reinterpret_cast<float*>(smem + S::MAIN);      // EP floats
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S::MAIN + EP * 4);
   uint64_t* empty_bar = full_bar + S::ST;
-  uint64_t* tfull_bar = empty_bar + S::ST;   // [2] accumulator written
-  uint64_t* tempty_bar = tfull_bar + 2;      // [2] accumulator read
+  uint64_t* tfull_bar = empty_bar + S::ST;   // [NBUF] accumulator written
+  uint64_t* tempty_bar = tfull_bar + 2;      // [NBUF] accumulator read
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
 
@@ -215,8 +225,9 @@ __global__ void __launch_bounds__(TTHREADS, 2)
     int stage = 0;
     uint32_t phase = 0;
     for (int c = 0; c < nchunks; ++c) {
-      const int b = c & 1;
-      if (!mbar_wait(&tempty_bar[b], ((uint32_t)(c >> 1) & 1u) ^ 1u) ||
+      const int gi = c / S::G, b = gi % S::NBUF;
+      const bool first = (c % S::G) == 0;
+      if ((first && !mbar_wait(&tempty_bar[b], ((uint32_t)(gi / S::NBUF) & 1u) ^ 1u)) ||
           !mbar_wait(&full_bar[stage], phase)) {
         report_error(a.err, kDevTimeoutMma);
         break;
@@ -224,17 +235,15 @@ __global__ void __launch_bounds__(TTHREADS, 2)
       tc_fence_after_sync();
       const uint32_t sx = smem_u32(smem + stage * S::STAGE);
       const uint32_t sw = sx + S::X_BYTES;
-      const uint32_t acc = tmem + (uint32_t)(b * EP);
+      const uint32_t acc = tmem + (uint32_t)(b * S::N);
 #pragma unroll
-      for (int kk = 0; kk < TBK / TUK; ++kk) {
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-          umma_bf16_ss(acc, desc_kmajor_sw128(sx + kk * TUK * 2),
-                       desc_kmajor_sw128(sw + p * S::W_PART + kk * TUK * 2), S::IDESC,
-                       (kk | p) != 0 ? 1u : 0u);
-      }
+      for (int kk = 0; kk < TBK / TUK; ++kk)
+        umma_bf16_ss(acc, desc_kmajor_sw128(sx + kk * TUK * 2),
+                     desc_kmajor_sw128(sw + kk * TUK * 2), S::IDESC,
+                     (!first || kk != 0) ? 1u : 0u);
       umma_commit(&empty_bar[stage]);   // frees the stage once these MMAs finish
-      umma_commit(&tfull_bar[b]);       // this block's sums are ready
+      if ((c % S::G) == S::G - 1 || c == nchunks - 1)
+        umma_commit(&tfull_bar[b]);     // this group's sums are ready
       if (++stage == S::ST) {
         stage = 0;
         phase ^= 1u;
@@ -248,30 +257,28 @@ __global__ void __launch_bounds__(TTHREADS, 2)
     float acc[EP];
 #pragma unroll
     for (int e = 0; e < EP; ++e) acc[e] = 0.f;
-    for (int c = 0; c < nchunks; ++c) {
-      const int b = c & 1;
-      const bool ready = mbar_wait(&tfull_bar[b], (uint32_t)(c >> 1) & 1u);
+    const int ngroups = (nchunks + S::G - 1) / S::G;
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int b = gi % S::NBUF;
+      const bool ready = mbar_wait(&tfull_bar[b], (uint32_t)(gi / S::NBUF) & 1u);
       if (!__all_sync(0xffffffffu, ready)) {
         if (lane == 0) report_error(a.err, kDevTimeoutEpilogue);
         break;
       }
       tc_fence_after_sync();
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * EP);
-      if (EP == 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr, r);
+      // Columns [p EP, (p+1) EP) of the accumulator hold term p's block sums;
+      // the block adds hi + (mid + lo) to the running fp32 logits.
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * S::N);
+#pragma unroll
+      for (int c0 = 0; c0 < EP; c0 += 16) {
+        uint32_t hi[16], mid[16], lo[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, hi);
+        tmem_ld_32x32b_x16(taddr + (uint32_t)(EP + c0), mid);
+        tmem_ld_32x32b_x16(taddr + (uint32_t)(2 * EP + c0), lo);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] += __uint_as_float(r[j]);
-      } else {
-#pragma unroll
-        for (int c0 = 0; c0 < EP; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + (uint32_t)c0, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[(c0 + j) % EP] += __uint_as_float(r[j]);
-        }
+        for (int j = 0; j < 16; ++j)
+          acc[c0 + j] += __uint_as_float(hi[j]) + (__uint_as_float(mid[j]) + __uint_as_float(lo[j]));
       }
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[b]);
@@ -386,12 +393,15 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   }
 }
 
-// Token tiles x splits: about one wave at two CTAs per SM, at most 8 CTAs per
-// cluster and at least one 64-wide d block per CTA.
+// CTAs per token tile: doubled while the grid stays within one wave at two
+// CTAs per SM and every CTA keeps at least four 64-wide d blocks (fewer
+// leave each CTA's fixed start-up and finishing costs exposed), at most 8.
+// Measured on B200 at T x d = 8192 x 4096, 16384 x 2048, 4096 x 768, 64 x
+// 4096, 1024 x 4096 and 32768 x 4096: this picks the fastest of 1, 2, 4, 8.
 int tc_splits(int tiles, int chunks) {
   const int slots = 2 * device_sm_count();
   int s = 1;
-  while (s < 8 && tiles * s * 2 <= slots && s * 2 <= chunks) s *= 2;
+  while (s < 8 && tiles * 2 * s <= slots && chunks >= 4 * 2 * s) s *= 2;
   return s;
 }
 
