@@ -42,11 +42,13 @@
 //    TMA.
 //  * Epilogue: each token's partial logits go to shared memory; after a
 //    cluster barrier, the CTA of rank r finishes tokens
-//    [r 128/S, (r+1) 128/S) of the tile, one thread per token: the S partial
-//    logit rows added in rank order through distributed shared memory, bias,
-//    noise, top-k by k scans in expert order (strictly greater wins, so the
-//    lower index wins ties), the softmax (its maximum is the first top-k
-//    logit) and the gates.  Each CTA then adds its tokens' probabilities per
+//    [r 128/S, (r+1) 128/S) of the tile.  All its threads add the S partial
+//    logit rows in rank order through distributed shared memory, then the
+//    bias and the noise (coalesced, consecutive experts on consecutive
+//    threads); then a group of EP/8 lanes per token (8 experts a lane): top-k
+//    by k rounds of a group-wide maximum of 64-bit keys (order-preserving
+//    logit bits, then the complemented expert index, so the lower index wins
+//    ties), the softmax (its maximum is the first top-k logit) and the gates.  Each CTA then adds its tokens' probabilities per
 //    expert in token order, and rank 0 adds the S sums in rank order into the
 //    tile's row of column sums (the fp64 mean over rows is router.cu's).
 //  * Every mbarrier wait is bounded; on expiry the error word is set, the
@@ -65,7 +67,8 @@ constexpr int TBM = 128;       // tokens per CTA (UMMA M)
 constexpr int TBK = 64;        // d per stage: one 128-byte swizzle row of bf16
 constexpr int TUK = 16;        // d per tcgen05.mma (kind::f16)
 constexpr int TTHREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 accumulate and finish
-constexpr int kTopKMax = 8;
+constexpr int kCoopBatch = 8;  // elements per thread per round of the logit pass
+constexpr int kMaxTopK = 8;    // largest top_k the library accepts
 
 template <int EP>
 struct TcShape {
@@ -86,6 +89,7 @@ struct TcShape {
   static constexpr int N = 3 * EP;
   static constexpr int NBUF = EP <= 32 ? 2 : 1;
   static constexpr int G = 1;   // 64-wide d blocks summed per accumulator before it is read
+  static constexpr int FG = EP / 8;  // lanes per token in the finishing pass (8 experts each)
   static constexpr uint32_t TMEM_COLS = NBUF * N <= 32 ? 32u : NBUF * N <= 64 ? 64u
                                         : NBUF * N <= 128 ? 128u : 256u;
   // kind::f16: D fp32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 =
@@ -291,84 +295,144 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   __syncwarp();
   cluster.sync();  // every CTA's partial logits are complete and visible
 
-  // ---------------------------------------------- finishing, one thread a token
-  const int rpc = TBM / nsplit;  // tokens finished by each CTA of the cluster
+  // --------------------------------------- the tile's logits, all threads
+  // CTA r finishes tokens [r0, r0 + rpc) of the tile.  Their logits are the
+  // partial rows of the S CTAs added in rank order (read through distributed
+  // shared memory, consecutive experts on consecutive threads), then the
+  // bias and the noise, each in fp32; they overwrite this CTA's own partial
+  // rows, which no other CTA reads.  Each thread takes kCoopBatch elements
+  // at a time and issues all their loads before using any, so the load
+  // latencies overlap.
+  const int rpc = TBM / nsplit;
   const int r0 = rank * rpc;
-  const int ft = (int)threadIdx.x - 64;  // warps 2-5 finish the tokens
-  if (ft >= 0 && ft < rpc) {
-    const int r = r0 + ft;
-    const int t = t_base + r;
-    if (t < T) {
-      float L[EP];
+  {
+    const int n = rpc * EP;
+    for (int base = threadIdx.x; base < n; base += TTHREADS * kCoopBatch) {
+      float acc[kCoopBatch], bv[kCoopBatch], nv[kCoopBatch];
 #pragma unroll
-      for (int e = 0; e < EP; ++e) L[e] = 0.f;
+      for (int u = 0; u < kCoopBatch; ++u) {
+        const int i = base + u * TTHREADS;
+        acc[u] = 0.f;
+        bv[u] = 0.f;
+        nv[u] = 0.f;
+        const int r = r0 + i / EP, e = i % EP, t = t_base + r;
+        if (i < n && e < E && t < T) {
+          if (a.bias != nullptr) bv[u] = a.bias[e];
+          if (a.noise != nullptr) nv[u] = a.noise[(size_t)t * E + e];
+        }
+      }
       for (int sp = 0; sp < nsplit; ++sp) {
-        const float* src = cluster.map_shared_rank(lg, sp) + r * S::LGS;
+        const float* src = cluster.map_shared_rank(lg, sp);
+        float pv[kCoopBatch];
 #pragma unroll
-        for (int e = 0; e < EP; e += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src + e);
-          L[e] += v.x;
-          L[e + 1] += v.y;
-          L[e + 2] += v.z;
-          L[e + 3] += v.w;
+        for (int u = 0; u < kCoopBatch; ++u) {
+          const int i = base + u * TTHREADS;
+          pv[u] = i < n ? src[(r0 + i / EP) * S::LGS + i % EP] : 0.f;
         }
+#pragma unroll
+        for (int u = 0; u < kCoopBatch; ++u) acc[u] += pv[u];
       }
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        if (e < E) {
-          if (a.bias != nullptr) L[e] = __fadd_rn(L[e], a.bias[e]);
-          if (a.noise != nullptr) L[e] = __fadd_rn(L[e], a.noise[(size_t)t * E + e]);
-          if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = L[e];
+      for (int u = 0; u < kCoopBatch; ++u) {
+        const int i = base + u * TTHREADS;
+        if (i < n) {
+          const int r = r0 + i / EP, e = i % EP, t = t_base + r;
+          float v = acc[u];
+          if (e < E && t < T) {
+            if (a.bias != nullptr) v = __fadd_rn(v, bv[u]);
+            if (a.noise != nullptr) v = __fadd_rn(v, nv[u]);
+            if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = v;
+          }
+          lg[r * S::LGS + e] = v;
         }
       }
-      // Top-k: k scans in expert order; strictly greater replaces, so the
-      // lower index wins ties (-0 and +0 compare equal).
-      uint64_t taken = 0ull;
-      float vals[kTopKMax];
-      int ids[kTopKMax];
-      const int k = a.k;
+    }
+  }
+  __syncthreads();
+
+  // ------------------------------ finishing, a group of G lanes per token
+  // Each lane of a group holds 8 consecutive experts' logits.  Top-k: k
+  // rounds of a group-wide maximum of 64-bit keys (order-preserving logit
+  // bits, then the complemented expert index, so the lower index wins ties;
+  // -0 and +0 are one key); the lane that holds the winner zeroes its key.
+  // Softmax: the maximum is the first top-k logit; the exponentials are
+  // summed per lane, then over the group.  The probabilities overwrite the
+  // token's logit row, and the group's first lane writes indices and gates.
+  {
+    constexpr int G = S::FG;                         // lanes per token
+    const int lane_in = lane & (G - 1);
+    const uint32_t gmask = (G == 32) ? 0xffffffffu
+                                     : (((1u << G) - 1u) << (lane & ~(G - 1)));
+    const int group = (int)threadIdx.x / G;
+    const int k = a.k;
+    for (int rr = group; rr < rpc; rr += TTHREADS / G) {
+      const int r = r0 + rr;
+      const int t = t_base + r;
+      if (t >= T) break;                             // later rows are past T too
+      float* row = lg + r * S::LGS + lane_in * 8;
+      float L[8];
+      {
+        const float4 v0 = *reinterpret_cast<const float4*>(row);
+        const float4 v1 = *reinterpret_cast<const float4*>(row + 4);
+        L[0] = v0.x; L[1] = v0.y; L[2] = v0.z; L[3] = v0.w;
+        L[4] = v1.x; L[5] = v1.y; L[6] = v1.z; L[7] = v1.w;
+      }
+      const int e0 = lane_in * 8;
+      // The 8 keys of this lane, made once; a taken expert's key becomes 0.
+      uint64_t key[8];
 #pragma unroll
-      for (int j = 0; j < kTopKMax; ++j) {
-        float best = 0.f;
-        int bi = -1;
+      for (int q = 0; q < 8; ++q) {
+        const int e = e0 + q;
+        key[q] = e < E ? ((uint64_t)ordered_key(L[q]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e)
+                       : 0ull;
+      }
+      float vals[kMaxTopK];
+      int ids[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        vals[j] = 0.f;
+        ids[j] = 0;
         if (j < k) {
+          uint64_t best = key[0];
 #pragma unroll
-          for (int e = 0; e < EP; ++e)
-            if (e < E && !((taken >> e) & 1ull) && (bi < 0 || L[e] > best)) {
-              best = L[e];
-              bi = e;
-            }
-          taken |= 1ull << bi;
+          for (int q = 1; q < 8; ++q) best = key[q] > best ? key[q] : best;
+#pragma unroll
+          for (int o = 1; o < G; o <<= 1) {
+            const uint64_t other = __shfl_xor_sync(gmask, best, o);
+            best = other > best ? other : best;
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) key[q] = key[q] == best ? 0ull : key[q];
+          const uint32_t kb = (uint32_t)(best >> 32);
+          vals[j] = __uint_as_float((kb & 0x80000000u) ? (kb & 0x7FFFFFFFu) : ~kb);
+          ids[j] = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
         }
-        vals[j] = best;
-        ids[j] = bi;
       }
-      // Softmax over the E logits; vals[0] is their maximum.
       const float m = vals[0];
-      float sum = 0.f;
+      float p[8];
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        L[e] = e < E ? expf(L[e] - m) : 0.f;
-        sum += L[e];
-      }
-      float* pr = lg + r * S::LGS;  // this CTA's own row: no other CTA reads it
+      for (int q = 0; q < 8; ++q) p[q] = (e0 + q < E) ? expf(L[q] - m) : 0.f;
+      float sum = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
 #pragma unroll
-      for (int e = 0; e < EP; e += 4)
-        *reinterpret_cast<float4*>(pr + e) =
-            make_float4(L[e] / sum, L[e + 1] / sum, L[e + 2] / sum, L[e + 3] / sum);
-      float ex[kTopKMax];
-      float sk = 0.f;
+      for (int o = 1; o < G; o <<= 1) sum += __shfl_xor_sync(gmask, sum, o);
+      *reinterpret_cast<float4*>(row) = make_float4(p[0] / sum, p[1] / sum, p[2] / sum, p[3] / sum);
+      *reinterpret_cast<float4*>(row + 4) =
+          make_float4(p[4] / sum, p[5] / sum, p[6] / sum, p[7] / sum);
+      if (lane_in == 0) {
+        float ex[kMaxTopK];
+        float sk = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTopKMax; ++j) {
-        ex[j] = j < k ? expf(vals[j] - vals[0]) : 0.f;
-        sk += ex[j];
-      }
-#pragma unroll
-      for (int j = 0; j < kTopKMax; ++j)
-        if (j < k) {
-          a.idx[(size_t)t * k + j] = ids[j];
-          a.gates[(size_t)t * k + j] = ex[j] / sk;
+        for (int j = 0; j < kMaxTopK; ++j) {
+          ex[j] = j < k ? expf(vals[j] - vals[0]) : 0.f;
+          sk += ex[j];
         }
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+          if (j < k) {
+            a.idx[(size_t)t * k + j] = ids[j];
+            a.gates[(size_t)t * k + j] = ex[j] / sk;
+          }
+      }
     }
   }
   __syncthreads();
