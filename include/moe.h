@@ -109,6 +109,10 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Synchronises `stream`, then copies the workspace's device error word to
  * *code_out (0 = no device-side error since the last clear) and clears it.
+ * The word holds the first error recorded: 1 an expert index outside [0, E);
+ * 2 offsets that are not a partition of the row buffer; 3 a gathered row
+ * index (perm_token) outside [0, T); 16-19 a pipeline wait that ran out of
+ * time (TMA producer, MMA issuer, epilogue, teardown drain).
  * Returns MOE_ERR_DEVICE_CHECK if the word was non-zero, MOE_OK otherwise. */
 int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t stream);
 
@@ -179,7 +183,9 @@ int moe_route_noalloc(const moe_config_t* cfg, const void* x, const float* W_rou
  *   drop_mask    (T, top_k) uint8 out: 1 where the slot was dropped
  *   f            (E) fp32 out: counts / (T * top_k)
  *   aux_loss     (1) fp32 out: E * sum_e f_e * P_e (f before capacity)
- *   x_perm       (T * top_k, d) act_dtype out: x_perm[dest[t,j]] = x[t]
+ *   x_perm       (T * top_k, d) act_dtype out: x_perm[dest[t,j]] = x[t]; or
+ *                NULL: the rows are not copied (moe_expert_ffn_gather reads
+ *                them from x through perm_token instead)
  * Bit-exact and deterministic: no floating-point atomics, no order that
  * depends on scheduling. */
 int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
@@ -206,6 +212,27 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
 int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
                    const void* W_in, const void* W_up, const void* W_out, void* y_perm,
                    void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_expert_ffn with the permute fused into the first projection: grouped
+ * row r is token row x[perm_token[r]], read in place by TMA row gathers, so
+ * no x_perm is ever written.  [MLG Algorithm 3: each expert gathers its own
+ * tokens; the grouped layout is moe_dispatch's]
+ *   x           (T, d) act_dtype, the layer input
+ *   perm_token  (T * top_k) int32 from moe_dispatch: rows [0, offsets[E])
+ *               must hold token indices in [0, T); an index outside it is
+ *               recorded on the error word (code 3) and row 0 is used
+ *   offsets, W_in, W_up, W_out, y_perm: as for moe_expert_ffn, with the same
+ *               results (every row is bit-identical to moe_expert_ffn on the
+ *               x_perm that moe_dispatch would have gathered).
+ * Use: no (T * top_k, d) x_perm buffer is needed.  Cost: the row gathers
+ * (four 128-byte rows per TMA instruction) are repeated for every output
+ * column block of the first projection; on B200 at the Mixtral shape the
+ * experts took 10.2 ms this way against 4.8 ms on a materialised x_perm
+ * (whose copy costs about 38 us), so moe_forward gathers into x_perm. */
+int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t* perm_token,
+                          const int32_t* offsets, const void* W_in, const void* W_up,
+                          const void* W_out, void* y_perm, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
 
 /* Combine: output[t] = sum over j = 0..top_k-1 with dest[t,j] >= 0 of
  * gates[t,j] * y_perm[dest[t,j]], accumulated in fp32 in increasing j,

@@ -33,6 +33,7 @@ _SIGNATURES = {
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
     "moe_dispatch": (ctypes.c_int, [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn": (ctypes.c_int, [_c_p] * 8 + [ctypes.c_size_t, _c_p]),
+    "moe_expert_ffn_gather": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_size_t, _c_p]),
     "moe_combine": (ctypes.c_int, [_c_p] * 6),
     "moe_forward": (ctypes.c_int, [_c_p] * 15 + [ctypes.c_size_t, _c_p]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -166,6 +167,13 @@ def moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws, stream=N
     _check(load_library().moe_expert_ffn(
         ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(W_in), _ptr(W_up), _ptr(W_out),
         _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_gather(cfg, x, perm_token, offsets, W_in, W_up, W_out, y_perm, ws,
+                          stream=None) -> None:
+    _check(load_library().moe_expert_ffn_gather(
+        ctypes.byref(cfg), _ptr(x), _ptr(perm_token), _ptr(offsets), _ptr(W_in), _ptr(W_up),
+        _ptr(W_out), _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn_gather")
 
 
 def moe_combine(cfg, y_perm, dest, gates, output, stream=None) -> None:

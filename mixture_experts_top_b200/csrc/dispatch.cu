@@ -22,7 +22,9 @@
 //             chunks (chunk bases) and the total count; kept, offsets, f and
 //             aux = E * sum f_e P_e (fp64, fixed-order butterfly).
 //   scatter - one warp per token: dest, drop mask, perm_token, and the copy
-//             of x[t] into every kept grouped row with 16-byte vectors.
+//             of x[t] into every kept grouped row with 16-byte vectors
+//             (skipped when x_perm is null: the up projection then gathers
+//             the rows through perm_token itself).
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(256)
       drop_mask[s] = my_dest < 0 ? 1 : 0;
       if (my_dest >= 0) perm_token[my_dest] = t;
     }
+    if (x_perm == nullptr) continue;   // rows are gathered later, by the expert GEMM
     int dj[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) dj[j] = __shfl_sync(0xffffffffu, my_dest, j);

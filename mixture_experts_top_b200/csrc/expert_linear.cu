@@ -2,6 +2,8 @@
 //
 // "Mixture-of-Experts Routing - LLM Internals" (mlgrind.dev), Background and
 // Inputs: expert_e(x) = x @ expert_weights[e], expert_weights (E, d, d_out).
+// With a row permutation the grouped row r is read from token row perm[r]
+// (the permute fused into the operand load).
 //
 // The fp32 results must hold to 1e-4 relative, which rules out TF32 tensor
 // cores (10-bit mantissa); this is a plain fp32 FMA kernel.  Each thread
@@ -21,7 +23,8 @@ constexpr int kMaxE = 256;
 __global__ void __launch_bounds__(256)
     linear_expert_kernel(const float* __restrict__ x_perm, const int32_t* __restrict__ offsets,
                          const float* __restrict__ W, float* __restrict__ y_perm, int rows_max,
-                         int E, int d, int d_out, int32_t* err) {
+                         int E, int d, int d_out, int32_t* err,
+                         const int32_t* __restrict__ perm, int T) {
   pdl_wait_and_release();
   __shared__ int32_t off[kMaxE + 1];
   __shared__ int ok;
@@ -46,7 +49,15 @@ __global__ void __launch_bounds__(256)
       const int mid = (lo + hi) >> 1;
       if (off[mid] <= r) lo = mid; else hi = mid;
     }
-    const float* xr = x_perm + (size_t)r * d;
+    int src = r;
+    if (perm != nullptr) {
+      src = perm[r];
+      if (src < 0 || src >= T) {
+        if (n == 0) report_error(err, kDevBadPerm);
+        continue;
+      }
+    }
+    const float* xr = x_perm + (size_t)src * d;
     const float* We = W + (size_t)lo * d * d_out + n;
     float acc = 0.f;
     for (int i = 0; i < d; ++i) acc = fmaf(xr[i], We[(size_t)i * d_out], acc);
@@ -58,13 +69,13 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
                                  const int32_t* offsets, const float* W, float* y_perm,
-                                 int32_t* err, cudaStream_t s) {
+                                 int32_t* err, cudaStream_t s, const int32_t* perm) {
   const int rows_max = c.T * c.top_k;
   if (rows_max == 0) return cudaSuccess;
   const dim3 block(32, 8);
   const dim3 grid(ceil_div(c.d_out, 32), min(ceil_div(rows_max, 8), 8192));
   return launch_kernel(linear_expert_kernel, grid, block, 0, s, 0, x_perm, offsets, W, y_perm,
-                       rows_max, c.E, c.d, c.d_out, err);
+                       rows_max, c.E, c.d, c.d_out, err, perm, c.T);
 }
 
 }  // namespace moe

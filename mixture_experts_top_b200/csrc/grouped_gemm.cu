@@ -93,6 +93,8 @@ __device__ __forceinline__ uint64_t desc_b_nmajor(uint32_t saddr) {
 
 struct GemmArgs {
   const int32_t* offsets;
+  const int32_t* perm;  // gathered A: grouped row r is row perm[r] of the A tensor (else null)
+  int a_rows;           // rows of the A tensor (gathered A: tokens)
   void* out;  // bf16 for kEpiRelu / kEpiSwiglu, fp32 for kEpiNone
   int32_t* err;
   int E, K, N, rows_max;
@@ -201,7 +203,7 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
   }
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
@@ -273,8 +275,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total_tiles = tile_prefix[E];
   const int num_kb = (g.K + BK - 1) / BK;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && (GATHER || lane == 0)) {
     // ------------------------------------------------------ TMA producer
+    // Lane 0 waits for a free stage and issues the B copies (and, without
+    // GATHER, the A tile).  With GATHER every lane of warp 0 fetches 4 of the
+    // tile's 128 rows by index (grouped row m -> A row perm[m]).
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_phase = 0;
@@ -283,39 +288,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
       const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
-          report_error(g.err, kDevTimeoutProducer);
-          alive = false;
-          break;
+      int r4[4] = {0, 0, 0, 0};
+      if (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = c.m0 + 4 * lane + i;
+          int r = m < row_off[E] ? g.perm[m] : 0;   // rows past the last expert: any valid row
+          if (r < 0 || r >= g.a_rows) {
+            report_error(g.err, kDevBadPerm);
+            r = 0;
+          }
+          r4[i] = r;
         }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
         uint8_t* sa = smem + stage * STAGE_BYTES;
         uint8_t* sb = sa + A_STAGE;
         const int k0 = kb * BK;
-        mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-        tma_load_2d_hint(sa, &tmA, &full_bar[stage], k0, c.m0, keep);
-        if (EPI == kEpiSwiglu) {
-          tma_load_3d_hint(sb, &tmB0, &full_bar[stage], n0, k0, c.e, stream);
-          tma_load_3d_hint(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e, stream);
-          tma_load_3d_hint(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e, stream);
-          tma_load_3d_hint(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e, stream);
-        } else {
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait(&empty_bar[stage], phase ^ 1u);
+          if (!ok) {
+            report_error(g.err, kDevTimeoutProducer);
+          } else {
+            mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+            if (!GATHER) tma_load_2d_hint(sa, &tmA, &full_bar[stage], k0, c.m0, keep);
+            if (EPI == kEpiSwiglu) {
+              tma_load_3d_hint(sb, &tmB0, &full_bar[stage], n0, k0, c.e, stream);
+              tma_load_3d_hint(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e, stream);
+              tma_load_3d_hint(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e, stream);
+              tma_load_3d_hint(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e, stream);
+            } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tma_load_3d_hint(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e, stream);
+              for (int i = 0; i < 4; ++i)
+                tma_load_3d_hint(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e,
+                                 stream);
+            }
+            issued_mask |= 1u << stage;
+            last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+          }
         }
-        issued_mask |= 1u << stage;
-        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (GATHER) {
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (ok)
+            tma_gather4_hint(sa + lane * 4 * (BK * 2), &tmA, &full_bar[stage], k0, r4[0], r4[1],
+                             r4[2], r4[3], keep);
+        }
+        if (!ok) {
+          alive = false;
+          break;
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    // Drain: every copy this thread issued must have landed before exit.
-    for (int s = 0; s < STAGES; ++s)
-      if ((issued_mask >> s) & 1u)
-        if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(g.err, kDevTimeoutDrain);
+    // Drain: every copy issued must have landed before exit.
+    if (lane == 0)
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued_mask >> s) & 1u)
+          if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------ MMA issuer
     int stage = 0;
@@ -415,7 +448,7 @@ constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES;
 constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
@@ -488,8 +521,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total_tiles = tile_prefix[E];
   const int num_kb = (g.K + BK - 1) / BK;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && (GATHER || lane == 0)) {
     // ------------------------------------------------ TMA producer (both)
+    // As in the single-CTA kernel: lane 0 waits and issues B (and A unless
+    // GATHER); with GATHER each lane of warp 0 fetches 4 of this CTA's 128
+    // rows by index.
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_phase = 0;
@@ -502,21 +538,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // this CTA's B half: gate / up for SwiGLU, else the column halves
       const int nb = (EPI == kEpiSwiglu) ? n0 : n0 + (int)rank * (BN / 2);
       const int my_m = c.m0 + (int)rank * BM;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u)) {
-          report_error(g.err, kDevTimeoutProducer);
-          alive = false;
-          break;
+      int r4[4] = {0, 0, 0, 0};
+      if (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = my_m + 4 * lane + i;
+          int r = m < row_off[E] ? g.perm[m] : 0;   // rows past the last expert: any valid row
+          if (r < 0 || r >= g.a_rows) {
+            report_error(g.err, kDevBadPerm);
+            r = 0;
+          }
+          r4[i] = r;
         }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
         uint8_t* sa = smem + stage * P_STAGE_BYTES;
         uint8_t* sb = sa + A_STAGE;
         const int k0 = kb * BK;
-        if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-        tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, keep);
-        tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, stream);
-        tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, stream);
-        issued_mask |= 1u << stage;
-        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait(&empty_bar[stage], phase ^ 1u);
+          if (!ok) {
+            report_error(g.err, kDevTimeoutProducer);
+          } else {
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
+            if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, keep);
+            tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, stream);
+            tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, stream);
+            issued_mask |= 1u << stage;
+            last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+          }
+        }
+        if (GATHER) {
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (ok)
+            tma_gather4_pair(sa + lane * 4 * (BK * 2), &tmA, &full_bar[stage], k0, r4[0], r4[1],
+                             r4[2], r4[3], keep);
+        }
+        if (!ok) {
+          alive = false;
+          break;
+        }
         if (++stage == P_STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -524,7 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     // Drain: the leader's full barriers count both CTAs' copies.
-    if (rank == 0)
+    if (rank == 0 && lane == 0)
       for (int s = 0; s < P_STAGES; ++s)
         if ((issued_mask >> s) & 1u)
           if (!mbar_wait(&full_bar[s], (last_phase >> s) & 1u)) report_error(g.err, kDevTimeoutDrain);
@@ -607,10 +669,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // A: (rows, K) bf16 row-major, box 64 (k) x 128 (rows), 128B swizzle.
-bool encode_a(CUtensorMap* m, const void* ptr, int rows, int K) {
+// Gathered A (box_rows = 1): the box is one row high, fetched four rows at a
+// time by index.
+bool encode_a(CUtensorMap* m, const void* ptr, int rows, int K, int box_rows = BM) {
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -630,19 +694,19 @@ bool encode_b(CUtensorMap* m, const void* ptr, int E, int K, int N) {
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                      const GemmArgs& g, int grid, cudaStream_t s) {
-  auto kern = grouped_gemm_kernel<EPI>;
+  auto kern = grouped_gemm_kernel<EPI, GATHER>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, grid, NUM_THREADS, SMEM_BYTES, s, 0, a, b0, b1, g);
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                           const GemmArgs& g, int pairs, cudaStream_t s) {
-  auto kern = grouped_gemm_pair_kernel<EPI>;
+  auto kern = grouped_gemm_pair_kernel<EPI, GATHER>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), P_SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, g);
@@ -665,17 +729,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, void* out, int32_t* err,
-                                cudaStream_t s) {
+                                const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
+                                const int32_t* perm, int a_rows) {
   if (rows_max == 0) return cudaSuccess;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  const bool gather = perm != nullptr;
+  if (gather && (epi == kEpiNone || a_rows <= 0)) return cudaErrorInvalidValue;
   CUtensorMap ta, tb0, tb1;
-  if (!encode_a(&ta, A, rows_max, K) || !encode_b(&tb0, B0, E, K, N) ||
+  const bool a_ok = gather ? encode_a(&ta, A, a_rows, K, 1) : encode_a(&ta, A, rows_max, K);
+  if (!a_ok || !encode_b(&tb0, B0, E, K, N) ||
       !encode_b(&tb1, B1 != nullptr ? B1 : B0, E, K, N))
     return cudaErrorInvalidValue;
   const int out_cols = epi == kEpiSwiglu ? BN / 2 : BN;
   GemmArgs g;
   g.offsets = offsets;
+  g.perm = perm;
+  g.a_rows = gather ? a_rows : rows_max;
   g.out = out;
   g.err = err;
   g.E = E;
@@ -689,18 +758,24 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   if (rows_max >= 1024 * E) {
     const long max_pairs = (long)(ceil_div(rows_max, PBM) + E) * g.n_tiles;
     const int pairs = (int)std::min<long>((long)(device_sm_count() / 2), max_pairs);
+    if (gather)
+      return epi == kEpiSwiglu ? run_gemm_pair<kEpiSwiglu, true>(ta, tb0, tb1, g, pairs, s)
+                               : run_gemm_pair<kEpiRelu, true>(ta, tb0, tb1, g, pairs, s);
     switch (epi) {
-      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu>(ta, tb0, tb1, g, pairs, s);
-      case kEpiRelu: return run_gemm_pair<kEpiRelu>(ta, tb0, tb1, g, pairs, s);
-      default: return run_gemm_pair<kEpiNone>(ta, tb0, tb1, g, pairs, s);
+      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, g, pairs, s);
+      default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, g, pairs, s);
     }
   }
   const long max_tiles = (long)(ceil_div(rows_max, BM) + E) * g.n_tiles;
   const int grid = (int)std::min<long>((long)device_sm_count(), max_tiles);
+  if (gather)
+    return epi == kEpiSwiglu ? run_gemm<kEpiSwiglu, true>(ta, tb0, tb1, g, grid, s)
+                             : run_gemm<kEpiRelu, true>(ta, tb0, tb1, g, grid, s);
   switch (epi) {
-    case kEpiSwiglu: return run_gemm<kEpiSwiglu>(ta, tb0, tb1, g, grid, s);
-    case kEpiRelu: return run_gemm<kEpiRelu>(ta, tb0, tb1, g, grid, s);
-    default: return run_gemm<kEpiNone>(ta, tb0, tb1, g, grid, s);
+    case kEpiSwiglu: return run_gemm<kEpiSwiglu, false>(ta, tb0, tb1, g, grid, s);
+    case kEpiRelu: return run_gemm<kEpiRelu, false>(ta, tb0, tb1, g, grid, s);
+    default: return run_gemm<kEpiNone, false>(ta, tb0, tb1, g, grid, s);
   }
 }
 

@@ -91,23 +91,25 @@ T* at(void* ws, size_t off) {
 int act_bytes(const moe_config_t& c) { return c.act_dtype == MOE_BF16 ? 2 : 4; }
 
 // Up and down projections (or the linear expert) on grouped rows.
-cudaError_t run_experts(const moe_config_t& c, const void* x_perm, const int32_t* offsets,
-                        const void* W_in, const void* W_up, const void* W_out, void* y_perm,
-                        void* ws, cudaStream_t s) {
+// perm == nullptr: A is x_perm, the grouped rows.  Otherwise A is x (T, d)
+// and grouped row r is x[perm[r]].
+cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* perm,
+                        const int32_t* offsets, const void* W_in, const void* W_up,
+                        const void* W_out, void* y_perm, void* ws, cudaStream_t s) {
   const WsLayout L = workspace_layout(c);
   int32_t* err = at<int32_t>(ws, L.ctrl);
   const int rows_max = c.T * c.top_k;
   if (c.expert_kind == MOE_EXPERT_LINEAR)
-    return launch_linear_expert(c, static_cast<const float*>(x_perm), offsets,
+    return launch_linear_expert(c, static_cast<const float*>(A), offsets,
                                 static_cast<const float*>(W_in), static_cast<float*>(y_perm), err,
-                                s);
+                                s, perm);
   __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
   const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
   cudaError_t e = launch_grouped_gemm(
-      epi, static_cast<const __nv_bfloat16*>(x_perm), rows_max, c.d,
+      epi, static_cast<const __nv_bfloat16*>(A), rows_max, c.d,
       static_cast<const __nv_bfloat16*>(W_in),
       epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
-      offsets, hidden, err, s);
+      offsets, hidden, err, s, perm, c.T);
   if (e != cudaSuccess) return e;
   return launch_grouped_gemm(kEpiNone, hidden, rows_max, c.d_hidden,
                              static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
@@ -258,7 +260,6 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
     MOE_REQUIRE(dest);
     MOE_REQUIRE(perm_token);
     MOE_REQUIRE(drop_mask);
-    MOE_REQUIRE(x_perm);
   }
   MOE_ALIGNED16(x);
   MOE_ALIGNED16(x_perm);
@@ -297,9 +298,36 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* o
   MOE_ALIGNED16(x_perm);
   MOE_ALIGNED16(y_perm);
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
-  const cudaError_t e = run_experts(c, x_perm, offsets, W_in, W_up, W_out, y_perm, ws,
+  const cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws,
                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn");
+}
+
+int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t* perm_token,
+                          const int32_t* offsets, const void* W_in, const void* W_up,
+                          const void* W_out, void* y_perm, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(W_in);
+  if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
+  if (c.expert_kind != MOE_EXPERT_LINEAR) MOE_REQUIRE(W_out);
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(perm_token);
+    MOE_REQUIRE(y_perm);
+  }
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
+  MOE_ALIGNED16(x);
+  MOE_ALIGNED16(y_perm);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const cudaError_t e = run_experts(c, x, perm_token, offsets, W_in, W_up, W_out, y_perm, ws,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_gather");
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
@@ -352,18 +380,22 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   uint8_t* drop = drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask);
   int32_t* offs = at<int32_t>(ws, L.offsets);
   int32_t* dest = at<int32_t>(ws, L.dest);
+  int32_t* perm = at<int32_t>(ws, L.perm_token);
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, P,
                                nullptr, at<float>(ws, L.router_part),
                                at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl), s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/route");
-  e = launch_dispatch(c, x, expert_indices, P, cnt, offs, dest, at<int32_t>(ws, L.perm_token),
-                      drop, at<float>(ws, L.f), aux_loss, x_perm, at<int32_t>(ws, L.chunk_counts),
+  e = launch_dispatch(c, x, expert_indices, P, cnt, offs, dest, perm, drop, at<float>(ws, L.f),
+                      aux_loss, x_perm, at<int32_t>(ws, L.chunk_counts),
                       at<int32_t>(ws, L.chunk_base), at<int32_t>(ws, L.local_rank),
                       at<int32_t>(ws, L.ctrl), s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/dispatch");
-  e = run_experts(c, x_perm, offs, W_in, W_up, W_out, y_perm, ws, s);
+  // The materialised permute (one copy of each kept row, ~38 us at the
+  // Mixtral shape) is far cheaper than gathering A rows inside the GEMM,
+  // which re-fetches them for every output column block.
+  e = run_experts(c, x_perm, nullptr, offs, W_in, W_up, W_out, y_perm, ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts");
   e = launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output, s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/combine");

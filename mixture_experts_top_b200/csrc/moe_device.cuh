@@ -18,6 +18,7 @@ enum DeviceError : int32_t {
   kDevOk = 0,
   kDevBadExpertIndex = 1,     // an expert index outside [0, E)
   kDevBadOffsets = 2,         // offsets not monotone or beyond the row buffer
+  kDevBadPerm = 3,            // a gathered row index outside [0, T)
   kDevTimeoutProducer = 16,   // TMA producer gave up waiting for a free stage
   kDevTimeoutMma = 17,        // MMA issuer gave up waiting for data / accumulator
   kDevTimeoutEpilogue = 18,   // epilogue gave up waiting for an accumulator
@@ -146,6 +147,21 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Row gather: four rows (row0..row3) of a 2-D tensor whose map has a box one
+// row high, columns [c0, c0 + box width), into four consecutive box rows of
+// shared memory (the swizzle follows the destination address, as for a tiled
+// load).  The second form counts its bytes on the pair leader's mbarrier.
+__device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t c0, int32_t r0, int32_t r1, int32_t r2,
+                                                 int32_t r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3), "l"(policy)
+      : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05 --
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -259,6 +275,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_smem_addr(bar)), "r"(c0), "r"(c1),
       "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t c0, int32_t r0, int32_t r1, int32_t r2,
+                                                 int32_t r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_smem_addr(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3), "l"(policy)
       : "memory");
 }
 

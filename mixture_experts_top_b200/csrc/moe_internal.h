@@ -115,9 +115,10 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
 cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int32_t* dest,
                            const float* gates, void* out, cudaStream_t s);
 
+// perm != nullptr: grouped row r is row perm[r] of x_perm, a (T, d) tensor.
 cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
                                  const int32_t* offsets, const float* W, float* y_perm,
-                                 int32_t* err, cudaStream_t s);
+                                 int32_t* err, cudaStream_t s, const int32_t* perm = nullptr);
 
 // Grouped bf16 GEMM on tcgen05: for every expert e, rows [offsets[e],
 // offsets[e+1]) of A (rows_max, K) times B_e (K, N) -> out rows, with a fused
@@ -126,10 +127,13 @@ cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
 // one up column).
 enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2 };
 
+// perm != nullptr (ReLU / SwiGLU only): grouped row r of A is row perm[r] of
+// A, an (a_rows, K) tensor, fetched by TMA row gathers (the permute fused into
+// the up projection's operand load).
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, void* out, int32_t* err,
-                                cudaStream_t s);
+                                const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
+                                const int32_t* perm = nullptr, int a_rows = 0);
 
 // Host-side capacity: ceil(((cf * T) * k) / E) in fp64, or -1 for no limit.
 int64_t capacity_slots(float capacity_factor, int T, int k, int E);
