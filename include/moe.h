@@ -111,7 +111,8 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * *code_out (0 = no device-side error since the last clear) and clears it.
  * The word holds the first error recorded: 1 an expert index outside [0, E);
  * 2 offsets that are not a partition of the row buffer; 3 a gathered row
- * index (perm_token) outside [0, T); 16-19 a pipeline wait that ran out of
+ * index (perm_token) outside [0, T); 4 a sharded dispatch whose all_counts
+ * row for this rank is not its own counts; 16-19 a pipeline wait that ran out of
  * time (TMA producer, MMA issuer, epilogue, teardown drain).
  * Returns MOE_ERR_DEVICE_CHECK if the word was non-zero, MOE_OK otherwise. */
 int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t stream);
@@ -192,6 +193,48 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
                  const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
                  int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss,
                  void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* A batch split over `world` ranks (GPUs), each holding a contiguous block of
+ * its tokens, in rank order: rank 0 the first cfg->T tokens, and so on.  The
+ * layer's two couplings across tokens are then global: P_e and f_e (hence
+ * aux) are means over the whole batch, and a slot's position on its expert
+ * counts the earlier ranks' slots first, so the capacity keeps and drops
+ * exactly the slots the single-batch layer would.  [MLG Algorithm 3-4 and
+ * Follow-up: positions in token order, capacity from the batch size; the
+ * pages do not split a batch, so this is the single-batch rule restated]
+ *   rank, world   this rank and the number of ranks (0 <= rank < world)
+ *   T_global      tokens of the whole batch (every rank's cfg->T summed)
+ *   all_counts    (world, E) int32 device: every rank's moe_dispatch_count
+ *                 result in rank order (an all-gather of E ints per rank)
+ * prob_mean given to moe_dispatch_shard must be the whole batch's P (the
+ * token-weighted mean of the ranks' moe_route outputs: an all-reduce of E
+ * floats).  Moving these two small arrays between GPUs is the caller's
+ * (NCCL or any collective); the library keeps to one GPU. */
+typedef struct {
+  int32_t rank;
+  int32_t world;
+  int32_t T_global;
+  const int32_t* all_counts;
+} moe_shard_t;
+
+/* Per-expert slot counts of expert_indices (T, top_k) into counts (E) int32
+ * (before any capacity): this rank's contribution to all_counts. */
+int moe_dispatch_count(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* counts,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_dispatch for one rank of a sharded batch (see moe_shard_t).  Outputs
+ * as moe_dispatch, with: counts = this rank's slots per expert; offsets,
+ * dest, perm_token and x_perm describe this rank's kept rows only (its own
+ * grouped layout); drop_mask holds the whole batch's keep decision for this
+ * rank's slots (capacity = ceil(((capacity_factor * T_global) * top_k) / E),
+ * positions offset by earlier ranks' slots); f and aux_loss are the whole
+ * batch's and the same on every rank.  A rank whose row of all_counts
+ * differs from its own counts records device error 4. */
+int moe_dispatch_shard(const moe_config_t* cfg, const moe_shard_t* shard, const void* x,
+                       const int32_t* expert_indices, const float* prob_mean, int32_t* counts,
+                       int32_t* offsets, int32_t* dest, int32_t* perm_token, uint8_t* drop_mask,
+                       float* f, float* aux_loss, void* x_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
 
 /* Experts on their grouped rows: rows [offsets[e], offsets[e+1]) of x_perm
  * go through expert e and land in the same rows of y_perm.

@@ -32,6 +32,8 @@ _SIGNATURES = {
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
     "moe_dispatch": (ctypes.c_int, [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
+    "moe_dispatch_count": (ctypes.c_int, [_c_p] * 4 + [ctypes.c_size_t, _c_p]),
+    "moe_dispatch_shard": (ctypes.c_int, [_c_p] * 14 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn": (ctypes.c_int, [_c_p] * 8 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn_gather": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_size_t, _c_p]),
     "moe_combine": (ctypes.c_int, [_c_p] * 6),
@@ -53,6 +55,12 @@ class MoeConfig(ctypes.Structure):
                 ("d_out", ctypes.c_int32), ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("expert_kind", ctypes.c_int32), ("act_dtype", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float)]
+
+
+class MoeShard(ctypes.Structure):
+    """Mirror of ``moe_shard_t``: this rank of a batch split over ranks."""
+    _fields_ = [("rank", ctypes.c_int32), ("world", ctypes.c_int32), ("T_global", ctypes.c_int32),
+                ("all_counts", ctypes.c_void_p)]
 
 
 def make_config(T: int, d: int, d_hidden: int, d_out: int, E: int, top_k: int, kind: str,
@@ -161,6 +169,23 @@ def moe_dispatch(cfg, x, expert_indices, prob_mean, counts, offsets, dest, perm_
         ctypes.byref(cfg), _ptr(x), _ptr(expert_indices), _ptr(prob_mean), _ptr(counts),
         _ptr(offsets), _ptr(dest), _ptr(perm_token), _ptr(drop_mask), _ptr(f), _ptr(aux_loss),
         _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_count(cfg, expert_indices, counts, ws, stream=None) -> None:
+    _check(load_library().moe_dispatch_count(
+        ctypes.byref(cfg), _ptr(expert_indices), _ptr(counts), _ptr(ws), ws.numel(),
+        _stream(stream)), "moe_dispatch_count")
+
+
+def moe_dispatch_shard(cfg, rank, world, T_global, all_counts, x, expert_indices, prob_mean,
+                       counts, offsets, dest, perm_token, drop_mask, f, aux_loss, x_perm, ws,
+                       stream=None) -> None:
+    shard = MoeShard(rank, world, T_global, _ptr(all_counts))
+    _check(load_library().moe_dispatch_shard(
+        ctypes.byref(cfg), ctypes.byref(shard), _ptr(x), _ptr(expert_indices), _ptr(prob_mean),
+        _ptr(counts), _ptr(offsets), _ptr(dest), _ptr(perm_token), _ptr(drop_mask), _ptr(f),
+        _ptr(aux_loss), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)),
+        "moe_dispatch_shard")
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws, stream=None) -> None:

@@ -101,9 +101,13 @@ __global__ void __launch_bounds__(1024)
                          int k, int64_t cap, const float* __restrict__ prob_mean,
                          int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, float* __restrict__ f,
-                         float* __restrict__ aux) {
+                         float* __restrict__ aux, const int32_t* __restrict__ all_counts,
+                         int rank, int world, int T_global, int32_t* __restrict__ prefix,
+                         int32_t* err) {
   pdl_wait_and_release();
   __shared__ int32_t s_counts[kMaxE];
+  __shared__ int32_t s_prefix[kMaxE];   // slots of earlier ranks (sharded batch), else 0
+  __shared__ int32_t s_total[kMaxE];    // slots of the whole batch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int e = warp; e < E; e += nwarps) {
     int carry = 0;
@@ -116,13 +120,34 @@ __global__ void __launch_bounds__(1024)
     }
     if (lane == 0) s_counts[e] = carry;
   }
+  // Sharded batch: this rank's tokens follow those of ranks 0..rank-1 in
+  // the batch order, so a slot's position on its expert is offset by their
+  // slots on it; the capacity, f and aux are those of the whole batch.
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int pre = 0, tot = 0;
+    if (all_counts != nullptr) {
+      for (int r = 0; r < world; ++r) {
+        const int v = all_counts[(size_t)r * E + e];
+        if (r < rank) pre += v;
+        tot += v;
+      }
+      prefix[e] = pre;
+    }
+    s_prefix[e] = pre;
+    s_total[e] = all_counts != nullptr ? tot : 0;
+  }
   __syncthreads();
+  if (all_counts != nullptr) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      if (all_counts[(size_t)rank * E + e] != s_counts[e]) report_error(err, kDevBadShard);
+  }
   if (warp == 0) {
     int run = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       const int cnt = e < E ? s_counts[e] : 0;
-      const int kept = (cap < 0 || cnt < cap) ? cnt : (int)cap;
+      const int64_t room = cap < 0 ? (int64_t)cnt : cap - (int64_t)(e < E ? s_prefix[e] : 0);
+      const int kept = room <= 0 ? 0 : (room < cnt ? (int)room : cnt);
       const int incl = warp_inclusive_scan(kept);
       if (e < E) {
         offsets[e] = run + incl - kept;
@@ -132,10 +157,11 @@ __global__ void __launch_bounds__(1024)
     }
     if (lane == 0) offsets[E] = run;
   } else if (warp == 1) {
-    const double slots = (double)T * (double)k;
+    const bool sharded = all_counts != nullptr;
+    const double slots = (double)(sharded ? T_global : T) * (double)k;
     double acc = 0.0;
     for (int e = lane; e < E; e += 32) {
-      const double fe = slots > 0.0 ? (double)s_counts[e] / slots : 0.0;
+      const double fe = slots > 0.0 ? (double)(sharded ? s_total[e] : s_counts[e]) / slots : 0.0;
       f[e] = (float)fe;
       acc += fe * (double)prob_mean[e];
     }
@@ -153,7 +179,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ local_rank,
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ dest,
                             int32_t* __restrict__ perm_token, uint8_t* __restrict__ drop_mask,
-                            uint8_t* __restrict__ x_perm) {
+                            uint8_t* __restrict__ x_perm, const int32_t* __restrict__ prefix) {
   pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -167,7 +193,8 @@ __global__ void __launch_bounds__(256)
       const int e = idx[s];
       if (e >= 0 && e < E) {
         const int pos = chunk_base[(size_t)(t / kChunkTokens) * E + e] + local_rank[s];
-        if (cap < 0 || pos < cap) my_dest = offsets[e] + pos;
+        const int64_t gpos = (int64_t)pos + (prefix != nullptr ? prefix[e] : 0);
+        if (cap < 0 || gpos < cap) my_dest = offsets[e] + pos;
       }
       dest[s] = my_dest;
       drop_mask[s] = my_dest < 0 ? 1 : 0;
@@ -196,24 +223,56 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             const float* prob_mean, int32_t* counts, int32_t* offsets,
                             int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
-                            int32_t* local_rank, int32_t* err, cudaStream_t s) {
+                            int32_t* local_rank, int32_t* err, cudaStream_t s,
+                            const ShardInfo* shard, int32_t* shard_prefix) {
   const int nchunks = ceil_div(c.T, kChunkTokens);
-  const int64_t cap = capacity_slots(c.capacity_factor, c.T, c.top_k, c.E);
+  const int64_t cap = capacity_slots(c.capacity_factor, shard != nullptr ? shard->T_global : c.T,
+                                     c.top_k, c.E);
   if (nchunks > 0) {
     cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
                                   c.T, c.top_k, c.E, chunk_counts, local_rank, err);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = launch_kernel(dispatch_scan_kernel, 1, 1024, 0, s, 0, chunk_counts, nchunks,
-                                c.E, c.T, c.top_k, cap, prob_mean, chunk_base, counts, offsets,
-                                f, aux);
+  cudaError_t e = launch_kernel(
+      dispatch_scan_kernel, 1, 1024, 0, s, 0, chunk_counts, nchunks, c.E, c.T, c.top_k, cap,
+      prob_mean, chunk_base, counts, offsets, f, aux,
+      shard != nullptr ? shard->all_counts : nullptr, shard != nullptr ? shard->rank : 0,
+      shard != nullptr ? shard->world : 1, shard != nullptr ? shard->T_global : c.T,
+      shard != nullptr ? shard_prefix : nullptr, err);
   if (e != cudaSuccess || c.T == 0) return e;
   const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
   return launch_kernel(elem == 2 ? dispatch_scatter_kernel<2> : dispatch_scatter_kernel<4>, blocks,
                        256, 0, s, 0, static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d,
                        cap, chunk_base, local_rank, offsets, dest, perm_token, drop_mask,
-                       static_cast<uint8_t*>(x_perm));
+                       static_cast<uint8_t*>(x_perm),
+                       shard != nullptr ? (const int32_t*)shard_prefix : nullptr);
+}
+
+// Slots per expert of these expert indices (the histogram every rank of a
+// sharded batch contributes before the sharded dispatch).
+__global__ void __launch_bounds__(256)
+    dispatch_total_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                          int32_t* __restrict__ counts) {
+  pdl_wait_and_release();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int v = 0;
+    for (int c = 0; c < nchunks; ++c) v += chunk_counts[(size_t)c * E + e];
+    counts[e] = v;
+  }
+}
+
+cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int32_t* counts,
+                                  int32_t* chunk_counts, int32_t* local_rank, int32_t* err,
+                                  cudaStream_t s) {
+  const int nchunks = ceil_div(c.T, kChunkTokens);
+  if (nchunks > 0) {
+    cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
+                                  c.T, c.top_k, c.E, chunk_counts, local_rank, err);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_kernel(dispatch_total_kernel, 1, 256, 0, s, 0, chunk_counts, nchunks, c.E,
+                       counts);
 }
 
 }  // namespace moe

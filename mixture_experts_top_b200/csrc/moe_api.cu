@@ -137,6 +137,7 @@ WsLayout workspace_layout(const moe_config_t& c) {
   L.prob_mean = take(E * 4);
   L.chunk_counts = take(n_chunks * E * 4);
   L.chunk_base = take(n_chunks * E * 4);
+  L.shard_prefix = take(E * 4);
   L.local_rank = take(Tk * 4);
   L.counts = take(E * 4);
   L.offsets = take((E + 1) * 4);
@@ -247,10 +248,15 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
 }
 
-int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
-                 const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
-                 int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss, void* x_perm,
-                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x,
+                   const int32_t* expert_indices, const float* prob_mean, int32_t* counts,
+                   int32_t* offsets, int32_t* dest, int32_t* perm_token, uint8_t* drop_mask,
+                   float* f, float* aux_loss, void* x_perm, void* ws, size_t ws_bytes,
+                   moe_stream_t stream, const char* name) {
   int st = check_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config_t& c = *cfg;
@@ -268,14 +274,65 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
   MOE_REQUIRE(offsets);
   MOE_REQUIRE(f);
   MOE_REQUIRE(aux_loss);
+  ShardInfo shard{};
+  if (sh != nullptr) {
+    if (sh->world < 1 || sh->rank < 0 || sh->rank >= sh->world)
+      return fail(MOE_ERR_INVALID_ARG, "shard: need 0 <= rank < world");
+    if (sh->T_global < c.T || (int64_t)sh->T_global * c.top_k >= ((int64_t)1 << 31))
+      return fail(MOE_ERR_INVALID_ARG, "shard: need T <= T_global and T_global * top_k < 2^31");
+    if (sh->all_counts == nullptr) return fail(MOE_ERR_INVALID_ARG, "shard->all_counts is NULL");
+    shard = ShardInfo{sh->rank, sh->world, sh->T_global, sh->all_counts};
+  }
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = workspace_layout(c);
   const cudaError_t e = launch_dispatch(
       c, x, expert_indices, prob_mean, counts, offsets, dest, perm_token, drop_mask, f, aux_loss,
       x_perm, at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
       at<int32_t>(ws, L.local_rank), at<int32_t>(ws, L.ctrl),
-      reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch");
+      reinterpret_cast<cudaStream_t>(stream), sh != nullptr ? &shard : nullptr,
+      at<int32_t>(ws, L.shard_prefix));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, name);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
+                 const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
+                 int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss, void* x_perm,
+                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return dispatch_entry(cfg, nullptr, x, expert_indices, prob_mean, counts, offsets, dest,
+                        perm_token, drop_mask, f, aux_loss, x_perm, ws, ws_bytes, stream,
+                        "moe_dispatch");
+}
+
+int moe_dispatch_count(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* counts,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) MOE_REQUIRE(expert_indices);
+  MOE_REQUIRE(counts);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_dispatch_count(c, expert_indices, counts,
+                                              at<int32_t>(ws, L.chunk_counts),
+                                              at<int32_t>(ws, L.local_rank),
+                                              at<int32_t>(ws, L.ctrl),
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch_count");
+}
+
+int moe_dispatch_shard(const moe_config_t* cfg, const moe_shard_t* shard, const void* x,
+                       const int32_t* expert_indices, const float* prob_mean, int32_t* counts,
+                       int32_t* offsets, int32_t* dest, int32_t* perm_token, uint8_t* drop_mask,
+                       float* f, float* aux_loss, void* x_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  if (shard == nullptr) return fail(MOE_ERR_INVALID_ARG, "shard is NULL");
+  return dispatch_entry(cfg, shard, x, expert_indices, prob_mean, counts, offsets, dest,
+                        perm_token, drop_mask, f, aux_loss, x_perm, ws, ws_bytes, stream,
+                        "moe_dispatch_shard");
 }
 
 int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,

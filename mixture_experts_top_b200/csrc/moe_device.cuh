@@ -19,6 +19,7 @@ enum DeviceError : int32_t {
   kDevBadExpertIndex = 1,     // an expert index outside [0, E)
   kDevBadOffsets = 2,         // offsets not monotone or beyond the row buffer
   kDevBadPerm = 3,            // a gathered row index outside [0, T)
+  kDevBadShard = 4,           // this rank's row of all_counts differs from its own counts
   kDevTimeoutProducer = 16,   // TMA producer gave up waiting for a free stage
   kDevTimeoutMma = 17,        // MMA issuer gave up waiting for data / accumulator
   kDevTimeoutEpilogue = 18,   // epilogue gave up waiting for an accumulator

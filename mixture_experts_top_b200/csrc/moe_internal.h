@@ -29,6 +29,7 @@ struct WsLayout {
   size_t prob_mean;      // (E) fp32, moe_forward only
   size_t chunk_counts;   // (chunks, E) int32
   size_t chunk_base;     // (chunks, E) int32
+  size_t shard_prefix;   // (E) int32: earlier ranks' slots per expert (sharded batch)
   size_t local_rank;     // (T*k) int32 position of a slot inside its chunk
   size_t counts;         // (E) int32           -- moe_forward intermediates
   size_t offsets;        // (E+1) int32
@@ -106,11 +107,23 @@ cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const
                             float* logits_out, float* router_part, __nv_bfloat16* w_split,
                             int32_t* err, cudaStream_t s, int* tiles_out);
 
+// A batch split over `world` ranks in contiguous token blocks, rank order:
+// every rank's per-expert slot counts (world, E) on the device, and the
+// whole batch's token count.
+struct ShardInfo {
+  int rank, world, T_global;
+  const int32_t* all_counts;
+};
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* idx,
                             const float* prob_mean, int32_t* counts, int32_t* offsets,
                             int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
-                            int32_t* local_rank, int32_t* err, cudaStream_t s);
+                            int32_t* local_rank, int32_t* err, cudaStream_t s,
+                            const ShardInfo* shard = nullptr, int32_t* shard_prefix = nullptr);
+// The per-expert slot counts of `idx` (T, top_k) into counts (E).
+cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int32_t* counts,
+                                  int32_t* chunk_counts, int32_t* local_rank, int32_t* err,
+                                  cudaStream_t s);
 
 cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int32_t* dest,
                            const float* gates, void* out, cudaStream_t s);
