@@ -131,6 +131,32 @@ def test_workspace_holds_the_split_router_weights(moe_lib):
     assert nb > 0
 
 
+def test_shard_and_gather_argument_checks(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    outs = [FAKE] * 7                      # counts, offsets, dest, perm, drop, f, aux
+    st = moe_lib.moe_dispatch_shard(ctypes.byref(cfg), None, FAKE, FAKE, FAKE, *outs, FAKE,
+                                    FAKE, ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "shard" in moe_lib.moe_last_error_message().decode()
+    for rank, world, T_g, counts in [(2, 2, 128, FAKE), (-1, 2, 128, FAKE), (0, 0, 128, FAKE),
+                                     (0, 2, 32, FAKE), (0, 2, 128, None)]:
+        sh = api.MoeShard(rank, world, T_g, counts)
+        st = moe_lib.moe_dispatch_shard(ctypes.byref(cfg), ctypes.byref(sh), FAKE, FAKE, FAKE,
+                                        *outs, FAKE, FAKE, ws, None)
+        assert st == api.MOE_ERR_INVALID_ARG, (rank, world, T_g)
+    assert moe_lib.moe_dispatch_count(ctypes.byref(cfg), FAKE, None, FAKE, ws, None) == \
+        api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_dispatch_count(ctypes.byref(cfg), FAKE, FAKE, FAKE, ws - 1, None) == \
+        api.MOE_ERR_WORKSPACE
+    # gather: perm_token required, x aligned
+    st = moe_lib.moe_expert_ffn_gather(ctypes.byref(cfg), FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, FAKE, ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "perm_token" in moe_lib.moe_last_error_message().decode()
+    st = moe_lib.moe_expert_ffn_gather(ctypes.byref(cfg), FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, FAKE, ws, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "16-byte" in moe_lib.moe_last_error_message().decode()
+
+
 def test_swiglu_needs_three_matrices(moe_lib):
     cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
     ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
