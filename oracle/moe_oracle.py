@@ -20,6 +20,8 @@ sides.  Pages cited (title, then section):
   rate limit" (capacity, first come first served, dropped tokens give 0).
 * [EB] "Sparsely-gated Mixture of Experts (MoE)" (Eli Bendersky's website):
   "A Minimal Numpy Implementation" (ReLU feed-forward expert, Wh/Wo).
+* Philox4x64-10: Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+  easy as 1, 2, 3" (SC 2011), for the noisy gate's draws.
 
 Readings taken where the pages are silent or disagree are listed in the
 repository's design notes; the ones that shape code are repeated at the step.
@@ -36,6 +38,65 @@ from typing import Optional
 import numpy as np
 
 KINDS = ("linear", "relu", "swiglu")
+
+
+# ----------------------------------------------------------------------------
+# noisy gating drawn from a counter-based generator
+# ----------------------------------------------------------------------------
+# [PFD The code, `router`] adds noise to the logits; the noisy top-k gate it
+# names draws, per token and expert, a standard normal scaled by
+# softplus(x @ W_noise).  The draw comes from Philox4x64-10 (Salmon, Moraes,
+# Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
+# implemented here from that definition with Python integers, and two of its
+# words become one normal by the Box-Muller transform.
+
+PHILOX_M = (0xD2E7470EE14C6C93, 0xCA5A826395121157)   # round multipliers, 4x64
+PHILOX_W = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)   # key increments (Weyl)
+_U64 = (1 << 64) - 1
+
+
+def philox4x64(counter, key, rounds: int = 10):
+    """Philox4x64-`rounds` of a 4-word counter under a 2-word key."""
+    x0, x1, x2, x3 = (int(v) & _U64 for v in counter)
+    k0, k1 = (int(v) & _U64 for v in key)
+    for r in range(rounds):
+        if r > 0:
+            k0 = (k0 + PHILOX_W[0]) & _U64
+            k1 = (k1 + PHILOX_W[1]) & _U64
+        p0 = PHILOX_M[0] * x0
+        p1 = PHILOX_M[1] * x2
+        x0, x1, x2, x3 = ((p1 >> 64) ^ x1 ^ k0, p1 & _U64, (p0 >> 64) ^ x3 ^ k1, p0 & _U64)
+    return x0, x1, x2, x3
+
+
+def gate_normal(seed: int, offset: int, t: int, e: int) -> float:
+    """The standard normal of token t (its index in the whole batch) and
+    expert e: Philox4x64-10 of the counter (t, e, offset, 0) under the key
+    (seed, 0); its first two words w0, w1 give u = ((w >> 11) + 1/2) / 2^53
+    in (0, 1), and z = sqrt(-2 ln u0) cos(2 pi u1), in fp64."""
+    w = philox4x64((t, e, offset, 0), (seed, 0))
+    u0 = ((w[0] >> 11) + 0.5) * 2.0 ** -53
+    u1 = ((w[1] >> 11) + 0.5) * 2.0 ** -53
+    return math.sqrt(-2.0 * math.log(u0)) * math.cos(2.0 * math.pi * u1)
+
+
+def softplus(v: np.ndarray) -> np.ndarray:
+    """log(1 + exp(v)), written as max(v, 0) + log1p(exp(-|v|)) (no overflow)."""
+    v = np.asarray(v, np.float64)
+    return np.maximum(v, 0.0) + np.log1p(np.exp(-np.abs(v)))
+
+
+def gate_noise(x: np.ndarray, W_noise: np.ndarray, dtype: str, seed: int, offset: int,
+               token_base: int = 0) -> np.ndarray:
+    """(T, E) fp32 noise: z(t, e) * softplus(l_te) with l = x @ W_noise the
+    fp32 noise logits (fp64 dot, rounded to fp32 like the router logits) and
+    the product rounded to fp32 once.  Token t of this call is token
+    token_base + t of the batch."""
+    L = (widen(x, dtype) @ np.asarray(W_noise, np.float64)).astype(np.float32).astype(np.float64)
+    T, E = L.shape
+    z = np.array([[gate_normal(seed, offset, token_base + t, e) for e in range(E)]
+                  for t in range(T)], np.float64).reshape(T, E)
+    return (z * softplus(L)).astype(np.float32)
 
 
 # ----------------------------------------------------------------------------
