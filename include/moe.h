@@ -140,6 +140,31 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
               int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,
               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The noisy gate's noise, drawn on the device: noise_out[t, e] =
+ * z(token_base + t, e) * softplus((x @ W_noise)[t, e]), to pass as moe_route's
+ * or moe_forward's `noise`.  [PFD The code, `router`: noise added to the
+ * logits; the noisy top-k gate: a standard normal scaled by
+ * softplus(x @ W_noise)]
+ *   x          (T, d) bf16 (this call supports bf16 activations, E <= 64)
+ *   W_noise    (d, E) fp32 row-major
+ *   seed, offset  the draws are Philox4x64-10 (Salmon et al., SC 2011) of the
+ *              counter (token, e, offset, 0) under the key (seed, 0); two
+ *              64-bit words give u = ((w >> 11) + 1/2) / 2^53 in (0, 1) and
+ *              z = sqrt(-2 ln u0) cos(2 pi u1) (Box-Muller, fp64).  Change
+ *              `offset` (e.g. a step counter) for fresh noise; the same
+ *              (seed, offset) always gives the same noise.
+ *   token_base index of this call's first token in the whole batch (0 for a
+ *              single batch; a rank's first token for a sharded one), so a
+ *              sharded batch draws exactly the single batch's noise.
+ *   noise_out  (T, E) fp32 out.
+ * The noise logits are fp32 (the tensor-core contraction of moe_route, with
+ * W_noise split exactly into three bf16 terms); softplus and the product
+ * are fp64, rounded once to fp32.  Uses the workspace's split-weight area
+ * (so not concurrently with moe_route on the same workspace). */
+int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise, uint64_t seed,
+                   uint64_t offset, int64_t token_base, float* noise_out, void* ws,
+                   size_t ws_bytes, moe_stream_t stream);
+
 /* moe_route without a workspace.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for
  * example a plugin running inside a host program whose memory pool owns the

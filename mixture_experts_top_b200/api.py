@@ -31,6 +31,9 @@ _SIGNATURES = {
     "moe_device_status": (ctypes.c_int, [_c_p, ctypes.c_size_t, _c_p, _c_p]),
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
+    "moe_gate_noise": (ctypes.c_int, [_c_p] * 3 + [ctypes.c_uint64, ctypes.c_uint64,
+                                                   ctypes.c_int64, _c_p, _c_p, ctypes.c_size_t,
+                                                   _c_p]),
     "moe_dispatch": (ctypes.c_int, [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "moe_dispatch_count": (ctypes.c_int, [_c_p] * 4 + [ctypes.c_size_t, _c_p]),
     "moe_dispatch_shard": (ctypes.c_int, [_c_p] * 14 + [ctypes.c_size_t, _c_p]),
@@ -161,6 +164,12 @@ def moe_route_noalloc(cfg, x, W_router, logit_bias, noise, expert_indices, gates
         ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
         _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _stream(stream)),
         "moe_route_noalloc")
+
+
+def moe_gate_noise(cfg, x, W_noise, seed, offset, token_base, noise_out, ws, stream=None) -> None:
+    _check(load_library().moe_gate_noise(
+        ctypes.byref(cfg), _ptr(x), _ptr(W_noise), int(seed), int(offset), int(token_base),
+        _ptr(noise_out), _ptr(ws), ws.numel(), _stream(stream)), "moe_gate_noise")
 
 
 def moe_dispatch(cfg, x, expert_indices, prob_mean, counts, offsets, dest, perm_token, drop_mask,

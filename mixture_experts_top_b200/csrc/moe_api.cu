@@ -298,6 +298,30 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
 
 extern "C" {
 
+int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise, uint64_t seed,
+                   uint64_t offset, int64_t token_base, float* noise_out, void* ws,
+                   size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (router_tc_width(c) == 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_gate_noise: bf16 activations and E <= 64 only");
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(noise_out);
+  }
+  MOE_REQUIRE(W_noise);
+  MOE_ALIGNED16(x);
+  if (token_base < 0) return fail(MOE_ERR_INVALID_ARG, "token_base must be >= 0");
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_gate_noise(
+      c, static_cast<const __nv_bfloat16*>(x), W_noise, seed, offset, (long long)token_base,
+      noise_out, at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl),
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_gate_noise");
+}
+
 int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
                  const float* prob_mean, int32_t* counts, int32_t* offsets, int32_t* dest,
                  int32_t* perm_token, uint8_t* drop_mask, float* f, float* aux_loss, void* x_perm,

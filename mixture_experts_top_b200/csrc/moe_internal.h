@@ -100,6 +100,12 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_ro
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
                          __nv_bfloat16* w_split, int32_t* err, cudaStream_t s);
+// The noisy gate's noise (router_tc.cu): noise_out (T, E) fp32 =
+// z(token_base + t, e) * softplus(x @ W_noise); bf16 x and E <= 64 only.
+cudaError_t launch_gate_noise(const moe_config_t& c, const __nv_bfloat16* x, const float* W_noise,
+                              uint64_t seed, uint64_t offset, long long token_base,
+                              float* noise_out, __nv_bfloat16* w_split, int32_t* err,
+                              cudaStream_t s);
 // Tensor-core router (router_tc.cu): logits, softmax, top-k, gates and one
 // row of probability column sums per 128-token tile; *tiles_out = rows.
 cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W_router,

@@ -147,7 +147,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-template <int EP>
+// LOGITS_ONLY: the contraction and the rank-ordered sum only, written to
+// a.logits_out (the noisy gate's noise logits); no top-k, gates or sums.
+template <int EP, bool LOGITS_ONLY>
 __global__ void __launch_bounds__(TTHREADS, 2)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const TcArgs a) {
@@ -350,6 +352,7 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   }
   __syncthreads();
 
+  if (LOGITS_ONLY) goto teardown;
   // ------------------------------ finishing, a group of G lanes per token
   // Each lane of a group holds 8 consecutive experts' logits.  Top-k: k
   // rounds of a group-wide maximum of 64-bit keys (order-preserving logit
@@ -449,7 +452,8 @@ __global__ void __launch_bounds__(TTHREADS, 2)
     for (int sp = 0; sp < nsplit; ++sp) v += cluster.map_shared_rank(csum, sp)[threadIdx.x];
     a.part[(size_t)tile * E + threadIdx.x] = v;
   }
-  cluster.sync();  // peers keep their shared memory until rank 0 has read it
+teardown:
+  cluster.sync();  // peers keep their shared memory until every read of it is done
 
   if (warp == 1) {
     tc_fence_after_sync();
@@ -479,7 +483,7 @@ bool encode_bf16(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* di
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EP>
+template <int EP, bool LOGITS_ONLY = false>
 cudaError_t run_router_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W,
                           const TcArgs& a, __nv_bfloat16* w_split, cudaStream_t s, int* tiles_out) {
   using S = TcShape<EP>;
@@ -499,7 +503,7 @@ cudaError_t run_router_tc(const moe_config_t& c, const __nv_bfloat16* x, const f
   const int tiles = ceil_div(c.T, TBM);
   const int nsplit = tc_splits(tiles, chunks);
   *tiles_out = tiles;
-  auto kern = router_tc_kernel<EP>;
+  auto kern = router_tc_kernel<EP, LOGITS_ONLY>;
   e = ensure_smem_limit(reinterpret_cast<const void*>(kern), S::SMEM);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, tiles * nsplit, TTHREADS, S::SMEM, s, nsplit, tx, tw, a);
@@ -519,6 +523,79 @@ cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const
     case 64: return run_router_tc<64>(c, x, W_router, a, w_split, s, tiles_out);
     default: return cudaErrorInvalidValue;
   }
+}
+
+namespace {
+
+// Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): ten rounds over a 4-word counter, the key
+// advanced by the two Weyl constants between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
+  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
+    const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
+    const uint64_t y0 = hi1 ^ x[1] ^ k0, y2 = hi0 ^ x[3] ^ k1;
+    x[0] = y0;
+    x[1] = lo1;
+    x[2] = y2;
+    x[3] = lo0;
+  }
+}
+
+// In place: noise logits l (T, E) -> z(t, e) * softplus(l), z the standard
+// normal of the batch token token_base + t and expert e: Philox4x64-10 of the
+// counter (token, e, offset, 0) under the key (seed, 0), two words to
+// u = ((w >> 11) + 1/2) 2^-53 and z = sqrt(-2 ln u0) cos(2 pi u1) in fp64;
+// softplus(l) = max(l, 0) + log1p(exp(-|l|)) in fp64; one rounding to fp32.
+__global__ void __launch_bounds__(256)
+    gate_noise_kernel(float* __restrict__ buf, long long n, int E, uint64_t seed, uint64_t offset,
+                      long long token_base) {
+  pdl_wait_and_release();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long t = i / E;
+    const int e = (int)(i - t * E);
+    uint64_t w[4] = {(uint64_t)(t + token_base), (uint64_t)e, offset, 0ull};
+    philox4x64_10(w, seed, 0ull);
+    const double u0 = ((double)(w[0] >> 11) + 0.5) * 0x1.0p-53;
+    const double u1 = ((double)(w[1] >> 11) + 0.5) * 0x1.0p-53;
+    const double z = sqrt(-2.0 * log(u0)) * cos(2.0 * 3.141592653589793 * u1);
+    const double l = (double)buf[i];
+    const double sp = fmax(l, 0.0) + log1p(exp(-fabs(l)));
+    buf[i] = (float)(z * sp);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gate_noise(const moe_config_t& c, const __nv_bfloat16* x, const float* W_noise,
+                              uint64_t seed, uint64_t offset, long long token_base,
+                              float* noise_out, __nv_bfloat16* w_split, int32_t* err,
+                              cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  const TcArgs a{nullptr, nullptr, nullptr, nullptr, noise_out, nullptr, err, c.T, c.d, c.E,
+                 c.top_k};
+  int tiles = 0;
+  cudaError_t e;
+  switch (router_tc_width(c)) {
+    case 16: e = run_router_tc<16, true>(c, x, W_noise, a, w_split, s, &tiles); break;
+    case 32: e = run_router_tc<32, true>(c, x, W_noise, a, w_split, s, &tiles); break;
+    case 64: e = run_router_tc<64, true>(c, x, W_noise, a, w_split, s, &tiles); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  const long long n = (long long)c.T * c.E;
+  const int blocks = (int)std::min<long long>((n + 255) / 256, (long long)device_sm_count() * 8);
+  return launch_kernel(gate_noise_kernel, blocks, 256, 0, s, 0, noise_out, n, c.E, seed, offset,
+                       token_base);
 }
 
 }  // namespace moe

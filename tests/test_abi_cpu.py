@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 14
+    assert len(names) == 15
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -155,6 +155,21 @@ def test_shard_and_gather_argument_checks(moe_lib):
     st = moe_lib.moe_expert_ffn_gather(ctypes.byref(cfg), FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE,
                                        FAKE, FAKE, ws, None)
     assert st == api.MOE_ERR_INVALID_ARG and "16-byte" in moe_lib.moe_last_error_message().decode()
+
+
+def test_gate_noise_argument_checks(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    assert moe_lib.moe_gate_noise(ctypes.byref(cfg), FAKE, None, 1, 0, 0, FAKE, FAKE, ws,
+                                  None) == api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_gate_noise(ctypes.byref(cfg), FAKE, FAKE, 1, 0, -1, FAKE, FAKE, ws,
+                                  None) == api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_gate_noise(ctypes.byref(cfg), FAKE + 8, FAKE, 1, 0, 0, FAKE, FAKE, ws,
+                                  None) == api.MOE_ERR_INVALID_ARG
+    wide = api.make_config(64, 64, 128, 64, 100, 2, "swiglu", "bf16")     # E > 64
+    ws2 = moe_lib.moe_workspace_size(ctypes.byref(wide))
+    assert moe_lib.moe_gate_noise(ctypes.byref(wide), FAKE, FAKE, 1, 0, 0, FAKE, FAKE, ws2,
+                                  None) == api.MOE_ERR_UNSUPPORTED
 
 
 def test_swiglu_needs_three_matrices(moe_lib):
