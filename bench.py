@@ -113,6 +113,20 @@ def profiled_traffic(kernel_file: str, summary: str):
     return float(m_b.group(1))
 
 
+def launches_per_step(w, cfg) -> int:
+    """Kernels of this library launched by one timed step (route, dispatch,
+    experts, combine), as the library picks them for this configuration:
+    route = weight split + tensor-core router + P mean (bf16, E <= 64) or
+    SIMT router + P mean; dispatch = count + scan + scatter; experts = up and
+    down GEMM (bf16) or the fp32 linear kernel; combine = 1."""
+    from mixture_experts_top_b200 import api as _api
+    if w.T == 0:
+        return 2                       # P mean and the dispatch scan only
+    route = 3 if _api.router_tc_width_supported(cfg) else 2
+    experts = 1 if w.kind == "linear" else 2
+    return route + 3 + experts + 1
+
+
 # ------------------------------------------------------------- ranks (N>1) --
 
 def rank_token_seed(rank: int) -> int:
@@ -237,6 +251,7 @@ def run_ours(args, rank, world):
 
     x, Wr, bias, noise = dev(inp["x"]), dev(inp["W_router"]), dev(inp["logit_bias"]), dev(inp["noise"])
     W_in, W_up, W_out = dev(inp["W_in"]), dev(inp["W_up"]), dev(inp["W_out"])
+    W_noise = dev(inp["W_noise"])
     del inp
     cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
                           w.capacity_factor)
@@ -371,6 +386,28 @@ def run_ours(args, rank, world):
     if rank != 0:
         return 0
 
+    # The noisy gate's noise made on the device (moe_gate_noise), timed on
+    # its own: the workload recipe hands the router a host-made noise tensor,
+    # so this is not part of the step above.
+    extras = {}
+    if W_noise is not None and api.router_tc_width_supported(cfg):
+        noise_dev = torch.empty((T, E), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            api.moe_gate_noise(cfg, x, W_noise, 7, 0, 0, noise_dev, ws)
+        n_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        reps = 20
+        n_ev[0].record(stream)
+        for i in range(reps):
+            api.moe_gate_noise(cfg, x, W_noise, 7, i, 0, noise_dev, ws)
+        n_ev[1].record(stream)
+        torch.cuda.synchronize()
+        us = n_ev[0].elapsed_time(n_ev[1]) / reps * 1e3
+        nb = T * w.d * 2 + w.d * E * 4 + T * E * 4
+        extras["gate_noise"] = {"us": us, "GB/s": nb / us / 1e3,
+                                "frac_hbm": nb / us / 1e3 / peaks["hbm_gbs"],
+                                "note": "moe_gate_noise at this shape (x read, W_noise read, "
+                                        "(T,E) fp32 noise written), back to back, x in L2"}
+
     counts = o.counts.cpu().numpy()
     rows = A.kept_rows(counts, w.capacity_factor, T, k)
     used = int((counts > 0).sum())
@@ -435,12 +472,13 @@ def run_ours(args, rank, world):
         "config": workload_config(w, world),
         "roofline": gemm,
         "stages": stages,
+        **({"extras": extras} if extras else {}),
         "e2e": {"value": job_value(world, T, e2e_ms / args.steps), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "moe_forward via the Python binding; every step copies x from pinned host "
                        "memory and output + aux_loss back to pinned host memory, on copy "
                        "streams overlapped with the previous/next step's compute"},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": launches_per_step(w, cfg) * args.steps,
         "clocks": clk,
         "routing": {"rows": rows, "used_experts": used, "aux_loss": float(o.aux_loss.item())},
     }

@@ -72,6 +72,12 @@ def make_config(T: int, d: int, d_hidden: int, d_out: int, E: int, top_k: int, k
                      float(capacity_factor))
 
 
+def router_tc_width_supported(cfg: "MoeConfig") -> bool:
+    """Whether the tensor-core router (and moe_gate_noise) serves `cfg`:
+    bf16 activations and at most 64 experts."""
+    return cfg.act_dtype == DTYPES["bf16"] and cfg.E <= 64
+
+
 _lib = None
 
 

@@ -133,7 +133,8 @@ def make_inputs(w: Workload, seed: int = 0, with_experts: bool = True) -> dict:
     """All inputs of one forward pass of workload ``w``.
 
     Keys: x (T,d), W_router (d,E) fp32, logit_bias (E,) fp32 or None,
-    noise (T,E) fp32 or None, W_in / W_up / W_out (E, in, out) or None.
+    noise (T,E) fp32 or None and the W_noise (d,E) fp32 it was made with,
+    W_in / W_up / W_out (E, in, out) or None.
     Activations and expert weights are uint16 bf16 bits for bf16 workloads,
     fp32 otherwise.
     """
@@ -154,6 +155,7 @@ def make_inputs(w: Workload, seed: int = 0, with_experts: bool = True) -> dict:
         softplus = np.logaddexp(0.0, s)
         noise = (z * softplus).astype(np.float32)
     inputs = dict(x=x, W_router=W_router, logit_bias=bias, noise=noise,
+                  W_noise=W_noise if w.noise else None,
                   W_in=None, W_up=None, W_out=None)
     if with_experts:
         per = [make_expert_weights(w, seed, e) for e in range(w.E)]
