@@ -132,9 +132,10 @@ int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t
  * bias and then the noise are each added in fp32.  With bf16 x and E <= 64
  * the dot product runs on the tensor cores: W_router is split exactly into
  * three bf16 terms (hi + mid + lo), so every product x_i * W_part is exact in
- * fp32 and the tensor core's fp32 accumulator adds them; the workspace holds
- * the split (3 * EP * d bf16, EP = E rounded up to 16, 32 or 64).  Otherwise
- * the fp32 pipes compute it. */
+ * fp32; the tensor core's fp32 accumulator sums one 64-wide block of d at a
+ * time and the blocks are added in round-to-nearest fp32.  The workspace
+ * holds the split (3 * EP * d bf16, EP = E rounded up to 16, 32 or 64).
+ * Otherwise the fp32 pipes compute it. */
 int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
               const float* logit_bias, const float* noise,
               int32_t* expert_indices, float* gates, float* prob_mean, float* logits_out,

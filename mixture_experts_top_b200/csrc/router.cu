@@ -9,10 +9,14 @@
 // code, `router`: an optional per-expert bias, then optional noise, are added
 // to the logits before the softmax and the top-k.
 //
+// This fp32 SIMT kernel serves fp32 tokens, more than 64 experts and
+// moe_route_noalloc; bf16 tokens with E <= 64 take the tensor-core router of
+// router_tc.cu (launch_route below picks).
+//
 // Design (B200): a thread-block cluster of S CTAs (S = 1..8) owns a tile of
 // 32 or 64 tokens; each CTA of the cluster takes 1/S of the contraction
 // range d.  The contraction x (tile, d/S) @ W (d/S, E) runs on the fp32 pipes
-// (fp32 logits are required, so no tensor cores): x and W stream through
+// (fp32 tokens have no exact bf16 tensor-core form): x and W stream through
 // shared memory in k chunks with a multi-stage cp.async pipeline; each lane
 // owns TM tokens and TN experts, so W values are warp-wide broadcasts and x
 // rows are read as conflict-free 16-byte vectors (rows padded by 16 bytes).
