@@ -112,7 +112,8 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * The word holds the first error recorded: 1 an expert index outside [0, E);
  * 2 offsets that are not a partition of the row buffer; 3 a gathered row
  * index (perm_token) outside [0, T); 4 a sharded dispatch whose all_counts
- * row for this rank is not its own counts; 16-19 a pipeline wait that ran out of
+ * row for this rank is not its own counts; 20 moe_check_wait_timeout's
+ * intended timeout; 16-19 a pipeline wait that ran out of
  * time (TMA producer, MMA issuer, epilogue, teardown drain).
  * Returns MOE_ERR_DEVICE_CHECK if the word was non-zero, MOE_OK otherwise. */
 int moe_device_status(void* ws, size_t ws_bytes, int32_t* code_out, moe_stream_t stream);
@@ -165,6 +166,17 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
 int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise, uint64_t seed,
                    uint64_t offset, int64_t token_base, float* noise_out, void* ws,
                    size_t ws_bytes, moe_stream_t stream);
+
+/* Self-test of the library's failure detection; the pages have no
+ * counterpart.  Every pipeline wait in the library's kernels is bounded:
+ * instead of hanging, a wait that does not complete in time records an
+ * error code on the workspace's error word and the kernel returns, leaving
+ * the CUDA context usable.  This call runs one such wait on an mbarrier that
+ * nothing completes, with a limit of limit_us microseconds (1 .. 10^7), so
+ * a caller (or a health check) can see the mechanism work: afterwards
+ * moe_device_status reports code 20.  It faults nothing and holds the GPU
+ * for about limit_us.  ws needs only its first 256 bytes (the error word). */
+int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream);
 
 /* moe_route without a workspace.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for

@@ -31,6 +31,7 @@ _SIGNATURES = {
     "moe_device_status": (ctypes.c_int, [_c_p, ctypes.c_size_t, _c_p, _c_p]),
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
+    "moe_check_wait_timeout": (ctypes.c_int, [_c_p, ctypes.c_size_t, ctypes.c_uint32, _c_p]),
     "moe_gate_noise": (ctypes.c_int, [_c_p] * 3 + [ctypes.c_uint64, ctypes.c_uint64,
                                                    ctypes.c_int64, _c_p, _c_p, ctypes.c_size_t,
                                                    _c_p]),
@@ -170,6 +171,11 @@ def moe_route_noalloc(cfg, x, W_router, logit_bias, noise, expert_indices, gates
         ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
         _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _stream(stream)),
         "moe_route_noalloc")
+
+
+def moe_check_wait_timeout(ws, limit_us: int, stream=None) -> None:
+    _check(load_library().moe_check_wait_timeout(_ptr(ws), ws.numel(), int(limit_us),
+                                                  _stream(stream)), "moe_check_wait_timeout")
 
 
 def moe_gate_noise(cfg, x, W_noise, seed, offset, token_base, noise_out, ws, stream=None) -> None:

@@ -118,6 +118,28 @@ cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* per
 
 }  // namespace
 
+namespace {
+
+// The library's bounded wait, made to run out: an mbarrier that nothing
+// arrives on.  The wait gives up after limit_ns, records the self-test code
+// on the error word and the kernel returns normally.
+__global__ void wait_self_test_kernel(int32_t* err, uint64_t limit_ns) {
+  pdl_wait_and_release();
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, limit_ns)) report_error(err, kDevTimeoutSelfTest);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_wait_self_test(int32_t* err, uint64_t limit_ns, cudaStream_t s) {
+  return launch_kernel(wait_self_test_kernel, 1, 32, 0, s, 0, err, limit_ns);
+}
+
+
 WsLayout workspace_layout(const moe_config_t& c) {
   WsLayout L{};
   size_t off = 0;
@@ -297,6 +319,17 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
 }  // namespace
 
 extern "C" {
+
+int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace missing or too small");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (limit_us == 0 || limit_us > 10000000u)
+    return fail(MOE_ERR_INVALID_ARG, "limit_us must be in [1, 10^7]");
+  const cudaError_t e = launch_wait_self_test(at<int32_t>(ws, 0), (uint64_t)limit_us * 1000ull,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_check_wait_timeout");
+}
 
 int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise, uint64_t seed,
                    uint64_t offset, int64_t token_base, float* noise_out, void* ws,

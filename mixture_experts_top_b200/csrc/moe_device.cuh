@@ -24,6 +24,7 @@ enum DeviceError : int32_t {
   kDevTimeoutMma = 17,        // MMA issuer gave up waiting for data / accumulator
   kDevTimeoutEpilogue = 18,   // epilogue gave up waiting for an accumulator
   kDevTimeoutDrain = 19,      // teardown gave up waiting for in-flight copies/MMAs
+  kDevTimeoutSelfTest = 20,   // moe_check_wait_timeout: its wait ran out, as intended
 };
 
 // A pipeline wait that has not completed after this many nanoseconds is
@@ -78,14 +79,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false if
-// it did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// it did not complete within limit_ns (kWaitLimitNs by default).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 

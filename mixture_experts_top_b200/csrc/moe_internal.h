@@ -154,6 +154,9 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
                                 const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
                                 const int32_t* perm = nullptr, int a_rows = 0);
 
+// One bounded mbarrier wait that nothing completes; after limit_ns the kernel
+// writes the self-test code to err and returns (moe_api.cu).
+cudaError_t launch_wait_self_test(int32_t* err, uint64_t limit_ns, cudaStream_t s);
 // Host-side capacity: ceil(((cf * T) * k) / E) in fp64, or -1 for no limit.
 int64_t capacity_slots(float capacity_factor, int T, int k, int E);
 
