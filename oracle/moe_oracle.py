@@ -108,6 +108,8 @@ def widen(a: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "bf16":
         a = np.asarray(a, dtype=np.uint16)
         return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    if dtype == "f64":
+        return np.asarray(a, dtype=np.float64)
     return np.asarray(a, dtype=np.float32).astype(np.float64)
 
 
@@ -348,6 +350,62 @@ def combine(Y: np.ndarray, dest: np.ndarray, gates: np.ndarray) -> np.ndarray:
             if r >= 0:
                 y[t] += float(gates[t, j]) * Y[r]
     return y
+
+
+# ----------------------------------------------------------------------------
+# Backward of the routing half (gradients of the combine and of the router)
+# ----------------------------------------------------------------------------
+# The pages train the layer but print no backward; these are the derivatives
+# of the forward above, in fp64, pinned by finite differences of it.
+# [MLG Algorithm 2-4; PFD The code, `switch_balance_loss`: f is a count and
+# carries no gradient, P does]
+
+def combine_backward(Y: np.ndarray, dest: np.ndarray, gates: np.ndarray, dy: np.ndarray):
+    """Gradients of y_t = sum over kept j of gates[t,j] * Y[dest[t,j]].
+
+    Returns dY (rows of Y; a row gets gates[t,j] * dy_t from its slot) and
+    dgates[t, j] = <dy_t, Y[dest[t,j]]> (0 for a dropped slot)."""
+    Y = np.asarray(Y, np.float64)
+    dy = np.asarray(dy, np.float64)
+    T, k = dest.shape
+    dY = np.zeros_like(Y)
+    dg = np.zeros((T, k), np.float64)
+    for t in range(T):
+        for j in range(k):
+            r = int(dest[t, j])
+            if r >= 0:
+                dY[r] += float(gates[t, j]) * dy[t]
+                dg[t, j] = float(dy[t] @ Y[r])
+    return dY, dg
+
+
+def route_backward(x, W_router, dtype: str, logits, idx, gates, f, dgates, daux: float,
+                   T_batch: Optional[int] = None):
+    """Gradients of the router's outputs back to its inputs.
+
+    gates (softmax over the chosen k): dL_m += g_m (dg_m - sum_j g_j dg_j)
+    for each chosen m; the top-k choice itself has no gradient.  aux =
+    E sum_e f_e P_e with P_e the batch mean of softmax(L)[:, e] (T_batch
+    tokens, this call's T by default) and f constant: dL_te += p_te (a_e -
+    sum_e' p_te' a_e') with a_e = daux E f_e / T_batch.  Then, for L = x @ W
+    (+ bias + noise): dx = dL @ W^T, dW = x^T @ dL, dbias = sum_t dL.
+    Returns dict(dlogits, dx, dW, dbias), fp64."""
+    L = np.asarray(logits, np.float64)
+    T, E = L.shape
+    p = softmax_rows(L)
+    g = np.asarray(gates, np.float64)
+    dg = np.asarray(dgates, np.float64)
+    dL = np.zeros((T, E), np.float64)
+    for t in range(T):
+        s = float(g[t] @ dg[t])
+        for j in range(idx.shape[1]):
+            dL[t, int(idx[t, j])] += g[t, j] * (dg[t, j] - s)
+    Tb = T if T_batch is None else T_batch
+    a = float(daux) * E * np.asarray(f, np.float64) / Tb
+    dL += p * (a[None, :] - (p @ a)[:, None])
+    W = np.asarray(W_router, np.float64)
+    xf = widen(x, dtype)
+    return dict(dlogits=dL, dx=dL @ W.T, dW=xf.T @ dL, dbias=dL.sum(axis=0))
 
 
 # ----------------------------------------------------------------------------
