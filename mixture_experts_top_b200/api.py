@@ -32,6 +32,9 @@ _SIGNATURES = {
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
     "moe_check_wait_timeout": (ctypes.c_int, [_c_p, ctypes.c_size_t, ctypes.c_uint32, _c_p]),
+    "moe_combine_backward": (ctypes.c_int, [_c_p] * 8),
+    "moe_route_backward": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_int32] + [_c_p] * 5 +
+                           [ctypes.c_size_t, _c_p]),
     "moe_gate_noise": (ctypes.c_int, [_c_p] * 3 + [ctypes.c_uint64, ctypes.c_uint64,
                                                    ctypes.c_int64, _c_p, _c_p, ctypes.c_size_t,
                                                    _c_p]),
@@ -171,6 +174,20 @@ def moe_route_noalloc(cfg, x, W_router, logit_bias, noise, expert_indices, gates
         ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
         _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _stream(stream)),
         "moe_route_noalloc")
+
+
+def moe_combine_backward(cfg, dy, y_perm, dest, gates, dy_perm, dgates, stream=None) -> None:
+    _check(load_library().moe_combine_backward(
+        ctypes.byref(cfg), _ptr(dy), _ptr(y_perm), _ptr(dest), _ptr(gates), _ptr(dy_perm),
+        _ptr(dgates), _stream(stream)), "moe_combine_backward")
+
+
+def moe_route_backward(cfg, x, W_router, logits, expert_indices, gates, f, dgates, daux, T_batch,
+                       dx, dW_router, dbias, dlogits, ws, stream=None) -> None:
+    _check(load_library().moe_route_backward(
+        ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logits), _ptr(expert_indices),
+        _ptr(gates), _ptr(f), _ptr(dgates), _ptr(daux), int(T_batch), _ptr(dx), _ptr(dW_router),
+        _ptr(dbias), _ptr(dlogits), _ptr(ws), ws.numel(), _stream(stream)), "moe_route_backward")
 
 
 def moe_check_wait_timeout(ws, limit_us: int, stream=None) -> None:

@@ -170,6 +170,10 @@ WsLayout workspace_layout(const moe_config_t& c) {
   L.x_perm = take(Tk * (size_t)c.d * s);
   L.hidden = take(c.expert_kind == MOE_EXPERT_LINEAR ? 0 : Tk * (size_t)c.d_hidden * 2);
   L.y_perm = take(Tk * (size_t)c.d_out * 4);
+  const size_t nch = (size_t)route_backward_chunks(c.T);
+  L.dlogits = take((size_t)c.T * E * 4);
+  L.dw_part = take(nch * (size_t)c.d * E * 4);
+  L.dbias_part = take(nch * E * 4);
   L.total = off;
   return L;
 }
@@ -319,6 +323,63 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
 }  // namespace
 
 extern "C" {
+
+int moe_combine_backward(const moe_config_t* cfg, const void* dy, const void* y_perm,
+                         const int32_t* dest, const float* gates, float* dy_perm, float* dgates,
+                         moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(dy);
+    MOE_REQUIRE(y_perm);
+    MOE_REQUIRE(dest);
+    MOE_REQUIRE(gates);
+    MOE_REQUIRE(dy_perm);
+    MOE_REQUIRE(dgates);
+  }
+  MOE_ALIGNED16(dy);
+  MOE_ALIGNED16(y_perm);
+  MOE_ALIGNED16(dy_perm);
+  const cudaError_t e = launch_combine_backward(c, dy, static_cast<const float*>(y_perm), dest,
+                                                gates, dy_perm, dgates,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine_backward");
+}
+
+int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_router,
+                       const float* logits, const int32_t* expert_indices, const float* gates,
+                       const float* f, const float* dgates, const float* daux, int32_t T_batch,
+                       float* dx, float* dW_router, float* dbias, float* dlogits, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(logits);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(gates);
+    MOE_REQUIRE(dgates);
+    MOE_REQUIRE(dx);
+  }
+  MOE_REQUIRE(W_router);
+  MOE_REQUIRE(f);
+  MOE_REQUIRE(daux);
+  MOE_REQUIRE(dW_router);
+  MOE_ALIGNED16(x);
+  MOE_ALIGNED16(dx);
+  const int Tb = T_batch > 0 ? T_batch : c.T;
+  if (T_batch < 0 || (c.T > 0 && Tb < c.T))
+    return fail(MOE_ERR_INVALID_ARG, "T_batch must be 0 (this call's T) or >= T");
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_route_backward(
+      c, x, W_router, logits, expert_indices, gates, f, dgates, daux, Tb, dx, dW_router, dbias,
+      dlogits != nullptr ? dlogits : at<float>(ws, L.dlogits), at<float>(ws, L.dw_part),
+      at<float>(ws, L.dbias_part), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_backward");
+}
 
 int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream) {
   if (ws == nullptr || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace missing or too small");

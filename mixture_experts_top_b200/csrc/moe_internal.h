@@ -40,6 +40,9 @@ struct WsLayout {
   size_t x_perm;         // (T*k, d) act
   size_t hidden;         // (T*k, d_hidden) bf16
   size_t y_perm;         // (T*k, d_out) fp32
+  size_t dlogits;        // (T, E) fp32: moe_route_backward's logit gradient
+  size_t dw_part;        // (chunks, d, E) fp32: per-chunk partial dW_router
+  size_t dbias_part;     // (chunks, E) fp32
   size_t total;
 };
 
@@ -154,6 +157,17 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
                                 const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
                                 const int32_t* perm = nullptr, int a_rows = 0);
 
+// Routing backward (backward.cu).
+int route_backward_chunks(int T);
+cudaError_t launch_combine_backward(const moe_config_t& c, const void* dy, const float* y_perm,
+                                    const int32_t* dest, const float* gates, float* dy_perm,
+                                    float* dgates, cudaStream_t s);
+cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const float* W,
+                                  const float* logits, const int32_t* idx, const float* gates,
+                                  const float* f, const float* dgates, const float* daux,
+                                  int T_batch, float* dx, float* dW, float* dbias,
+                                  float* dlogits, float* dw_part, float* dbias_part,
+                                  cudaStream_t s);
 // One bounded mbarrier wait that nothing completes; after limit_ns the kernel
 // writes the self-test code to err and returns (moe_api.cu).
 cudaError_t launch_wait_self_test(int32_t* err, uint64_t limit_ns, cudaStream_t s);

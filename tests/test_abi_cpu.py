@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 16
+    assert len(names) == 18
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -126,8 +126,7 @@ def test_workspace_holds_the_split_router_weights(moe_lib):
     b = api.make_config(64, 4096, 128, 64, 100, 2, "swiglu", "bf16")   # E > 64: SIMT router
     c = api.make_config(64, 4096, 128, 64, 16, 2, "swiglu", "bf16")
     na, nb, nc = (moe_lib.moe_workspace_size(ctypes.byref(x)) for x in (a, b, c))
-    assert nc - na == 0                                  # E = 8 and 16 both pad to 16
-    assert na >= 3 * 16 * 4096 * 2
+    assert na >= 3 * 16 * 4096 * 2 and nc >= 3 * 16 * 4096 * 2
     assert nb > 0
 
 
@@ -170,6 +169,26 @@ def test_gate_noise_argument_checks(moe_lib):
     ws2 = moe_lib.moe_workspace_size(ctypes.byref(wide))
     assert moe_lib.moe_gate_noise(ctypes.byref(wide), FAKE, FAKE, 1, 0, 0, FAKE, FAKE, ws2,
                                   None) == api.MOE_ERR_UNSUPPORTED
+
+
+def test_backward_argument_checks(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    assert moe_lib.moe_combine_backward(ctypes.byref(cfg), None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        None) == api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_combine_backward(ctypes.byref(cfg), FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        None) == api.MOE_ERR_INVALID_ARG
+    args = [FAKE] * 8                        # x, W, logits, idx, gates, f, dgates, daux
+    ok_tail = [FAKE, FAKE, None, None, FAKE, ws, None]
+    # T_batch below this call's T
+    assert moe_lib.moe_route_backward(ctypes.byref(cfg), *args, 32, *ok_tail) == \
+        api.MOE_ERR_INVALID_ARG
+    # dW missing
+    assert moe_lib.moe_route_backward(ctypes.byref(cfg), *args, 0, FAKE, None, None, None, FAKE,
+                                      ws, None) == api.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert moe_lib.moe_route_backward(ctypes.byref(cfg), *args, 0, FAKE, FAKE, None, None, FAKE,
+                                      ws - 256, None) == api.MOE_ERR_WORKSPACE
 
 
 def test_swiglu_needs_three_matrices(moe_lib):
