@@ -408,6 +408,44 @@ def run_ours(args, rank, world):
                                 "note": "moe_gate_noise at this shape (x read, W_noise read, "
                                         "(T,E) fp32 noise written), back to back, x in L2"}
 
+    # The routing half of the backward (moe_combine_backward +
+    # moe_route_backward) on this step's intermediates, timed on its own.
+    Lg = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    api.moe_route(cfg, x, Wr, bias, noise, o.expert_indices, o.gates, P, Lg, ws)
+    api.moe_dispatch(cfg, x, o.expert_indices, P, o.counts, offsets, dest, perm, o.drop_mask,
+                     f, o.aux_loss, x_perm, ws)
+    api.moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws)
+    dyb = torch.randn((T, w.d_out), device="cuda").to(o.output.dtype)
+    dyp = torch.empty((R, w.d_out), dtype=torch.float32, device="cuda")
+    dgb = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    dxb = torch.empty((T, w.d), dtype=torch.float32, device="cuda")
+    dWb = torch.empty((w.d, E), dtype=torch.float32, device="cuda")
+    dbb = torch.empty(E, dtype=torch.float32, device="cuda")
+    dab = torch.ones(1, dtype=torch.float32, device="cuda")
+
+    def backward_once():
+        api.moe_combine_backward(cfg, dyb, y_perm, dest, o.gates, dyp, dgb)
+        api.moe_route_backward(cfg, x, Wr, Lg, o.expert_indices, o.gates, f, dgb, dab, 0, dxb,
+                               dWb, dbb, None, ws)
+
+    for _ in range(3):
+        backward_once()
+    b_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    b_ev[0].record(stream)
+    for _ in range(10):
+        backward_once()
+    b_ev[1].record(stream)
+    torch.cuda.synchronize()
+    b_us = b_ev[0].elapsed_time(b_ev[1]) / 10 * 1e3
+    elem = 2 if w.dtype == "bf16" else 4
+    kept = int((dest >= 0).sum().item())
+    b_bytes = (T * w.d_out * elem + 2 * kept * w.d_out * 4
+               + T * E * 4 * 2 + T * w.d * (elem + 4) + T * k * 16)
+    extras["routing_backward"] = {
+        "us": b_us, "GB/s": b_bytes / b_us / 1e3, "frac_hbm": b_bytes / b_us / 1e3 / peaks["hbm_gbs"],
+        "note": "moe_combine_backward + moe_route_backward (6 launches): dy read, expert rows "
+                "read and their gradients written, logits and dlogits, x read and dx written"}
+
     counts = o.counts.cpu().numpy()
     rows = A.kept_rows(counts, w.capacity_factor, T, k)
     used = int((counts > 0).sum())

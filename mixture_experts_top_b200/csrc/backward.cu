@@ -15,10 +15,10 @@
 //   logits:   L = x W (+ bias + noise):  dx = dL W^T,  dW = x^T dL,  dbias = sum_t dL
 //
 // All in fp32 with fixed summation orders (no atomics): the combine and the
-// logit gradient one warp per token; dx one thread per 4 output columns, the
-// E terms in order; dW and dbias as per-chunk partial sums over token chunks,
-// then the chunks added in order.  Everything here is bound by HBM or by
-// launch latency.
+// logit gradient one warp per token; dx one thread per column and 16 tokens,
+// the E terms in order; dW and dbias as per-chunk partial sums over token
+// chunks (tokens in order), then the chunks added in order.  Everything here
+// is bound by HBM or by launch latency.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -176,66 +176,101 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// dx[t, c..c+3] = sum_e dL[t, e] W[c..c+3, e], e in increasing order.
+// dx[t, c] = sum_e dL[t, e] W[c, e], e in increasing order.  A CTA owns 256
+// columns and kTg tokens; W and dL stream through shared memory 32 experts
+// at a time, so each thread keeps kTg accumulators for its column.
+constexpr int kTg = 16;
+constexpr int kEb = 32;
+
 __global__ void __launch_bounds__(256)
     route_dx_kernel(const float* __restrict__ dlogits, const float* __restrict__ W, int T, int d,
                     int E, float* __restrict__ dx) {
   pdl_wait_and_release();
-  const long long n4 = (long long)T * (d / 4);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long t = i / (d / 4);
-    const int c = (int)(i - t * (d / 4)) * 4;
-    const float* dl = dlogits + t * E;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int e = 0; e < E; ++e) {
-      const float g = dl[e];
+  __shared__ float ws[kEb][256];
+  __shared__ float dls[kTg][kEb];
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  const int t0 = blockIdx.y * kTg;
+  float acc[kTg];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(g, W[(size_t)(c + u) * E + e], acc[u]);
+  for (int i = 0; i < kTg; ++i) acc[i] = 0.f;
+  for (int e0 = 0; e0 < E; e0 += kEb) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kEb * 256; i += 256) {
+      const int e = i / 256, cc = blockIdx.x * 256 + i % 256;
+      ws[e][i % 256] = (e0 + e < E && cc < d) ? W[(size_t)cc * E + e0 + e] : 0.f;
     }
-    *reinterpret_cast<float4*>(dx + t * d + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    for (int i = threadIdx.x; i < kTg * kEb; i += 256) {
+      const int tt = i / kEb, e = i % kEb;
+      dls[tt][e] = (t0 + tt < T && e0 + e < E) ? dlogits[(size_t)(t0 + tt) * E + e0 + e] : 0.f;
+    }
+    __syncthreads();
+    const int ne = min(kEb, E - e0);
+    for (int e = 0; e < ne; ++e) {
+      const float wv = ws[e][threadIdx.x];
+#pragma unroll
+      for (int i = 0; i < kTg; ++i) acc[i] = fmaf(dls[i][e], wv, acc[i]);
+    }
   }
+  if (c < d)
+#pragma unroll
+    for (int i = 0; i < kTg; ++i)
+      if (t0 + i < T) dx[(size_t)(t0 + i) * d + c] = acc[i];
 }
 
-constexpr int kDwOuts = 8;        // (c, e) outputs per thread
-constexpr int kDwThreads = 256;
+constexpr int kCt = 64;           // columns of x per dW CTA
+constexpr int kTs = 32;           // tokens staged in shared memory at a time
 
-// Partial dW and dbias over one chunk of tokens: CTA (tile, chunk) owns the
-// outputs o = tile * 2048 + [0, 2048) of the flattened (d, E) dW, i.e.
-// c = o / E, e = o % E, and sums its tokens in increasing order.
-template <typename XT>
-__global__ void __launch_bounds__(kDwThreads)
+// Partial dW and dbias over one chunk of tokens.  CTA (tile, chunk) owns
+// columns [64 tile, 64 tile + 64) of x: thread (c, g) accumulates
+// dW[c, e] for the experts e of group g (EPT of them), over the chunk's
+// tokens in increasing order, x and dL staged 32 tokens at a time.  Tile 0
+// also sums dL over the chunk for dbias.
+template <typename XT, int EPT>
+__global__ void __launch_bounds__(256)
     route_dw_partial_kernel(const XT* __restrict__ x, const float* __restrict__ dlogits, int T,
                             int d, int E, int nchunks, float* __restrict__ dw_part,
                             float* __restrict__ dbias_part) {
   pdl_wait_and_release();
+  __shared__ float xs[kTs][kCt];
+  extern __shared__ float dls[];   // [kTs][E]
   const int chunk = blockIdx.y;
   const int t0 = (int)((long long)T * chunk / nchunks);
   const int t1 = (int)((long long)T * (chunk + 1) / nchunks);
-  const long long total = (long long)d * E;
-  long long o[kDwOuts];
-  int cc[kDwOuts], ee[kDwOuts];
-  float acc[kDwOuts];
+  const int cl = threadIdx.x % kCt, grp = threadIdx.x / kCt;   // 4 groups of experts
+  const int c = blockIdx.x * kCt + cl;
+  const int ebase = grp * EPT;
+  float acc[EPT];
 #pragma unroll
-  for (int i = 0; i < kDwOuts; ++i) {
-    o[i] = (long long)blockIdx.x * (kDwThreads * kDwOuts) + threadIdx.x + i * kDwThreads;
-    cc[i] = (int)(o[i] / E);
-    ee[i] = (int)(o[i] - (long long)cc[i] * E);
-    acc[i] = 0.f;
-  }
-  float bacc = 0.f;                          // dbias[threadIdx.x], tile 0 only
+  for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
+  float bacc = 0.f;
   const bool do_bias = blockIdx.x == 0 && (int)threadIdx.x < E;
-  for (int t = t0; t < t1; ++t) {
-    const XT* xr = x + (size_t)t * d;
-    const float* dl = dlogits + (size_t)t * E;
+  for (int ts0 = t0; ts0 < t1; ts0 += kTs) {
+    const int n = min(kTs, t1 - ts0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kTs * kCt; i += 256) {
+      const int tt = i / kCt, cc = blockIdx.x * kCt + i % kCt;
+      xs[tt][i % kCt] = (tt < n && cc < d) ? static_cast<float>(x[(size_t)(ts0 + tt) * d + cc])
+                                          : 0.f;
+    }
+    for (int i = threadIdx.x; i < kTs * E; i += 256) {
+      const int tt = i / E;
+      dls[i] = tt < n ? dlogits[(size_t)(ts0 + tt) * E + (i - tt * E)] : 0.f;
+    }
+    __syncthreads();
+    for (int tt = 0; tt < n; ++tt) {
+      const float xv = xs[tt][cl];
+      const float* dl = dls + tt * E + ebase;
 #pragma unroll
-    for (int i = 0; i < kDwOuts; ++i)
-      if (o[i] < total) acc[i] = fmaf(static_cast<float>(xr[cc[i]]), dl[ee[i]], acc[i]);
-    if (do_bias) bacc += dl[threadIdx.x];
+      for (int i = 0; i < EPT; ++i)
+        if (ebase + i < E) acc[i] = fmaf(xv, dl[i], acc[i]);
+      if (do_bias) bacc += dls[tt * E + threadIdx.x];
+    }
   }
+  const long long total = (long long)d * E;
+  if (c < d)
 #pragma unroll
-  for (int i = 0; i < kDwOuts; ++i)
-    if (o[i] < total) dw_part[(size_t)chunk * total + o[i]] = acc[i];
+    for (int i = 0; i < EPT; ++i)
+      if (ebase + i < E) dw_part[(size_t)chunk * total + (size_t)c * E + ebase + i] = acc[i];
   if (do_bias) dbias_part[(size_t)chunk * E + threadIdx.x] = bacc;
 }
 
@@ -295,21 +330,44 @@ cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const fl
                                 dgates, f, daux, c.T, c.E, c.top_k,
                                 (double)c.E / (double)T_batch, dlogits);
   if (e != cudaSuccess) return e;
-  const long long n4 = (long long)c.T * (c.d / 4);
-  const int xblocks = (int)std::min<long long>((n4 + 255) / 256, (long long)device_sm_count() * 16);
-  e = launch_kernel(route_dx_kernel, xblocks, 256, 0, s, 0, dlogits, W, c.T, c.d, c.E, dx);
+  e = launch_kernel(route_dx_kernel, dim3((unsigned)ceil_div(c.d, 256), (unsigned)ceil_div(c.T, kTg)),
+                    256, 0, s, 0, dlogits, W, c.T, c.d, c.E, dx);
   if (e != cudaSuccess) return e;
   const int nchunks = route_backward_chunks(c.T);
-  const dim3 grid((unsigned)((total + kDwThreads * kDwOuts - 1) / (kDwThreads * kDwOuts)),
-                  (unsigned)nchunks);
-  if (c.act_dtype == MOE_BF16)
-    e = launch_kernel(route_dw_partial_kernel<__nv_bfloat16>, grid, kDwThreads, 0, s, 0,
-                      static_cast<const __nv_bfloat16*>(x), dlogits, c.T, c.d, c.E, nchunks,
-                      dw_part, dbias_part);
-  else
-    e = launch_kernel(route_dw_partial_kernel<float>, grid, kDwThreads, 0, s, 0,
-                      static_cast<const float*>(x), dlogits, c.T, c.d, c.E, nchunks, dw_part,
-                      dbias_part);
+  const dim3 grid((unsigned)ceil_div(c.d, kCt), (unsigned)nchunks);
+  const size_t dsm = (size_t)kTs * c.E * sizeof(float);
+  const int ept = c.E <= 8 ? 2 : c.E <= 16 ? 4 : c.E <= 32 ? 8 : c.E <= 64 ? 16 : c.E <= 128 ? 32 : 64;
+  auto run = [&](auto kern) {
+    cudaError_t r = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)dsm);
+    if (r != cudaSuccess) return r;
+    return launch_kernel(kern, grid, 256, dsm, s, 0, static_cast<const __nv_bfloat16*>(x),
+                         dlogits, c.T, c.d, c.E, nchunks, dw_part, dbias_part);
+  };
+  auto runf = [&](auto kern) {
+    cudaError_t r = ensure_smem_limit(reinterpret_cast<const void*>(kern), (int)dsm);
+    if (r != cudaSuccess) return r;
+    return launch_kernel(kern, grid, 256, dsm, s, 0, static_cast<const float*>(x), dlogits, c.T,
+                         c.d, c.E, nchunks, dw_part, dbias_part);
+  };
+  if (c.act_dtype == MOE_BF16) {
+    switch (ept) {
+      case 2: e = run(route_dw_partial_kernel<__nv_bfloat16, 2>); break;
+      case 4: e = run(route_dw_partial_kernel<__nv_bfloat16, 4>); break;
+      case 8: e = run(route_dw_partial_kernel<__nv_bfloat16, 8>); break;
+      case 16: e = run(route_dw_partial_kernel<__nv_bfloat16, 16>); break;
+      case 32: e = run(route_dw_partial_kernel<__nv_bfloat16, 32>); break;
+      default: e = run(route_dw_partial_kernel<__nv_bfloat16, 64>); break;
+    }
+  } else {
+    switch (ept) {
+      case 2: e = runf(route_dw_partial_kernel<float, 2>); break;
+      case 4: e = runf(route_dw_partial_kernel<float, 4>); break;
+      case 8: e = runf(route_dw_partial_kernel<float, 8>); break;
+      case 16: e = runf(route_dw_partial_kernel<float, 16>); break;
+      case 32: e = runf(route_dw_partial_kernel<float, 32>); break;
+      default: e = runf(route_dw_partial_kernel<float, 64>); break;
+    }
+  }
   if (e != cudaSuccess) return e;
   const int rblocks = (int)std::min<long long>((total + 255) / 256, (long long)device_sm_count() * 8);
   return launch_kernel(route_dw_reduce_kernel, rblocks, 256, 0, s, 0, dw_part, dbias_part, total,
