@@ -379,6 +379,79 @@ def combine_backward(Y: np.ndarray, dest: np.ndarray, gates: np.ndarray, dy: np.
     return dY, dg
 
 
+def expert_backward(kind: str, xe: np.ndarray, W_in: np.ndarray, W_up: Optional[np.ndarray],
+                    W_out: Optional[np.ndarray], dY: np.ndarray) -> dict:
+    """Gradients of one expert (expert_forward) on its rows, fp64.
+
+    With A = x W_in (and B = x W_up for SwiGLU), H the hidden activation and
+    dH = dY W_out^T:
+    * linear: dx = dY W_in^T, dW_in = x^T dY
+    * relu:   dA = dH * [A > 0]
+    * swiglu: H = silu(A) * B; dA = dH * B * silu'(A), dB = dH * silu(A),
+              silu'(a) = s (1 + a (1 - s)) with s = sigmoid(a)
+    then dW_out = H^T dY, dW_in = x^T dA, dW_up = x^T dB, dx = dA W_in^T
+    (+ dB W_up^T).  Returns dict(dx, dW_in, dW_up, dW_out)."""
+    xe = np.asarray(xe, np.float64)
+    dY = np.asarray(dY, np.float64)
+    if kind == "linear":
+        return dict(dx=dY @ W_in.T, dW_in=xe.T @ dY, dW_up=None, dW_out=None)
+    A = xe @ W_in
+    if kind == "relu":
+        H = np.maximum(A, 0.0)
+        dH = dY @ W_out.T
+        dA = dH * (A > 0.0)
+        return dict(dx=dA @ W_in.T, dW_in=xe.T @ dA, dW_up=None, dW_out=H.T @ dY)
+    if kind == "swiglu":
+        B = xe @ W_up
+        sg = 1.0 / (1.0 + np.exp(-A))
+        H = A * sg * B
+        dH = dY @ W_out.T
+        dA = dH * B * (sg * (1.0 + A * (1.0 - sg)))
+        dB = dH * (A * sg)
+        return dict(dx=dA @ W_in.T + dB @ W_up.T, dW_in=xe.T @ dA, dW_up=xe.T @ dB,
+                    dW_out=H.T @ dY)
+    raise ValueError(f"unknown expert kind {kind!r}")
+
+
+def moe_backward(x, W_router, weights: dict, *, top_k: int, kind: str, dtype: str,
+                 d_out: int, dy: np.ndarray, daux: float, capacity_factor: float = 0.0,
+                 logit_bias=None, noise=None) -> dict:
+    """The whole layer's backward in fp64, composed of the pieces above: the
+    forward (moe_forward), the combine backward into each kept row, each
+    expert's backward on its rows, the rows' input gradients added back to
+    their tokens (dx_t = sum over kept j of dX[dest[t,j]]), and the router
+    backward (gates and aux) added to dx.  Returns dict(dx, dW_router, dbias,
+    dW_in, dW_up, dW_out) (weights' gradients stacked over experts)."""
+    fw = moe_forward(x, W_router, weights, top_k=top_k, kind=kind, dtype=dtype, d_out=d_out,
+                     capacity_factor=capacity_factor, logit_bias=logit_bias, noise=noise)
+    dY, dg = combine_backward(fw["Y"], fw["dest"], fw["gates"].astype(np.float64), dy)
+    xf = widen(x, dtype)
+    T, d = xf.shape
+    E = np.asarray(W_router).shape[1]
+    dx = np.zeros((T, d), np.float64)
+    grads = {key: None for key in ("W_in", "W_up", "W_out")}
+    for key in grads:
+        if weights.get(key) is not None:
+            grads[key] = np.zeros(np.asarray(weights[key]).shape, np.float64)
+    offs = fw["offsets"]
+    perm = fw["perm_token"]
+    for e in range(E):
+        lo, hi = int(offs[e]), int(offs[e + 1])
+        if hi <= lo:
+            continue
+        rows = perm[lo:hi]
+        g = expert_backward(kind, xf[rows], *expert_weights(weights, e, dtype), dY[lo:hi])
+        np.add.at(dx, rows, g["dx"])
+        for key, gk in (("W_in", "dW_in"), ("W_up", "dW_up"), ("W_out", "dW_out")):
+            if grads[key] is not None:
+                grads[key][e] += g[gk]
+    r = route_backward(x, W_router, dtype, fw["logits"], fw["expert_indices"],
+                       fw["gates"].astype(np.float64), fw["f"], dg, daux)
+    dx += r["dx"]
+    return dict(dx=dx, dW_router=r["dW"], dbias=r["dbias"], dW_in=grads["W_in"],
+                dW_up=grads["W_up"], dW_out=grads["W_out"])
+
+
 def route_backward(x, W_router, dtype: str, logits, idx, gates, f, dgates, daux: float,
                    T_batch: Optional[int] = None):
     """Gradients of the router's outputs back to its inputs.

@@ -104,3 +104,59 @@ def test_aux_gradient_closed_form_uniform():
     a0 = 2.0 * E * 1.0 / T
     assert np.allclose(r["dlogits"][:, 0], (1 / E) * (a0 - a0 / E))
     assert np.allclose(r["dlogits"][:, 1:], (1 / E) * (0 - a0 / E))
+
+
+def _layer_loss(x, W, bias, weights, kind, idx, disp, dy, f, daux):
+    """The layer in fp64 with the routing decisions held fixed."""
+    L = x @ W + bias
+    g = _gates64(L, idx)
+    E = W.shape[1]
+    R = int(disp["offsets"][-1])
+    Y = np.zeros((R, dy.shape[1]))
+    for e in range(E):
+        lo, hi = int(disp["offsets"][e]), int(disp["offsets"][e + 1])
+        if hi > lo:
+            Y[lo:hi] = O.expert_forward(kind, x[disp["perm_token"][lo:hi]],
+                                        *O.expert_weights(weights, e, "f64"))
+    y = O.combine(Y, disp["dest"], g)
+    aux = E * float(f @ O.softmax_rows(L).mean(axis=0))
+    return float(np.sum(dy * y)) + daux * aux
+
+
+@pytest.mark.parametrize("kind", ["linear", "relu", "swiglu"])
+@pytest.mark.parametrize("cf", [0.0, 0.75])
+def test_layer_backward_matches_finite_differences(kind, cf):
+    T, d, h, d_out, E, k = 6, 4, 5, 3, 4, 2
+    rng = np.random.default_rng(7 + len(kind))
+    x = rng.standard_normal((T, d))
+    W = rng.standard_normal((d, E))
+    bias = rng.standard_normal(E)
+    L = x @ W + bias
+    Ls = -np.sort(-L, axis=1)
+    assert (Ls[:, :k] - Ls[:, 1:k + 1]).min() > 1e-3            # no near-tie in the top k
+    weights = {"W_in": rng.standard_normal((E, d, d_out if kind == "linear" else h)),
+               "W_up": rng.standard_normal((E, d, h)) if kind == "swiglu" else None,
+               "W_out": rng.standard_normal((E, h, d_out)) if kind != "linear" else None}
+    dy = rng.standard_normal((T, d_out))
+    daux = 0.3
+    got = O.moe_backward(x, W, weights, top_k=k, kind=kind, dtype="f64", d_out=d_out, dy=dy,
+                         daux=daux, capacity_factor=cf, logit_bias=bias)
+    idx = O.top_k(L.astype(np.float32), k)
+    disp = O.dispatch(idx, E, cf)
+    f = disp["f"].astype(np.float64)
+    params = dict(x=x, W=W, bias=bias, **{key: v for key, v in weights.items() if v is not None})
+    want = dict(x="dx", W="dW_router", bias="dbias", W_in="dW_in", W_up="dW_up", W_out="dW_out")
+    hstep = 1e-6
+    for name, a in params.items():
+        num = np.zeros_like(a)
+        for i in np.ndindex(a.shape):
+            vals = []
+            for sgn in (1, -1):
+                p = {key: v.copy() for key, v in params.items()}
+                p[name][i] += sgn * hstep
+                wts = {key: p.get(key) for key in ("W_in", "W_up", "W_out")}
+                vals.append(_layer_loss(p["x"], p["W"], p["bias"], wts, kind, idx, disp, dy, f,
+                                        daux))
+            num[i] = (vals[0] - vals[1]) / (2 * hstep)
+        # the oracle's forward decides on fp32 logits and fp32 gates: ~1e-7 relative
+        assert np.allclose(got[want[name]], num, rtol=2e-5, atol=2e-6), (kind, cf, name)
