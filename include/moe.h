@@ -167,56 +167,6 @@ int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise,
                    uint64_t offset, int64_t token_base, float* noise_out, void* ws,
                    size_t ws_bytes, moe_stream_t stream);
 
-/* Backward of the routing half (combine and router), for training.  The
- * pages print no backward; these are the derivatives of the forward above.
- * [MLG Algorithm 2-4; PFD The code, `switch_balance_loss`: f is a count and
- * carries no gradient, P_e does]
- *
- * moe_combine_backward: from dy = dLoss/d output (T, d_out) act_dtype:
- *   dy_perm (T*top_k, d_out) fp32 out: row dest[t,j] = gates[t,j] * dy[t]
- *           (the gradient into the experts' outputs; other rows untouched)
- *   dgates  (T, top_k) fp32 out: <dy[t], y_perm[dest[t,j]]>, 0 if dropped
- *   y_perm and dest, gates as in the forward (y_perm fp32, moe_expert_ffn's).
- * Fixed orders: per token, the columns in order per lane, then a fixed
- * butterfly over the warp.  No workspace. */
-int moe_combine_backward(const moe_config_t* cfg, const void* dy, const void* y_perm,
-                         const int32_t* dest, const float* gates, float* dy_perm, float* dgates,
-                         moe_stream_t stream);
-
-/* moe_route_backward: gradients of the gates and of aux_loss back to the
- * router's inputs.  With p = softmax(logits) per token and g the gates:
- *   dL[t,m] = g_m (dg_m - sum_j g_j dg_j) for each chosen m (the top-k
- *             choice itself has no gradient), plus
- *             p_te (a_e - sum_e' p_te' a_e'),  a_e = daux * E * f_e / T_batch
- *   dx = dL @ W_router^T, dW_router = x^T @ dL, dbias = sum_t dL.
- *   x (T, d) act_dtype; W_router (d, E) fp32; logits (T, E) fp32 (moe_route's
- *   logits_out: the logits the top-k decided on, after bias and noise);
- *   expert_indices, gates (T, top_k); f (E) fp32 (moe_dispatch's, before
- *   capacity); dgates (T, top_k) fp32 (e.g. moe_combine_backward's); daux
- *   (1) fp32 device: dLoss/d aux_loss; T_batch: tokens P_e and f_e are
- *   means over (0 = this call's T; a rank's share of a sharded batch passes
- *   the whole batch's T, and the ranks then add their dW and dbias).
- *   dx (T, d) fp32 out; dW_router (d, E) fp32 out; dbias (E) fp32 out or
- *   NULL; dlogits (T, E) fp32 out or NULL (kept in the workspace then).
- * fp32 throughout with fixed summation orders (dW and dbias: token chunks
- * in order). */
-int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_router,
-                       const float* logits, const int32_t* expert_indices, const float* gates,
-                       const float* f, const float* dgates, const float* daux, int32_t T_batch,
-                       float* dx, float* dW_router, float* dbias, float* dlogits, void* ws,
-                       size_t ws_bytes, moe_stream_t stream);
-
-/* Self-test of the library's failure detection; the pages have no
- * counterpart.  Every pipeline wait in the library's kernels is bounded:
- * instead of hanging, a wait that does not complete in time records an
- * error code on the workspace's error word and the kernel returns, leaving
- * the CUDA context usable.  This call runs one such wait on an mbarrier that
- * nothing completes, with a limit of limit_us microseconds (1 .. 10^7), so
- * a caller (or a health check) can see the mechanism work: afterwards
- * moe_device_status reports code 20.  It faults nothing and holds the GPU
- * for about limit_us.  ws needs only its first 256 bytes (the error word). */
-int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream);
-
 /* moe_route without a workspace.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for
  * example a plugin running inside a host program whose memory pool owns the
@@ -375,6 +325,56 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
                 void* output, int32_t* expert_indices, float* gates, float* aux_loss,
                 int32_t* counts, uint8_t* drop_mask,
                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Backward of the routing half (combine and router), for training.  The
+ * pages print no backward; these are the derivatives of the forward above.
+ * [MLG Algorithm 2-4; PFD The code, `switch_balance_loss`: f is a count and
+ * carries no gradient, P_e does]
+ *
+ * moe_combine_backward: from dy = dLoss/d output (T, d_out) act_dtype:
+ *   dy_perm (T*top_k, d_out) fp32 out: row dest[t,j] = gates[t,j] * dy[t]
+ *           (the gradient into the experts' outputs; other rows untouched)
+ *   dgates  (T, top_k) fp32 out: <dy[t], y_perm[dest[t,j]]>, 0 if dropped
+ *   y_perm and dest, gates as in the forward (y_perm fp32, moe_expert_ffn's).
+ * Fixed orders: per token, the columns in order per lane, then a fixed
+ * butterfly over the warp.  No workspace. */
+int moe_combine_backward(const moe_config_t* cfg, const void* dy, const void* y_perm,
+                         const int32_t* dest, const float* gates, float* dy_perm, float* dgates,
+                         moe_stream_t stream);
+
+/* moe_route_backward: gradients of the gates and of aux_loss back to the
+ * router's inputs.  With p = softmax(logits) per token and g the gates:
+ *   dL[t,m] = g_m (dg_m - sum_j g_j dg_j) for each chosen m (the top-k
+ *             choice itself has no gradient), plus
+ *             p_te (a_e - sum_e' p_te' a_e'),  a_e = daux * E * f_e / T_batch
+ *   dx = dL @ W_router^T, dW_router = x^T @ dL, dbias = sum_t dL.
+ *   x (T, d) act_dtype; W_router (d, E) fp32; logits (T, E) fp32 (moe_route's
+ *   logits_out: the logits the top-k decided on, after bias and noise);
+ *   expert_indices, gates (T, top_k); f (E) fp32 (moe_dispatch's, before
+ *   capacity); dgates (T, top_k) fp32 (e.g. moe_combine_backward's); daux
+ *   (1) fp32 device: dLoss/d aux_loss; T_batch: tokens P_e and f_e are
+ *   means over (0 = this call's T; a rank's share of a sharded batch passes
+ *   the whole batch's T, and the ranks then add their dW and dbias).
+ *   dx (T, d) fp32 out; dW_router (d, E) fp32 out; dbias (E) fp32 out or
+ *   NULL; dlogits (T, E) fp32 out or NULL (kept in the workspace then).
+ * fp32 throughout with fixed summation orders (dW and dbias: token chunks
+ * in order). */
+int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_router,
+                       const float* logits, const int32_t* expert_indices, const float* gates,
+                       const float* f, const float* dgates, const float* daux, int32_t T_batch,
+                       float* dx, float* dW_router, float* dbias, float* dlogits, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Self-test of the library's failure detection; the pages have no
+ * counterpart.  Every pipeline wait in the library's kernels is bounded:
+ * instead of hanging, a wait that does not complete in time records an
+ * error code on the workspace's error word and the kernel returns, leaving
+ * the CUDA context usable.  This call runs one such wait on an mbarrier that
+ * nothing completes, with a limit of limit_us microseconds (1 .. 10^7), so
+ * a caller (or a health check) can see the mechanism work: afterwards
+ * moe_device_status reports code 20.  It faults nothing and holds the GPU
+ * for about limit_us.  ws needs only its first 256 bytes (the error word). */
+int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream);
 
 /* Static text for a status code. */
 const char* moe_status_string(int status);
