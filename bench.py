@@ -8,12 +8,21 @@ router), synthetic seeded inputs, random-init weights of that shape.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
-(data parallel, weak scaling, no collective on the data path); the step time
-is the max over ranks; value = tokens of all ranks / that time.
+Multi-GPU (launched by torch.distributed.run): one batch of N x T tokens is
+split over the ranks in contiguous blocks (weak scaling: T tokens per GPU);
+every step all-gathers each rank's exchange record (2E+1 ints: slot counts,
+probability means, token count) over NCCL, from which each rank's sharded
+dispatch takes the batch's capacity positions, f and P; the step time is the
+max over ranks; value = tokens of all ranks / that time.
+
+At N=1 the line's `extras.workloads` adds the other configurations (decode,
+fine-grained, Switch top-1, the small linear case), each timed the same way
+after the main timed region.
 
 The reference arm (--impl reference) times the CPU oracle, as it stands, on
-the host cores (rank 0 only), one token of the workload per step.
+the host cores (rank 0 only), one token of the workload per step, run as a
+batch of its own (so each step also widens that token's two experts' bf16
+weights to fp64).
 """
 from __future__ import annotations
 
@@ -31,6 +40,8 @@ import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+
+from mixture_experts_top_b200 import accounting as A  # noqa: E402  (pure-Python counts)
 
 METRIC = "MoE layer tokens/s at 1 B200 (Mixtral-shape bf16); GEMM % tensor peak, route GB/s"
 WORKLOAD = "mixtral"
@@ -113,18 +124,27 @@ def profiled_traffic(kernel_file: str, summary: str):
     return float(m_b.group(1))
 
 
-def launches_per_step(w, cfg) -> int:
+def fused_combine(w) -> bool:
+    """Top-1 with bf16 experts: the combine runs in the down projection's
+    epilogue (moe_expert_ffn_combine), with no combine kernel."""
+    return w.top_k == 1 and w.kind != "linear"
+
+
+def launches_per_step(w, cfg, world: int = 1) -> int:
     """Kernels of this library launched by one timed step (route, dispatch,
     experts, combine), as the library picks them for this configuration:
     route = weight split + tensor-core router + P mean (bf16, E <= 64) or
     SIMT router + P mean; dispatch = count + scan + scatter; experts = up and
-    down GEMM (bf16) or the fp32 linear kernel; combine = 1."""
+    down GEMM (bf16) or the fp32 linear kernel; combine = 1, or 0 where it is
+    fused into the down projection (top-1).  A rank of a split batch adds
+    its exchange record (count + total)."""
     from mixture_experts_top_b200 import api as _api
     if w.T == 0:
         return 2                       # P mean and the dispatch scan only
     route = 3 if _api.router_tc_width_supported(cfg) else 2
     experts = 1 if w.kind == "linear" else 2
-    return route + 3 + experts + 1
+    record = 2 if world > 1 else 0
+    return route + record + 3 + experts + (0 if fused_combine(w) else 1)
 
 
 # ------------------------------------------------------------- ranks (N>1) --
@@ -197,7 +217,8 @@ def run_reference(args, rank, world):
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle",
                          "sample": "one token of the batch per step, run as a batch of its own "
-                                   "through the full oracle forward"},
+                                   "through the full oracle forward in fp64 (each step widens "
+                                   "its experts' bf16 weights to fp64, which dominates)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -205,26 +226,368 @@ def run_reference(args, rank, world):
     return 0
 
 
+WORKLOAD_TITLES = {
+    "mixtral": "Mixtral-shaped SwiGLU MoE layer",
+    "decode": "Mixtral-shaped SwiGLU MoE layer, decode-sized batch",
+    "fine_grained": "fine-grained SwiGLU MoE layer with four hot experts",
+    "switch_relu": "Switch-style top-1 ReLU-MLP MoE layer with a noisy gate",
+    "tiny_linear": "small linear-expert MoE layer",
+}
+
+
+def describe(w) -> str:
+    """One-line description of a workload, from its own fields."""
+    expert = {"linear": f"linear experts (d_out={w.d_out})",
+              "relu": f"ReLU-MLP experts (DH={w.d_hidden})",
+              "swiglu": f"SwiGLU experts (DH={w.d_hidden})"}[w.kind]
+    cap = (f"capacity factor {w.capacity_factor:g} (ceil(cf*T*k/E) = "
+           f"{A.capacity_slots(w.capacity_factor, w.T, w.top_k, w.E)} slots per expert)"
+           if w.capacity_factor > 0 else "no capacity limit")
+    prec = ("bf16 tokens and weights, fp32 router and accumulation" if w.dtype == "bf16"
+            else "fp32 throughout")
+    extras = []
+    if w.n_hot:
+        extras.append(f"+{w.hot_bias:g} logit bias on {w.n_hot} seeded experts")
+    if w.noise:
+        extras.append("noise z*softplus(x@W_noise) made on the host")
+    return (f"{w.name}: {WORKLOAD_TITLES.get(w.name, 'MoE layer')}, T={w.T} tokens per GPU, "
+            f"d={w.d}, E={w.E}, top_k={w.top_k}, {expert}, {cap}, {prec}"
+            + ("; " + "; ".join(extras) if extras else ""))
+
+
+def l2_note(w) -> str:
+    nb = A.expert_weight_bytes(w.E, w.d, w.d_hidden, w.d_out, w.kind,
+                               2 if w.dtype == "bf16" else 4)
+    if nb > 126e6:
+        return (f"no flush: each step streams {nb / 1e9:.2f} GB of expert weights "
+                "(> 126 MB L2)")
+    return f"no flush: the whole layer ({nb / 1e3:.0f} KB of weights) stays in L2"
+
+
 def workload_config(w, n):
-    return {"workload": f"{w.name}: Mixtral-shaped SwiGLU MoE layer, T={w.T} tokens per GPU, "
-                        f"D={w.d}, DH={w.d_hidden}, E={w.E}, top_k={w.top_k}, bf16 with fp32 "
-                        "router and fp32 accumulation, no capacity limit",
-            "T": w.T, "d": w.d, "d_hidden": w.d_hidden, "E": w.E, "top_k": w.top_k,
+    par = ("dp1" if n == 1 else
+           f"dp{n}: one batch of {n} x {w.T} tokens split over the ranks in contiguous blocks, "
+           "replicated weights; per step one NCCL all-gather of each rank's 2E+1-int exchange "
+           "record (slot counts, probability means, tokens) couples the capacity and the aux loss")
+    return {"workload": describe(w),
+            "T": w.T, "d": w.d, "d_hidden": w.d_hidden, "d_out": w.d_out, "E": w.E,
+            "top_k": w.top_k, "capacity_factor": w.capacity_factor,
             "global_batch": w.T * n,
-            "parallelism": f"dp{n} (independent batch per GPU, replicated weights)",
-            "l2": "no flush: each step streams 2.8 GB of expert weights, > 126 MB L2"}
+            "parallelism": par,
+            "l2": l2_note(w)}
 
 
 # ---------------------------------------------------------------- our arm --
 
-def run_ours(args, rank, world):
+def to_device(inp):
     import numpy as np
+    import torch
+
+    def dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return {k: dev(v) for k, v in inp.items()}
+
+
+class LayerBench:
+    """Buffers and timed loops of one workload on this GPU: the staged step
+    (moe_route, moe_dispatch, moe_expert_ffn, moe_combine with device
+    inputs) and the end-to-end step (moe_forward with host copies)."""
+
+    def __init__(self, w, D, shard=None):
+        """shard = (rank, world, group): this rank's block of one batch of
+        world * T tokens, with the exchange of the ranks' records per step."""
+        import torch
+        from mixture_experts_top_b200 import api
+        from mixture_experts_top_b200 import shard as S
+        from mixture_experts_top_b200.layer import MoeForward
+        self.w, self.D, self.shard = w, D, shard
+        self.cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
+                                   w.capacity_factor)
+        self.layer = MoeForward(self.cfg)
+        T, k, E = w.T, w.top_k, w.E
+        R = T * k
+        i32 = dict(dtype=torch.int32, device="cuda")
+        act = D["x"].dtype
+        self.P = torch.empty(E, dtype=torch.float32, device="cuda")
+        self.offsets = torch.empty(E + 1, **i32)
+        self.dest = torch.empty(R, **i32)
+        self.perm = torch.empty(R, **i32)
+        self.f = torch.empty(E, dtype=torch.float32, device="cuda")
+        self.x_perm = torch.empty((R, w.d), dtype=act, device="cuda")
+        self.y_perm = torch.empty((R, w.d_out), dtype=torch.float32, device="cuda")
+        self.stream = torch.cuda.current_stream()
+        self.fused_combine = fused_combine(w)
+        if shard is not None:
+            self.record = torch.empty(S.record_ints(E), **i32)
+            self.records = torch.empty((shard[1], S.record_ints(E)), **i32)
+
+    def step(self, ev=None, marks=(0, 1, 2, 3, 4), x=None, noise=None, out=None, aux=None):
+        """One pass of the hot path (x, noise, out, aux: other buffers than
+        the bench's own, for the end-to-end loop).  ev[j] is recorded before stage j
+        (route, dispatch, experts, combine) and ev[4] after the last, for
+        the stage indices in `marks`.  Every recorded event separates two
+        launches that could otherwise overlap (each kernel is launched as a
+        programmatic dependent of the one before), so timed loops mark only
+        the expert stage."""
+        from mixture_experts_top_b200 import api
+        D, o, cfg, s = self.D, self.layer.out, self.cfg, self.stream
+
+        def mark(j):
+            if ev is not None and j in marks:
+                ev[j].record(s)
+        mark(0)
+        x = D["x"] if x is None else x
+        noise = D["noise"] if noise is None else noise
+        out = o.output if out is None else out
+        aux = o.aux_loss if aux is None else aux
+        api.moe_route(cfg, x, D["W_router"], D["logit_bias"], noise, o.expert_indices,
+                      o.gates, self.P, None, self.layer.ws)
+        if self.shard is not None:
+            # this rank's record, all-gathered (NCCL) in rank order
+            from mixture_experts_top_b200 import shard as S
+            rank, world, group = self.shard
+            api.moe_shard_record(cfg, o.expert_indices, self.P, self.record, self.layer.ws)
+            S.gather_records(self.record, self.records, group)
+        mark(1)
+        if self.shard is not None:
+            rank, world, _ = self.shard
+            api.moe_dispatch_shard(cfg, rank, world, world * self.w.T, self.records, x,
+                                   o.expert_indices, None, o.counts, self.offsets, self.dest,
+                                   self.perm, o.drop_mask, self.f, aux, self.x_perm,
+                                   self.layer.ws)
+        else:
+            api.moe_dispatch(cfg, x, o.expert_indices, self.P, o.counts, self.offsets,
+                             self.dest, self.perm, o.drop_mask, self.f, aux, self.x_perm,
+                             self.layer.ws)
+        mark(2)
+        if self.fused_combine:
+            # top-1: the combine is the down projection's epilogue
+            api.moe_expert_ffn_combine(cfg, self.x_perm, self.offsets, self.perm, self.dest,
+                                       o.gates, D["W_in"], D["W_up"], D["W_out"], out,
+                                       self.layer.ws)
+            mark(3)
+        else:
+            api.moe_expert_ffn(cfg, self.x_perm, self.offsets, D["W_in"], D["W_up"], D["W_out"],
+                               self.y_perm, self.layer.ws)
+            mark(3)
+            api.moe_combine(cfg, self.y_perm, self.dest, o.gates, out)
+        mark(4)
+
+    def timed(self, steps, warmup, barrier, clocks=None):
+        """Device-timed loop: returns (ms for all steps, mean experts ms)."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        barrier()
+        if clocks is not None:
+            clocks.start()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(self.stream)
+        for i in range(steps):
+            self.step(evs[i], marks=(2, 3))
+        end.record(self.stream)
+        barrier()
+        self._evs = evs
+        return start.elapsed_time(end), sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+
+    def stage_breakdown(self, steps, barrier):
+        """The same steps again with an event between every two stages
+        (diagnostic, outside the timed region): mean ms per stage."""
+        evs = self._evs
+        for i in range(steps):
+            self.step(evs[i])
+        barrier()
+        return [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j in range(4)]
+
+    def e2e(self, steps, warmup, barrier):
+        """End to end through the public call (moe_forward): every step
+        copies its tokens (and noise) from pinned host memory and its output
+        and aux_loss back to pinned host memory, on copy streams, double
+        buffered, so step i's upload and step i-1's download overlap step
+        i's compute.  Returns (ms for all steps, h2d bytes, d2h bytes)."""
+        import torch
+        from mixture_experts_top_b200 import api
+        D, o, cfg, stream = self.D, self.layer.out, self.cfg, self.stream
+        x, noise = D["x"], D["noise"]
+        x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x)
+        n_host = None if noise is None else torch.empty(noise.shape, dtype=noise.dtype,
+                                                        pin_memory=True).copy_(noise)
+        h2d = x.numel() * x.element_size() + (0 if noise is None else noise.numel() * 4)
+        d2h = o.output.numel() * o.output.element_size() + 4
+        s_up, s_dn = torch.cuda.Stream(), torch.cuda.Stream()
+        bufs = []
+        for _ in range(2):
+            bufs.append(dict(
+                x=torch.empty_like(x), noise=None if noise is None else torch.empty_like(noise),
+                out=torch.empty_like(o.output), aux=torch.empty_like(o.aux_loss),
+                out_host=torch.empty(o.output.shape, dtype=o.output.dtype, pin_memory=True),
+                aux_host=torch.empty(1, dtype=torch.float32, pin_memory=True),
+                uploaded=torch.cuda.Event(), computed=torch.cuda.Event(),
+                downloaded=torch.cuda.Event()))
+        self.ws_e2e = api.alloc_workspace(cfg)
+
+        def run(n):
+            for i in range(n):
+                b = bufs[i % 2]
+                with torch.cuda.stream(s_up):
+                    s_up.wait_event(b["computed"])   # step i-2 finished reading b["x"]
+                    b["x"].copy_(x_host, non_blocking=True)
+                    if noise is not None:
+                        b["noise"].copy_(n_host, non_blocking=True)
+                    b["uploaded"].record(s_up)
+                stream.wait_event(b["uploaded"])
+                stream.wait_event(b["downloaded"])   # step i-2's output was copied out
+                if self.shard is not None:
+                    # a rank of a split batch: its public calls in order
+                    self.step(x=b["x"], noise=b["noise"], out=b["out"], aux=b["aux"])
+                else:
+                    api.moe_forward(cfg, b["x"], D["W_router"], D["logit_bias"], b["noise"],
+                                    D["W_in"], D["W_up"], D["W_out"], b["out"],
+                                    o.expert_indices, o.gates, b["aux"], None, None,
+                                    self.ws_e2e)
+                b["computed"].record(stream)
+                with torch.cuda.stream(s_dn):
+                    s_dn.wait_event(b["computed"])
+                    b["out_host"].copy_(b["out"], non_blocking=True)
+                    b["aux_host"].copy_(b["aux"], non_blocking=True)
+                    b["downloaded"].record(s_dn)
+
+        run(warmup)
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        s_up.wait_stream(stream)                     # the first upload starts after s2
+        run(steps)
+        stream.wait_stream(s_dn)
+        e2.record(stream)
+        barrier()
+        return s2.elapsed_time(e2), h2d, d2h
+
+    def device_status(self):
+        from mixture_experts_top_b200 import api
+        st = self.layer.device_status()
+        if st == 0 and getattr(self, "ws_e2e", None) is not None:
+            st = api.moe_device_status(self.ws_e2e)
+        return st
+
+
+def gemm_roofline(w, rows, used, expert_ms, peaks, peak_src, regime):
+    """The expert GEMMs (both launches) against their binding roofline.
+    Algorithmic work: 2 FLOP per multiply-add of the kept rows; where
+    streaming the used experts' weights takes longer than the FLOPs take on
+    the tensor cores, the bound is HBM and the algorithmic bytes are the
+    used experts' weights + rows in + the hidden activation written and
+    read + fp32 rows out.  `regime` picks the tensor peak: "burst" (cuBLAS
+    timed alone; a timed region well under a second) or "sustained" (cuBLAS
+    back to back for seconds under the power cap)."""
+    flops = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
+    t = expert_ms / 1e3
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained") or burst
+    tensor_peak = burst if regime == "burst" else sustained
+    if w.kind == "linear":
+        # fp32 SIMT kernel: its peak is the fp32 FMA rate, not the tensor cores
+        tensor_peak = burst = sustained = None
+    hbm = peaks["hbm_gbs"]
+    elem = 4 if w.kind == "linear" else 2
+    # rows out: fp32 expert rows, or (top-1, combine in the epilogue) every
+    # token's bf16 output row
+    out_bytes = w.T * w.d_out * 2 if fused_combine(w) else rows * w.d_out * 4
+    gemm_bytes = (A.expert_weight_bytes(used, w.d, w.d_hidden, w.d_out, w.kind, elem)
+                  + rows * w.d * elem + out_bytes
+                  + (0 if w.kind == "linear" else 2 * rows * w.d_hidden * 2))
+    tensor_bound = tensor_peak is not None and \
+        flops / (tensor_peak * 1e12) >= gemm_bytes / (hbm * 1e9)
+    if tensor_bound:
+        ach = flops / t / 1e12
+        g = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
+             "frac": ach / tensor_peak, "frac_of_burst": ach / burst,
+             "frac_of_sustained": ach / sustained, "regime": regime,
+             "peak_source": f"{peak_src} {regime} bf16 (cuBLAS)"}
+    else:
+        ach = gemm_bytes / t / 1e9
+        g = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+             "peak_source": f"{peak_src} HBM copy bandwidth"}
+    g.update({"algorithmic_bytes": gemm_bytes, "algorithmic_flops": flops, "ms": expert_ms})
+    return g
+
+
+def stage_rooflines(w, rows, stage_ms, hbm):
+    elem = 2 if w.dtype == "bf16" else 4
+    rb = A.router_bytes(w.T, w.d, w.E, w.top_k, elem, w.noise)
+    pb = A.permute_bytes(w.T, rows, w.d, elem)
+    cb = A.combine_bytes(w.T, rows, w.d_out, w.top_k, elem)
+    out = {}
+    for name, ms, nb in (("route", stage_ms[0], rb), ("dispatch", stage_ms[1], pb),
+                         ("combine", stage_ms[3], cb)):
+        if name == "combine" and fused_combine(w):
+            out[name] = {"fused": "in the down projection's epilogue (no kernel)"}
+            continue
+        out[name] = {"ms": ms, "GB/s": nb / ms / 1e6, "frac_hbm": nb / ms / 1e6 / hbm,
+                     "algorithmic_bytes": nb}
+    return out
+
+
+def regime_of(timed_s: float) -> str:
+    """A timed region under two seconds runs at burst clocks (cuBLAS timed
+    alone is the matching peak); longer ones settle under the power cap."""
+    return "burst" if timed_s < 2.0 else "sustained"
+
+
+def extra_workload(name, steps, warmup, peaks, peak_src, base_inputs=None):
+    """tokens/s (device and end to end) and each stage's roofline fraction
+    of another configuration, on this GPU, outside the main timed region."""
+    import torch
+    from workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[name]
+    t0 = time.time()
+    if base_inputs is not None:
+        # the decode batch: the Mixtral-shaped weights (same seed, same shapes)
+        inp = make_inputs(w, seed=0, with_experts=False)
+        D = to_device(inp)
+        D.update({k: base_inputs[k] for k in ("W_in", "W_up", "W_out")})
+    else:
+        D = to_device(make_inputs(w, seed=0))
+    gen_s = time.time() - t0
+    lb = LayerBench(w, D)
+    sync = torch.cuda.synchronize
+    ms, expert_ms = lb.timed(steps, warmup, sync)
+    stage_ms = lb.stage_breakdown(steps, sync)
+    stage_ms[2] = expert_ms
+    e2e_ms, h2d, d2h = lb.e2e(steps, warmup, sync)
+    if lb.device_status() != 0:
+        raise RuntimeError(f"{name}: device error word set")
+    counts = lb.layer.out.counts.cpu().numpy()
+    rows = A.kept_rows(counts, w.capacity_factor, w.T, w.top_k)
+    used = int((counts > 0).sum())
+    regime = regime_of(ms / 1e3)
+    res = {
+        "workload": describe(w), "tokens_per_s": w.T / (ms / steps / 1e3),
+        "ms_per_step": ms / steps,
+        "e2e_tokens_per_s": w.T / (e2e_ms / steps / 1e3),
+        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "experts": gemm_roofline(w, rows, used, expert_ms, peaks, peak_src, regime),
+        "stages": stage_rooflines(w, rows, stage_ms, peaks["hbm_gbs"]),
+        "rows": rows, "used_experts": used,
+        "aux_loss": float(lb.layer.out.aux_loss.item()),
+        "steps": steps, "warmup": warmup, "inputs_s": gen_s,
+    }
+    del lb, D
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, rank, world):
     import torch
     import torch.distributed as dist
 
-    from mixture_experts_top_b200 import accounting as A
     from mixture_experts_top_b200 import api
-    from mixture_experts_top_b200.layer import MoeForward
     from workloads import WORKLOADS, make_inputs
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
@@ -241,142 +604,33 @@ def run_ours(args, rank, world):
                                                  with_experts=False).items()
                     if k in ("x", "noise")})
     log(f"[rank {rank}] inputs generated in {time.time() - t0:.1f}s")
-
-    def dev(a):
-        if a is None:
-            return None
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
-        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-    x, Wr, bias, noise = dev(inp["x"]), dev(inp["W_router"]), dev(inp["logit_bias"]), dev(inp["noise"])
-    W_in, W_up, W_out = dev(inp["W_in"]), dev(inp["W_up"]), dev(inp["W_out"])
-    W_noise = dev(inp["W_noise"])
+    D = to_device(inp)
     del inp
-    cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
-                          w.capacity_factor)
-    layer = MoeForward(cfg)
-    o = layer.out
+    # N > 1: one batch of N * T tokens split over the ranks in contiguous
+    # blocks (rank r holds tokens [r T, (r + 1) T)); the capacity and aux
+    # couple them through one all-gather of 2E+1 ints per rank and step.
+    lb = LayerBench(w, D, shard=(rank, world, None) if world > 1 else None)
+    cfg, o = lb.cfg, lb.layer.out
     T, k, E = w.T, w.top_k, w.E
-    R = T * k
-    i32 = dict(dtype=torch.int32, device="cuda")
-    P = torch.empty(E, dtype=torch.float32, device="cuda")
-    offsets = torch.empty(E + 1, **i32)
-    dest = torch.empty(R, **i32)
-    perm = torch.empty(R, **i32)
-    f = torch.empty(E, dtype=torch.float32, device="cuda")
-    x_perm = torch.empty((R, w.d), dtype=torch.bfloat16, device="cuda")
-    y_perm = torch.empty((R, w.d_out), dtype=torch.float32, device="cuda")
-    ws = layer.ws
-    stream = torch.cuda.current_stream()
-
-    def step(ev=None, marks=(0, 1, 2, 3, 4)):
-        # ev[j] is recorded before stage j (route, dispatch, experts, combine)
-        # and ev[4] after the last, for the stage indices listed in `marks`.
-        # Every recorded event separates two launches that could otherwise
-        # overlap (each kernel is launched as a programmatic dependent of the
-        # one before), so the timed loop marks only the expert stage.
-        def mark(j):
-            if ev is not None and j in marks:
-                ev[j].record(stream)
-        mark(0)
-        api.moe_route(cfg, x, Wr, bias, noise, o.expert_indices, o.gates, P, None, ws)
-        mark(1)
-        api.moe_dispatch(cfg, x, o.expert_indices, P, o.counts, offsets, dest, perm, o.drop_mask,
-                         f, o.aux_loss, x_perm, ws)
-        mark(2)
-        api.moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws)
-        mark(3)
-        api.moe_combine(cfg, y_perm, dest, o.gates, o.output)
-        mark(4)
+    stream = lb.stream
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(0).uuid)
     except Exception:
         pass
     clocks = ClockSampler(uuid)
-    clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    barrier()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(args.steps):
-        step(evs[i], marks=(2, 3))
-    end.record(stream)
-    barrier()
-    elapsed_ms = start.elapsed_time(end)
-    expert_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-
-    # Stage breakdown (diagnostic, outside the timed region): the same steps
-    # again with an event between every two stages.
-    for i in range(args.steps):
-        step(evs[i])
-    barrier()
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(4)]
+    elapsed_ms, expert_ms = lb.timed(args.steps, args.warmup, barrier, clocks)
+    stage_ms = lb.stage_breakdown(args.steps, barrier)
     stage_ms[2] = expert_ms
-
-    # End to end through the public call (moe_forward): every step copies its
-    # tokens from pinned host memory and its output and aux_loss back to pinned
-    # host memory.  Copies run on their own streams, double-buffered, so step
-    # i's upload and step i-1's download overlap step i's compute.
-    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x)
-    n_host = None if noise is None else torch.empty(noise.shape, dtype=noise.dtype,
-                                                    pin_memory=True).copy_(noise)
-    h2d = x.numel() * x.element_size() + (0 if noise is None else noise.numel() * 4)
-    d2h = o.output.numel() * o.output.element_size() + 4
-    s_up, s_dn = torch.cuda.Stream(), torch.cuda.Stream()
-    bufs = []
-    for _ in range(2):
-        bufs.append(dict(
-            x=torch.empty_like(x), noise=None if noise is None else torch.empty_like(noise),
-            out=torch.empty_like(o.output), aux=torch.empty_like(o.aux_loss),
-            out_host=torch.empty(o.output.shape, dtype=o.output.dtype, pin_memory=True),
-            aux_host=torch.empty(1, dtype=torch.float32, pin_memory=True),
-            uploaded=torch.cuda.Event(), computed=torch.cuda.Event(),
-            downloaded=torch.cuda.Event()))
-    ws_e2e = api.alloc_workspace(cfg)
-
-    def e2e_steps(n):
-        for i in range(n):
-            b = bufs[i % 2]
-            with torch.cuda.stream(s_up):
-                s_up.wait_event(b["computed"])       # step i-2 finished reading b["x"]
-                b["x"].copy_(x_host, non_blocking=True)
-                if noise is not None:
-                    b["noise"].copy_(n_host, non_blocking=True)
-                b["uploaded"].record(s_up)
-            stream.wait_event(b["uploaded"])
-            stream.wait_event(b["downloaded"])       # step i-2's output was copied out
-            api.moe_forward(cfg, b["x"], Wr, bias, b["noise"], W_in, W_up, W_out, b["out"],
-                            o.expert_indices, o.gates, b["aux"], None, None, ws_e2e)
-            b["computed"].record(stream)
-            with torch.cuda.stream(s_dn):
-                s_dn.wait_event(b["computed"])
-                b["out_host"].copy_(b["out"], non_blocking=True)
-                b["aux_host"].copy_(b["aux"], non_blocking=True)
-                b["downloaded"].record(s_dn)
-
-    e2e_steps(args.warmup)
-    barrier()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    s_up.wait_stream(stream)                         # the first upload starts after s2
-    e2e_steps(args.steps)
-    stream.wait_stream(s_dn)
-    e2.record(stream)
-    barrier()
-    e2e_ms = s2.elapsed_time(e2)
+    e2e_ms, h2d, d2h = lb.e2e(args.steps, args.warmup, barrier)
     clk = clocks.stop()
-    status = layer.device_status() or api.moe_device_status(ws_e2e)
+    status = lb.device_status()
     if status != 0:
         raise RuntimeError(f"device error word {status} after the benchmark")
 
@@ -386,19 +640,19 @@ def run_ours(args, rank, world):
     if rank != 0:
         return 0
 
+    extras = {}
     # The noisy gate's noise made on the device (moe_gate_noise), timed on
     # its own: the workload recipe hands the router a host-made noise tensor,
     # so this is not part of the step above.
-    extras = {}
-    if W_noise is not None and api.router_tc_width_supported(cfg):
+    if D.get("W_noise") is not None and api.router_tc_width_supported(cfg):
         noise_dev = torch.empty((T, E), dtype=torch.float32, device="cuda")
         for _ in range(3):
-            api.moe_gate_noise(cfg, x, W_noise, 7, 0, 0, noise_dev, ws)
+            api.moe_gate_noise(cfg, D["x"], D["W_noise"], 7, 0, 0, noise_dev, lb.layer.ws)
         n_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         reps = 20
         n_ev[0].record(stream)
         for i in range(reps):
-            api.moe_gate_noise(cfg, x, W_noise, 7, i, 0, noise_dev, ws)
+            api.moe_gate_noise(cfg, D["x"], D["W_noise"], 7, i, 0, noise_dev, lb.layer.ws)
         n_ev[1].record(stream)
         torch.cuda.synchronize()
         us = n_ev[0].elapsed_time(n_ev[1]) / reps * 1e3
@@ -409,78 +663,19 @@ def run_ours(args, rank, world):
                                         "(T,E) fp32 noise written), back to back, x in L2"}
 
     # The routing half of the backward (moe_combine_backward +
-    # moe_route_backward) on this step's intermediates, timed on its own.
-    Lg = torch.empty((T, E), dtype=torch.float32, device="cuda")
-    api.moe_route(cfg, x, Wr, bias, noise, o.expert_indices, o.gates, P, Lg, ws)
-    api.moe_dispatch(cfg, x, o.expert_indices, P, o.counts, offsets, dest, perm, o.drop_mask,
-                     f, o.aux_loss, x_perm, ws)
-    api.moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws)
-    dyb = torch.randn((T, w.d_out), device="cuda").to(o.output.dtype)
-    dyp = torch.empty((R, w.d_out), dtype=torch.float32, device="cuda")
-    dgb = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    dxb = torch.empty((T, w.d), dtype=torch.float32, device="cuda")
-    dWb = torch.empty((w.d, E), dtype=torch.float32, device="cuda")
-    dbb = torch.empty(E, dtype=torch.float32, device="cuda")
-    dab = torch.ones(1, dtype=torch.float32, device="cuda")
-
-    def backward_once():
-        api.moe_combine_backward(cfg, dyb, y_perm, dest, o.gates, dyp, dgb)
-        api.moe_route_backward(cfg, x, Wr, Lg, o.expert_indices, o.gates, f, dgb, dab, 0, dxb,
-                               dWb, dbb, None, ws)
-
-    for _ in range(3):
-        backward_once()
-    b_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    b_ev[0].record(stream)
-    for _ in range(10):
-        backward_once()
-    b_ev[1].record(stream)
-    torch.cuda.synchronize()
-    b_us = b_ev[0].elapsed_time(b_ev[1]) / 10 * 1e3
-    elem = 2 if w.dtype == "bf16" else 4
-    kept = int((dest >= 0).sum().item())
-    b_bytes = (T * w.d_out * elem + 2 * kept * w.d_out * 4
-               + T * E * 4 * 2 + T * w.d * (elem + 4) + T * k * 16)
-    extras["routing_backward"] = {
-        "us": b_us, "GB/s": b_bytes / b_us / 1e3, "frac_hbm": b_bytes / b_us / 1e3 / peaks["hbm_gbs"],
-        "note": "moe_combine_backward + moe_route_backward (6 launches): dy read, expert rows "
-                "read and their gradients written, logits and dlogits, x read and dx written"}
+    # moe_route_backward) and the experts' backward on this step's
+    # intermediates, each timed on its own.
+    if w.dtype == "bf16":
+        extras["routing_backward"] = routing_backward(w, lb, peaks)
+        extras["experts_backward"] = experts_backward(w, lb, peaks)
 
     counts = o.counts.cpu().numpy()
     rows = A.kept_rows(counts, w.capacity_factor, T, k)
     used = int((counts > 0).sum())
     ms_step = elapsed_ms / args.steps
     value = job_value(world, T, ms_step)
-    flops = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
-    t_exp = stage_ms[2] / 1e3
-    # The GEMMs run back to back for the whole timed loop (seconds at the power
-    # cap), so the sustained cuBLAS figure is the denominator; the burst
-    # fraction is given beside it.  Where the expert weights take longer to
-    # stream than the FLOPs take on the tensor cores (few rows per expert),
-    # the bound is HBM instead: algorithmic bytes = the used experts' weights
-    # + rows in + the hidden activation written and read + fp32 rows out.
-    tensor_peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
-    burst_peak = peaks["bf16_tflops"]
-    hbm = peaks["hbm_gbs"]
-    elem = 4 if w.kind == "linear" else 2
-    gemm_bytes = (A.expert_weight_bytes(used, w.d, w.d_hidden, w.d_out, w.kind, elem)
-                  + rows * w.d * elem + rows * w.d_out * 4
-                  + (0 if w.kind == "linear" else 2 * rows * w.d_hidden * 2))
-    tensor_bound = flops / (tensor_peak * 1e12) >= gemm_bytes / (hbm * 1e9)
-    kernel_note = ("grouped_gemm_kernel (2 launches per step: up-projection with fused "
-                   "activation, down-projection); achieved = algorithmic work of both / their "
-                   "summed time")
-    if tensor_bound:
-        gemm = {"bound": "tensor", "achieved": flops / t_exp / 1e12, "peak": tensor_peak,
-                "unit": "TFLOP/s", "frac": flops / t_exp / 1e12 / tensor_peak,
-                "frac_of_burst": flops / t_exp / 1e12 / burst_peak,
-                "peak_source": (f"{peak_src} sustained bf16 (cuBLAS back to back for 4 s)"
-                                if peaks.get("bf16_tflops_sustained") else
-                                f"{peak_src} burst bf16 (cuBLAS)")}
-    else:
-        gemm = {"bound": "hbm", "achieved": gemm_bytes / t_exp / 1e9, "peak": hbm,
-                "unit": "GB/s", "frac": gemm_bytes / t_exp / 1e9 / hbm,
-                "peak_source": f"{peak_src} HBM copy bandwidth"}
+    regime = regime_of(elapsed_ms / 1e3)
+    gemm = gemm_roofline(w, rows, used, stage_ms[2], peaks, peak_src, regime)
     # DRAM counters exist only for the captured workload (Mixtral shape, T = 8192).
     captured = w.name == "mixtral" and T == 8192 and w.d == 4096
     gemm.update({
@@ -488,24 +683,32 @@ def run_ours(args, rank, world):
                    else None,
         "traffic_note": "DRAM bytes of both launches of one step (ncu, Mixtral shape T=8192 "
                         "only), bytes per step",
-        "algorithmic_bytes": gemm_bytes, "algorithmic_flops": flops,
-        "kernel": kernel_note})
-    rb = A.router_bytes(T, w.d, E, k, 2, w.noise)
-    pb = A.permute_bytes(T, rows, w.d, 2)
-    cb = A.combine_bytes(T, rows, w.d_out, k, 2)
-    stages = {
-        "route": {"ms": stage_ms[0], "GB/s": rb / stage_ms[0] / 1e6, "frac_hbm": rb / stage_ms[0] / 1e6 / hbm},
-        "dispatch": {"ms": stage_ms[1], "GB/s": pb / stage_ms[1] / 1e6, "frac_hbm": pb / stage_ms[1] / 1e6 / hbm},
-        "experts": {"ms": stage_ms[2], "TFLOP/s": flops / t_exp / 1e12,
-                    "frac_tensor": flops / t_exp / 1e12 / tensor_peak},
-        "combine": {"ms": stage_ms[3], "GB/s": cb / stage_ms[3] / 1e6, "frac_hbm": cb / stage_ms[3] / 1e6 / hbm},
-        "note": "experts: events inside the timed loop; route, dispatch, combine: a second "
-                "pass of the same steps with an event between every two stages",
-    }
+        "kernel": "grouped_gemm_kernel (2 launches per step: up-projection with fused "
+                  "activation, down-projection); achieved = algorithmic work of both / their "
+                  "summed time (CUDA events on the launching stream, inside the timed loop)"})
+    stages = stage_rooflines(w, rows, stage_ms, peaks["hbm_gbs"])
+    stages["experts"] = {"ms": stage_ms[2], "frac": gemm["frac"], "bound": gemm["bound"]}
+    stages["note"] = ("experts: events inside the timed loop; route, dispatch, combine: a "
+                      "second pass of the same steps with an event between every two stages")
+
+    # The other configurations, each on this GPU after the main line's
+    # timed region (tokens/s, end to end, and each stage against its bound).
+    if world == 1 and not args.no_extras and args.workload == WORKLOAD and not args.tokens:
+        wl = {}
+        for name in ("decode", "fine_grained", "switch_relu", "tiny_linear"):
+            try:
+                wl[name] = extra_workload(name, args.steps, args.warmup, peaks, peak_src,
+                                          base_inputs=D if name == "decode" else None)
+            except Exception as exc:   # reported, never hidden
+                wl[name] = {"error": repr(exc)}
+            log(f"[extras] {name}: done")
+        extras["workloads"] = wl
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) random-init weights)",
         "config": workload_config(w, world),
         "roofline": gemm,
@@ -516,22 +719,127 @@ def run_ours(args, rank, world):
                 "api": "moe_forward via the Python binding; every step copies x from pinned host "
                        "memory and output + aux_loss back to pinned host memory, on copy "
                        "streams overlapped with the previous/next step's compute"},
-        "gpu_launches": launches_per_step(w, cfg) * args.steps,
+        "gpu_launches": launches_per_step(w, cfg, world) * args.steps,
         "clocks": clk,
         "routing": {"rows": rows, "used_experts": used, "aux_loss": float(o.aux_loss.item())},
     }
     if world == 1 and not args.no_cpu_baseline:
-        import numpy as np  # noqa: F811
-        from workloads import make_inputs as mk
-        inp = mk(w, seed=0)
-        times = oracle_token_steps(w, inp, list(range(args.cpu_tokens)))
-        line["cpu_baseline"] = {
-            "value": len(times) / sum(times), "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": f"{len(times)} tokens of the batch, each run as a batch of its own through "
-                      f"the full oracle forward ({sum(times):.1f} s of CPU work)"}
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def routing_backward(w, lb, peaks):
+    import torch
+    from mixture_experts_top_b200 import api
+    D, o, cfg, stream = lb.D, lb.layer.out, lb.cfg, lb.stream
+    T, k, E = w.T, w.top_k, w.E
+    Lg = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    api.moe_route(cfg, D["x"], D["W_router"], D["logit_bias"], D["noise"], o.expert_indices,
+                  o.gates, lb.P, Lg, lb.layer.ws)
+    api.moe_dispatch(cfg, D["x"], o.expert_indices, lb.P, o.counts, lb.offsets, lb.dest, lb.perm,
+                     o.drop_mask, lb.f, o.aux_loss, lb.x_perm, lb.layer.ws)
+    api.moe_expert_ffn(cfg, lb.x_perm, lb.offsets, D["W_in"], D["W_up"], D["W_out"], lb.y_perm,
+                       lb.layer.ws)
+    dyb = torch.randn((T, w.d_out), device="cuda").to(o.output.dtype)
+    dyp = torch.empty((T * k, w.d_out), dtype=torch.float32, device="cuda")
+    dgb = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    dxb = torch.empty((T, w.d), dtype=torch.float32, device="cuda")
+    dWb = torch.empty((w.d, E), dtype=torch.float32, device="cuda")
+    dbb = torch.empty(E, dtype=torch.float32, device="cuda")
+    dab = torch.ones(1, dtype=torch.float32, device="cuda")
+
+    def once():
+        api.moe_combine_backward(cfg, dyb, lb.y_perm, lb.dest, o.gates, dyp, dgb)
+        api.moe_route_backward(cfg, D["x"], D["W_router"], Lg, o.expert_indices, o.gates, lb.f,
+                               dgb, dab, 0, dxb, dWb, dbb, None, lb.layer.ws)
+
+    for _ in range(3):
+        once()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for _ in range(10):
+        once()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    us = ev[0].elapsed_time(ev[1]) / 10 * 1e3
+    elem = 2 if w.dtype == "bf16" else 4
+    kept = int((lb.dest >= 0).sum().item())
+    nb = (T * w.d_out * elem + 2 * kept * w.d_out * 4
+          + T * E * 4 * 2 + T * w.d * (elem + 4) + T * k * 16)
+    return {"us": us, "GB/s": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / peaks["hbm_gbs"],
+            "note": "moe_combine_backward + moe_route_backward (6 launches): dy read, expert rows "
+                    "read and their gradients written, logits and dlogits, x read and dx written"}
+
+
+def experts_backward(w, lb, peaks):
+    """moe_expert_ffn_backward on this step's grouped rows with a seeded
+    dy_perm: pack, recompute of the pre-activations, dH (with the activation
+    backward in its epilogue), dX and the weight gradients, back to back."""
+    import torch
+    from mixture_experts_top_b200 import api
+    D, o, cfg, stream = lb.D, lb.layer.out, lb.cfg, lb.stream
+    T, k, E = w.T, w.top_k, w.E
+    R = T * k
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    dyp = torch.randn((R, w.d_out), device="cuda", generator=gen)
+    dxp = torch.empty((R, w.d), device="cuda")
+    dWi = torch.empty(tuple(D["W_in"].shape), device="cuda")
+    dWu = None if D["W_up"] is None else torch.empty(tuple(D["W_up"].shape), device="cuda")
+    dWo = torch.empty(tuple(D["W_out"].shape), device="cuda")
+    bws = api.alloc_backward_workspace(cfg)
+
+    def once():
+        api.moe_expert_ffn_backward(cfg, lb.x_perm, lb.offsets, D["W_in"], D["W_up"], D["W_out"],
+                                    dyp, dxp, dWi, dWu, dWo, bws)
+
+    for _ in range(2):
+        once()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    reps = 5
+    ev[0].record(stream)
+    for _ in range(reps):
+        once()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    if api.moe_device_status(bws) != 0:
+        raise RuntimeError("experts' backward: device error word set")
+    ms = ev[0].elapsed_time(ev[1]) / reps
+    counts = o.counts.cpu().numpy()
+    rows = A.kept_rows(counts, w.capacity_factor, T, k)
+    mats = A.MATRICES[w.kind]
+    fwd = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
+    algo = 2 * fwd                     # dgrad + wgrad: two products per forward product
+    executed = algo + (fwd * (mats - 1) // mats)   # + the recomputed up projection(s)
+    ach = algo / (ms / 1e3) / 1e12
+    del dyp, dxp, dWi, dWu, dWo, bws
+    torch.cuda.empty_cache()
+    return {"ms": ms, "TFLOP/s": ach, "frac_of_burst": ach / peaks["bf16_tflops"],
+            "algorithmic_flops": algo, "executed_flops": executed,
+            "note": "moe_expert_ffn_backward (pack, recompute of the pre-activations, dH with "
+                    "the activation backward fused, dX, weight gradients): algorithmic FLOPs = "
+                    "the dgrad and wgrad products (2x the forward's), executed adds the "
+                    "recomputed up projection; back to back, 5 calls"}
+
+
+def cpu_baseline(w, tokens):
+    """The oracle, as it stands, on one batch of `tokens` tokens of the
+    workload (its first tokens), timed on the host cores."""
+    from oracle import moe_oracle as O
+    from workloads import make_inputs
+    inp = make_inputs(w, seed=0)
+    n = min(tokens, w.T)
+    weights = {k: inp[k] for k in ("W_in", "W_up", "W_out")}
+    t0 = time.perf_counter()
+    O.moe_forward(inp["x"][:n], inp["W_router"], weights, top_k=w.top_k, kind=w.kind,
+                  dtype=w.dtype, d_out=w.d_out, capacity_factor=w.capacity_factor,
+                  logit_bias=inp["logit_bias"],
+                  noise=None if inp["noise"] is None else inp["noise"][:n])
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one batch of the workload's first {n} tokens through the full oracle "
+                      f"forward in fp64 ({dt:.1f} s of CPU work, which includes widening the "
+                      "used experts' bf16 weights to fp64 once per expert)"}
 
 
 def main():
@@ -543,8 +851,11 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling; not a bench line)")
-    ap.add_argument("--cpu-tokens", type=int, default=8)
+    ap.add_argument("--cpu-tokens", type=int, default=64,
+                    help="tokens in the oracle's timed batch (cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations' figures (extras.workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -111,8 +111,9 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * *code_out (0 = no device-side error since the last clear) and clears it.
  * The word holds the first error recorded: 1 an expert index outside [0, E);
  * 2 offsets that are not a partition of the row buffer; 3 a gathered row
- * index (perm_token) outside [0, T); 4 a sharded dispatch whose all_counts
- * row for this rank is not its own counts; 20 moe_check_wait_timeout's
+ * index (perm_token) outside [0, T); 4 a sharded dispatch whose exchange
+ * record for this rank is not its own, or whose records' token counts do
+ * not add up to T_global; 20 moe_check_wait_timeout's
  * intended timeout; 16-19 a pipeline wait that ran out of
  * time (TMA producer, MMA issuer, epilogue, teardown drain).
  * Returns MOE_ERR_DEVICE_CHECK if the word was non-zero, MOE_OK otherwise. */
@@ -184,8 +185,13 @@ int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise,
  *   different streams, or from different host threads without ordering)
  *   race on it; order such calls on one stream.
  *   Set-up: the first call on each device looks up the array's device
- *   address (with that device current) and caches it; make that first call
- *   before any stream capture.  No call allocates or frees memory.
+ *   address (with that device current) and caches it with the id of the
+ *   device's current context; make that first call before any stream
+ *   capture.  The cache does not outlive the context: after cudaDeviceReset
+ *   (or any new context on the device) the module is loaded again, the
+ *   array may move, and the next call looks the address up afresh -- so
+ *   that call, too, should come before any capture.  No call allocates or
+ *   frees memory.
  *   Arithmetic: this entry point always computes the logits on the fp32
  *   pipes (it has no room for moe_route's split copy of W_router), so its
  *   logits may differ from moe_route's in the last bits; both are fp32 dot
@@ -229,25 +235,35 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_i
  * exactly the slots the single-batch layer would.  [MLG Algorithm 3-4 and
  * Follow-up: positions in token order, capacity from the batch size; the
  * pages do not split a batch, so this is the single-batch rule restated]
+ * Each rank contributes one exchange record of 2E+1 int32 (moe_shard_record):
+ * its E slot counts per expert, its E probability means P_e over its own
+ * tokens (fp32 bit patterns) and its token count.  The caller gathers every
+ * rank's record in rank order (an all-gather of 2E+1 ints per rank: NCCL or
+ * any collective; the library keeps to one GPU) and passes them here:
  *   rank, world   this rank and the number of ranks (0 <= rank < world)
  *   T_global      tokens of the whole batch (every rank's cfg->T summed)
- *   all_counts    (world, E) int32 device: every rank's moe_dispatch_count
- *                 result in rank order (an all-gather of E ints per rank)
- * prob_mean given to moe_dispatch_shard must be the whole batch's P (the
- * token-weighted mean of the ranks' moe_route outputs: an all-reduce of E
- * floats).  Moving these two small arrays between GPUs is the caller's
- * (NCCL or any collective); the library keeps to one GPU. */
+ *   records       (world, 2E+1) int32 device: every rank's record in rank order
+ * From the records moe_dispatch_shard takes the earlier ranks' slots per
+ * expert, the batch's f_e, and the batch's P_e = (sum over ranks r in order
+ * of P_e(r) * T(r)) / T_global in fp64, rounded to fp32. */
 typedef struct {
   int32_t rank;
   int32_t world;
   int32_t T_global;
-  const int32_t* all_counts;
+  const int32_t* records;
 } moe_shard_t;
 
 /* Per-expert slot counts of expert_indices (T, top_k) into counts (E) int32
- * (before any capacity): this rank's contribution to all_counts. */
+ * (before any capacity). */
 int moe_dispatch_count(const moe_config_t* cfg, const int32_t* expert_indices, int32_t* counts,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* This rank's exchange record (see moe_shard_t) into record (2E+1) int32:
+ * the slot counts of expert_indices (T, top_k) per expert, the fp32 bits of
+ * prob_mean (E) (moe_route's P over this rank's tokens) and cfg->T. */
+int moe_shard_record(const moe_config_t* cfg, const int32_t* expert_indices,
+                     const float* prob_mean, int32_t* record, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
 
 /* moe_dispatch for one rank of a sharded batch (see moe_shard_t).  Outputs
  * as moe_dispatch, with: counts = this rank's slots per expert; offsets,
@@ -255,8 +271,10 @@ int moe_dispatch_count(const moe_config_t* cfg, const int32_t* expert_indices, i
  * grouped layout); drop_mask holds the whole batch's keep decision for this
  * rank's slots (capacity = ceil(((capacity_factor * T_global) * top_k) / E),
  * positions offset by earlier ranks' slots); f and aux_loss are the whole
- * batch's and the same on every rank.  A rank whose row of all_counts
- * differs from its own counts records device error 4. */
+ * batch's and the same on every rank.  prob_mean is not read (may be NULL):
+ * the batch's P comes from the records.  A rank whose record's counts differ
+ * from its own, or records whose token counts do not add up to T_global,
+ * record device error 4. */
 int moe_dispatch_shard(const moe_config_t* cfg, const moe_shard_t* shard, const void* x,
                        const int32_t* expert_indices, const float* prob_mean, int32_t* counts,
                        int32_t* offsets, int32_t* dest, int32_t* perm_token, uint8_t* drop_mask,
@@ -303,6 +321,23 @@ int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t*
                           const int32_t* offsets, const void* W_in, const void* W_up,
                           const void* W_out, void* y_perm, void* ws, size_t ws_bytes,
                           moe_stream_t stream);
+
+/* The experts and the combine in one call: output as moe_combine would
+ * write it from moe_expert_ffn's rows.  [MLG Algorithm 3; PFD Switch: top-1,
+ * a dropped token outputs 0]  With top_k = 1 and bf16 experts the combine
+ * is the down projection's epilogue: each kept grouped row r writes
+ * gates[t] * row into output row t = perm_token[r] (the same fp32 product
+ * and one rounding as moe_combine, so the same bits), tokens whose slot was
+ * dropped get a zero row, and neither y_perm nor a combine kernel is used.
+ * Otherwise it runs moe_expert_ffn into the workspace's y_perm, then the
+ * combine kernel.
+ *   x_perm, offsets, perm_token, dest, gates: moe_dispatch's (and
+ *   moe_route's) outputs; W_in, W_up, W_out as in moe_expert_ffn;
+ *   output (T, d_out) act_dtype out. */
+int moe_expert_ffn_combine(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                           const int32_t* perm_token, const int32_t* dest, const float* gates,
+                           const void* W_in, const void* W_up, const void* W_out, void* output,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Combine: output[t] = sum over j = 0..top_k-1 with dest[t,j] >= 0 of
  * gates[t,j] * y_perm[dest[t,j]], accumulated in fp32 in increasing j,
@@ -364,6 +399,56 @@ int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_ro
                        const float* f, const float* dgates, const float* daux, int32_t T_batch,
                        float* dx, float* dW_router, float* dbias, float* dlogits, void* ws,
                        size_t ws_bytes, moe_stream_t stream);
+
+/* Backward of the experts, for training.  The pages print no backward; these
+ * are the derivatives of moe_expert_ffn's experts ([MLG Algorithm 3]: each
+ * expert on its routed rows; [PFD The code, `expert_forward`]: the ReLU
+ * expert; SwiGLU as in moe_expert_ffn; [PFD Hot shards]: an expert that
+ * receives no row gets no gradient).  For the rows X of expert e, the
+ * gradient dY of its outputs, A = X W_in (B = X W_up) and H the hidden
+ * activation:
+ *   dH = dY W_out^T
+ *   ReLU:   dA = dH * [A > 0]
+ *   SwiGLU: s = sigmoid(A), dA = dH * B * s (1 + A (1 - s)), dB = dH * A s
+ *   dX = dA W_in^T (+ dB W_up^T);  dW_out = H^T dY, dW_in = X^T dA,
+ *   dW_up = X^T dB.  Linear experts: dX = dY W_in^T, dW_in = X^T dY.
+ *
+ * moe_expert_backward_workspace_size: bytes of the workspace this call
+ *   needs (its own, not moe_workspace_size's; 0 on a bad config).  Its
+ *   first 256 bytes are an error word like the forward workspace's
+ *   (moe_workspace_init / moe_device_status apply).
+ * moe_expert_ffn_backward:
+ *   x_perm  (T*top_k, d) act_dtype, offsets (E+1) int32: moe_dispatch's
+ *           grouped rows and their expert ranges
+ *   W_in, W_up, W_out as in moe_expert_ffn (W_up NULL unless SwiGLU,
+ *           W_out NULL for linear experts)
+ *   dy_perm (T*top_k, d_out) fp32: gradient of each kept row's expert output
+ *           (moe_combine_backward's dy_perm)
+ *   dx_perm (T*top_k, d) fp32 out: gradient of each kept grouped row; rows
+ *           at and beyond offsets[E] untouched
+ *   dW_in, dW_up, dW_out fp32 out, shaped like the weights (E, in, out);
+ *           NULL where the weight is NULL; every expert's block is written
+ *           (zeros for an expert without rows)
+ * bf16 experts run on the tensor cores (bf16 operands, fp32 accumulation):
+ * the rows are copied into a layout padded to 128 rows per expert, dY is
+ * rounded to bf16, the forward's A and B are recomputed and kept as bf16,
+ * dA, dB and H are rounded to bf16 between the GEMMs.  Linear experts run
+ * in fp32.  Deterministic: no atomics, fixed summation orders. */
+size_t moe_expert_backward_workspace_size(const moe_config_t* cfg);
+int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                            const void* W_in, const void* W_up, const void* W_out,
+                            const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
+                            float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_permute_backward: the grouped rows' input gradients back to their
+ * tokens, dx[t] = dx_add[t] + sum over kept slots j (j increasing) of
+ * dx_perm[dest[t, j]] (each token's input feeds its kept rows; [MLG
+ * Algorithm 3]).  dx_perm (T*top_k, d) fp32; dest (T, top_k) int32 from
+ * moe_dispatch; dx_add (T, d) fp32 or NULL (e.g. moe_route_backward's dx, so
+ * that dx is the whole layer's input gradient); dx (T, d) fp32 out (may be
+ * dx_add).  fp32, fixed order, no workspace. */
+int moe_permute_backward(const moe_config_t* cfg, const float* dx_perm, const int32_t* dest,
+                         const float* dx_add, float* dx, moe_stream_t stream);
 
 /* Self-test of the library's failure detection; the pages have no
  * counterpart.  Every pipeline wait in the library's kernels is bounded:

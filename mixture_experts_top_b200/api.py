@@ -32,6 +32,9 @@ _SIGNATURES = {
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
     "moe_check_wait_timeout": (ctypes.c_int, [_c_p, ctypes.c_size_t, ctypes.c_uint32, _c_p]),
+    "moe_expert_backward_workspace_size": (ctypes.c_size_t, [_c_p]),
+    "moe_expert_ffn_backward": (ctypes.c_int, [_c_p] * 12 + [ctypes.c_size_t, _c_p]),
+    "moe_permute_backward": (ctypes.c_int, [_c_p] * 6),
     "moe_combine_backward": (ctypes.c_int, [_c_p] * 8),
     "moe_route_backward": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_int32] + [_c_p] * 5 +
                            [ctypes.c_size_t, _c_p]),
@@ -40,10 +43,12 @@ _SIGNATURES = {
                                                    _c_p]),
     "moe_dispatch": (ctypes.c_int, [_c_p] * 13 + [ctypes.c_size_t, _c_p]),
     "moe_dispatch_count": (ctypes.c_int, [_c_p] * 4 + [ctypes.c_size_t, _c_p]),
+    "moe_shard_record": (ctypes.c_int, [_c_p] * 5 + [ctypes.c_size_t, _c_p]),
     "moe_dispatch_shard": (ctypes.c_int, [_c_p] * 14 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn": (ctypes.c_int, [_c_p] * 8 + [ctypes.c_size_t, _c_p]),
     "moe_expert_ffn_gather": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_size_t, _c_p]),
     "moe_combine": (ctypes.c_int, [_c_p] * 6),
+    "moe_expert_ffn_combine": (ctypes.c_int, [_c_p] * 11 + [ctypes.c_size_t, _c_p]),
     "moe_forward": (ctypes.c_int, [_c_p] * 15 + [ctypes.c_size_t, _c_p]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_error_message": (ctypes.c_char_p, []),
@@ -65,9 +70,10 @@ class MoeConfig(ctypes.Structure):
 
 
 class MoeShard(ctypes.Structure):
-    """Mirror of ``moe_shard_t``: this rank of a batch split over ranks."""
+    """Mirror of ``moe_shard_t``: this rank of a batch split over ranks and
+    every rank's exchange record (world, 2E+1) int32."""
     _fields_ = [("rank", ctypes.c_int32), ("world", ctypes.c_int32), ("T_global", ctypes.c_int32),
-                ("all_counts", ctypes.c_void_p)]
+                ("records", ctypes.c_void_p)]
 
 
 def make_config(T: int, d: int, d_hidden: int, d_out: int, E: int, top_k: int, kind: str,
@@ -190,6 +196,36 @@ def moe_route_backward(cfg, x, W_router, logits, expert_indices, gates, f, dgate
         _ptr(dbias), _ptr(dlogits), _ptr(ws), ws.numel(), _stream(stream)), "moe_route_backward")
 
 
+def moe_expert_backward_workspace_size(cfg: MoeConfig) -> int:
+    n = load_library().moe_expert_backward_workspace_size(ctypes.byref(cfg))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_expert_backward_workspace_size",
+                       load_library().moe_last_error_message().decode())
+    return n
+
+
+def alloc_backward_workspace(cfg: MoeConfig, device="cuda", stream=None):
+    """Caller-owned workspace of moe_expert_ffn_backward, error word cleared."""
+    import torch
+    ws = torch.empty(moe_expert_backward_workspace_size(cfg), dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream)
+    return ws
+
+
+def moe_expert_ffn_backward(cfg, x_perm, offsets, W_in, W_up, W_out, dy_perm, dx_perm, dW_in,
+                            dW_up, dW_out, ws, stream=None) -> None:
+    _check(load_library().moe_expert_ffn_backward(
+        ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(W_in), _ptr(W_up), _ptr(W_out),
+        _ptr(dy_perm), _ptr(dx_perm), _ptr(dW_in), _ptr(dW_up), _ptr(dW_out), _ptr(ws),
+        ws.numel(), _stream(stream)), "moe_expert_ffn_backward")
+
+
+def moe_permute_backward(cfg, dx_perm, dest, dx_add, dx, stream=None) -> None:
+    _check(load_library().moe_permute_backward(
+        ctypes.byref(cfg), _ptr(dx_perm), _ptr(dest), _ptr(dx_add), _ptr(dx), _stream(stream)),
+        "moe_permute_backward")
+
+
 def moe_check_wait_timeout(ws, limit_us: int, stream=None) -> None:
     _check(load_library().moe_check_wait_timeout(_ptr(ws), ws.numel(), int(limit_us),
                                                   _stream(stream)), "moe_check_wait_timeout")
@@ -215,10 +251,16 @@ def moe_dispatch_count(cfg, expert_indices, counts, ws, stream=None) -> None:
         _stream(stream)), "moe_dispatch_count")
 
 
-def moe_dispatch_shard(cfg, rank, world, T_global, all_counts, x, expert_indices, prob_mean,
+def moe_shard_record(cfg, expert_indices, prob_mean, record, ws, stream=None) -> None:
+    _check(load_library().moe_shard_record(
+        ctypes.byref(cfg), _ptr(expert_indices), _ptr(prob_mean), _ptr(record), _ptr(ws),
+        ws.numel(), _stream(stream)), "moe_shard_record")
+
+
+def moe_dispatch_shard(cfg, rank, world, T_global, records, x, expert_indices, prob_mean,
                        counts, offsets, dest, perm_token, drop_mask, f, aux_loss, x_perm, ws,
                        stream=None) -> None:
-    shard = MoeShard(rank, world, T_global, _ptr(all_counts))
+    shard = MoeShard(rank, world, T_global, _ptr(records))
     _check(load_library().moe_dispatch_shard(
         ctypes.byref(cfg), ctypes.byref(shard), _ptr(x), _ptr(expert_indices), _ptr(prob_mean),
         _ptr(counts), _ptr(offsets), _ptr(dest), _ptr(perm_token), _ptr(drop_mask), _ptr(f),
@@ -237,6 +279,14 @@ def moe_expert_ffn_gather(cfg, x, perm_token, offsets, W_in, W_up, W_out, y_perm
     _check(load_library().moe_expert_ffn_gather(
         ctypes.byref(cfg), _ptr(x), _ptr(perm_token), _ptr(offsets), _ptr(W_in), _ptr(W_up),
         _ptr(W_out), _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn_gather")
+
+
+def moe_expert_ffn_combine(cfg, x_perm, offsets, perm_token, dest, gates, W_in, W_up, W_out,
+                           output, ws, stream=None) -> None:
+    _check(load_library().moe_expert_ffn_combine(
+        ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(perm_token), _ptr(dest), _ptr(gates),
+        _ptr(W_in), _ptr(W_up), _ptr(W_out), _ptr(output), _ptr(ws), ws.numel(), _stream(stream)),
+        "moe_expert_ffn_combine")
 
 
 def moe_combine(cfg, y_perm, dest, gates, output, stream=None) -> None:

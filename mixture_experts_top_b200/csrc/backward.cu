@@ -189,32 +189,37 @@ __global__ void __launch_bounds__(256)
   __shared__ float ws[kEb][256];
   __shared__ float dls[kTg][kEb];
   const int c = blockIdx.x * 256 + threadIdx.x;
-  const int t0 = blockIdx.y * kTg;
-  float acc[kTg];
+  // Token groups are strided over grid.y (at most 65535 rows of CTAs), so
+  // any T is covered; each group's arithmetic is unchanged.
+  const int ngroups = (T + kTg - 1) / kTg;
+  for (int tg = blockIdx.y; tg < ngroups; tg += gridDim.y) {
+    const int t0 = tg * kTg;
+    float acc[kTg];
 #pragma unroll
-  for (int i = 0; i < kTg; ++i) acc[i] = 0.f;
-  for (int e0 = 0; e0 < E; e0 += kEb) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kEb * 256; i += 256) {
-      const int e = i / 256, cc = blockIdx.x * 256 + i % 256;
-      ws[e][i % 256] = (e0 + e < E && cc < d) ? W[(size_t)cc * E + e0 + e] : 0.f;
-    }
-    for (int i = threadIdx.x; i < kTg * kEb; i += 256) {
-      const int tt = i / kEb, e = i % kEb;
-      dls[tt][e] = (t0 + tt < T && e0 + e < E) ? dlogits[(size_t)(t0 + tt) * E + e0 + e] : 0.f;
-    }
-    __syncthreads();
-    const int ne = min(kEb, E - e0);
-    for (int e = 0; e < ne; ++e) {
-      const float wv = ws[e][threadIdx.x];
+    for (int i = 0; i < kTg; ++i) acc[i] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += kEb) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < kEb * 256; i += 256) {
+        const int e = i / 256, cc = blockIdx.x * 256 + i % 256;
+        ws[e][i % 256] = (e0 + e < E && cc < d) ? W[(size_t)cc * E + e0 + e] : 0.f;
+      }
+      for (int i = threadIdx.x; i < kTg * kEb; i += 256) {
+        const int tt = i / kEb, e = i % kEb;
+        dls[tt][e] = (t0 + tt < T && e0 + e < E) ? dlogits[(size_t)(t0 + tt) * E + e0 + e] : 0.f;
+      }
+      __syncthreads();
+      const int ne = min(kEb, E - e0);
+      for (int e = 0; e < ne; ++e) {
+        const float wv = ws[e][threadIdx.x];
 #pragma unroll
-      for (int i = 0; i < kTg; ++i) acc[i] = fmaf(dls[i][e], wv, acc[i]);
+        for (int i = 0; i < kTg; ++i) acc[i] = fmaf(dls[i][e], wv, acc[i]);
+      }
     }
+    if (c < d)
+#pragma unroll
+      for (int i = 0; i < kTg; ++i)
+        if (t0 + i < T) dx[(size_t)(t0 + i) * d + c] = acc[i];
   }
-  if (c < d)
-#pragma unroll
-    for (int i = 0; i < kTg; ++i)
-      if (t0 + i < T) dx[(size_t)(t0 + i) * d + c] = acc[i];
 }
 
 constexpr int kCt = 64;           // columns of x per dW CTA
@@ -330,7 +335,8 @@ cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const fl
                                 dgates, f, daux, c.T, c.E, c.top_k,
                                 (double)c.E / (double)T_batch, dlogits);
   if (e != cudaSuccess) return e;
-  e = launch_kernel(route_dx_kernel, dim3((unsigned)ceil_div(c.d, 256), (unsigned)ceil_div(c.T, kTg)),
+  e = launch_kernel(route_dx_kernel,
+                    dim3((unsigned)ceil_div(c.d, 256), (unsigned)std::min(ceil_div(c.T, kTg), 65535)),
                     256, 0, s, 0, dlogits, W, c.T, c.d, c.E, dx);
   if (e != cudaSuccess) return e;
   const int nchunks = route_backward_chunks(c.T);

@@ -101,13 +101,15 @@ __global__ void __launch_bounds__(1024)
                          int k, int64_t cap, const float* __restrict__ prob_mean,
                          int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, float* __restrict__ f,
-                         float* __restrict__ aux, const int32_t* __restrict__ all_counts,
+                         float* __restrict__ aux, const int32_t* __restrict__ records,
                          int rank, int world, int T_global, int32_t* __restrict__ prefix,
                          int32_t* err) {
   pdl_wait_and_release();
   __shared__ int32_t s_counts[kMaxE];
   __shared__ int32_t s_prefix[kMaxE];   // slots of earlier ranks (sharded batch), else 0
   __shared__ int32_t s_total[kMaxE];    // slots of the whole batch
+  __shared__ float s_P[kMaxE];          // P_e of the batch (sharded) or prob_mean
+  const int rec = 2 * E + 1;            // ints per exchange record
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int e = warp; e < E; e += nwarps) {
     int carry = 0;
@@ -122,24 +124,40 @@ __global__ void __launch_bounds__(1024)
   }
   // Sharded batch: this rank's tokens follow those of ranks 0..rank-1 in
   // the batch order, so a slot's position on its expert is offset by their
-  // slots on it; the capacity, f and aux are those of the whole batch.
+  // slots on it; the capacity, f and aux are those of the whole batch, and
+  // P_e is the token-weighted mean of the ranks' P_e, summed in fp64 in rank
+  // order and rounded once to fp32.
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int pre = 0, tot = 0;
-    if (all_counts != nullptr) {
+    float P = 0.f;
+    if (records != nullptr) {
+      double acc = 0.0;
       for (int r = 0; r < world; ++r) {
-        const int v = all_counts[(size_t)r * E + e];
+        const int32_t* rr = records + (size_t)r * rec;
+        const int v = rr[e];
         if (r < rank) pre += v;
         tot += v;
+        acc += (double)__int_as_float(rr[E + e]) * (double)rr[2 * E];
       }
       prefix[e] = pre;
+      P = T_global > 0 ? (float)(acc / (double)T_global) : 0.f;
+    } else {
+      P = prob_mean[e];
     }
     s_prefix[e] = pre;
-    s_total[e] = all_counts != nullptr ? tot : 0;
+    s_total[e] = records != nullptr ? tot : 0;
+    s_P[e] = P;
   }
   __syncthreads();
-  if (all_counts != nullptr) {
+  if (records != nullptr) {
     for (int e = threadIdx.x; e < E; e += blockDim.x)
-      if (all_counts[(size_t)rank * E + e] != s_counts[e]) report_error(err, kDevBadShard);
+      if (records[(size_t)rank * rec + e] != s_counts[e]) report_error(err, kDevBadShard);
+    if (threadIdx.x == 0) {
+      long long tokens = 0;
+      for (int r = 0; r < world; ++r) tokens += records[(size_t)r * rec + 2 * E];
+      if (tokens != (long long)T_global || records[(size_t)rank * rec + 2 * E] != T)
+        report_error(err, kDevBadShard);
+    }
   }
   if (warp == 0) {
     int run = 0;
@@ -157,13 +175,13 @@ __global__ void __launch_bounds__(1024)
     }
     if (lane == 0) offsets[E] = run;
   } else if (warp == 1) {
-    const bool sharded = all_counts != nullptr;
+    const bool sharded = records != nullptr;
     const double slots = (double)(sharded ? T_global : T) * (double)k;
     double acc = 0.0;
     for (int e = lane; e < E; e += 32) {
       const double fe = slots > 0.0 ? (double)(sharded ? s_total[e] : s_counts[e]) / slots : 0.0;
       f[e] = (float)fe;
-      acc += fe * (double)prob_mean[e];
+      acc += fe * (double)s_P[e];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -236,7 +254,7 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
   cudaError_t e = launch_kernel(
       dispatch_scan_kernel, 1, 1024, 0, s, 0, chunk_counts, nchunks, c.E, c.T, c.top_k, cap,
       prob_mean, chunk_base, counts, offsets, f, aux,
-      shard != nullptr ? shard->all_counts : nullptr, shard != nullptr ? shard->rank : 0,
+      shard != nullptr ? shard->records : nullptr, shard != nullptr ? shard->rank : 0,
       shard != nullptr ? shard->world : 1, shard != nullptr ? shard->T_global : c.T,
       shard != nullptr ? shard_prefix : nullptr, err);
   if (e != cudaSuccess || c.T == 0) return e;
@@ -250,21 +268,25 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
 }
 
 // Slots per expert of these expert indices (the histogram every rank of a
-// sharded batch contributes before the sharded dispatch).
+// sharded batch contributes before the sharded dispatch); with prob_mean,
+// the rank's whole exchange record: counts, the bits of prob_mean, T.
 __global__ void __launch_bounds__(256)
     dispatch_total_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                          int32_t* __restrict__ counts) {
+                          int32_t* __restrict__ counts, const float* __restrict__ prob_mean,
+                          int T) {
   pdl_wait_and_release();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int v = 0;
     for (int c = 0; c < nchunks; ++c) v += chunk_counts[(size_t)c * E + e];
     counts[e] = v;
+    if (prob_mean != nullptr) counts[E + e] = __float_as_int(prob_mean[e]);
   }
+  if (prob_mean != nullptr && threadIdx.x == 0) counts[2 * E] = T;
 }
 
 cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int32_t* counts,
                                   int32_t* chunk_counts, int32_t* local_rank, int32_t* err,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const float* prob_mean) {
   const int nchunks = ceil_div(c.T, kChunkTokens);
   if (nchunks > 0) {
     cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
@@ -272,7 +294,7 @@ cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int
     if (e != cudaSuccess) return e;
   }
   return launch_kernel(dispatch_total_kernel, 1, 256, 0, s, 0, chunk_counts, nchunks, c.E,
-                       counts);
+                       counts, prob_mean, c.T);
 }
 
 }  // namespace moe

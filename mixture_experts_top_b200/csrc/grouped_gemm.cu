@@ -36,7 +36,10 @@
 //    block (read from HBM once, reused from L2) across the expert's row blocks.
 //    Row tiles are re-read for every column block, so they are loaded with an
 //    evict-last L2 policy; weights keep the normal policy (an evict-first
-//    policy on them made CTAs that share a weight block re-read it from HBM).
+//    policy on all of them made CTAs that share a weight block re-read it
+//    from HBM).  The last reader of a block (a row block's last column block,
+//    a weight block's last row block) loads it evict-first, so that blocks
+//    no tile needs again leave L2 before live ones.
 //  * A tile that straddles two experts' rows reads the next expert's rows,
 //    computes them, and masks them at the store: no padding of the grouped
 //    layout is needed.
@@ -95,10 +98,16 @@ struct GemmArgs {
   const int32_t* offsets;
   const int32_t* perm;  // gathered A: grouped row r is row perm[r] of the A tensor (else null)
   int a_rows;           // rows of the A tensor (gathered A: tokens)
-  void* out;  // bf16 for kEpiRelu / kEpiSwiglu, fp32 for kEpiNone
+  void* out;  // bf16 for kEpiRelu / kEpiSwiglu / kEpiScatter, fp32 for kEpiNone
   int32_t* err;
   int E, K, N, rows_max;
   int n_tiles;  // output-column blocks
+  // kEpiScatter (top-1 combine in the epilogue): grouped row r is the only
+  // kept slot of token rows[r]; its output row is gates[token] * acc.
+  const int32_t* rows;
+  const float* gates;
+  const int32_t* dest;  // (T) slot of each token, -1 if dropped: that output row is zeroed
+  int T;
 };
 
 struct TileCoord {
@@ -134,7 +143,37 @@ template <int EPI>
 __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
                                                 const GemmArgs& g) {
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
-  if (EPI == kEpiSwiglu) {
+  if (EPI == kEpiScatter) {
+    // orow_off is the grouped row; its token's output row gets gate * acc,
+    // one rounding to bf16 (the combine's fp32 product, then its rounding).
+    int tok = 0;
+    float gate = 0.f;
+    if (valid) {
+      tok = g.rows[orow_off];
+      valid = tok >= 0 && tok < g.T;
+      if (valid) gate = g.gates[tok];
+    }
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + (size_t)tok * g.N;
+#pragma unroll 1
+    for (int cc = 0; cc < OUT_COLS; cc += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tacc + cc, r);
+      tmem_ld_wait();
+      if (valid) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(gate * __uint_as_float(r[2 * i]), gate * __uint_as_float(r[2 * i + 1]));
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int col = n0 + cc + v * 8;
+          if (col < g.N)
+            *reinterpret_cast<uint4*>(orow + col) =
+                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  } else if (EPI == kEpiSwiglu) {
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t gr[32], ur[32];
@@ -200,6 +239,19 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
         }
       }
     }
+  }
+}
+
+// kEpiScatter: the output rows of tokens whose only slot was dropped are
+// zero; the epilogue warps of every CTA write a strided share of them before
+// their first tile (no grouped row maps to such a token, so no tile writes it).
+__device__ __forceinline__ void zero_dropped_rows(const GemmArgs& g, int warp, int lane) {
+  const int w = (int)blockIdx.x * 4 + (warp - 2), nw = (int)gridDim.x * 4;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
+  for (int t = w; t < g.T; t += nw) {
+    if (g.dest[t] >= 0) continue;
+    uint4* row = reinterpret_cast<uint4*>(out + (size_t)t * g.N);
+    for (int v = lane; v < g.N / 8; v += 32) row[v] = make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -284,10 +336,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
-    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal();
+    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal(),
+                   done = l2_policy_evict_first();
     for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
       const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
+      // The row block's last column block and the weight block's last row
+      // block read their operand for the last time.
+      const uint64_t pol_a = c.n_tile == g.n_tiles - 1 ? done : keep;
+      const uint64_t pol_b = c.m0 + BM >= row_off[c.e + 1] ? done : stream;
       int r4[4] = {0, 0, 0, 0};
       if (GATHER) {
 #pragma unroll
@@ -312,17 +369,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             report_error(g.err, kDevTimeoutProducer);
           } else {
             mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-            if (!GATHER) tma_load_2d_hint(sa, &tmA, &full_bar[stage], k0, c.m0, keep);
+            if (!GATHER) tma_load_2d_hint(sa, &tmA, &full_bar[stage], k0, c.m0, pol_a);
             if (EPI == kEpiSwiglu) {
-              tma_load_3d_hint(sb, &tmB0, &full_bar[stage], n0, k0, c.e, stream);
-              tma_load_3d_hint(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e, stream);
-              tma_load_3d_hint(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e, stream);
-              tma_load_3d_hint(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e, stream);
+              tma_load_3d_hint(sb, &tmB0, &full_bar[stage], n0, k0, c.e, pol_b);
+              tma_load_3d_hint(sb + B_BOX, &tmB0, &full_bar[stage], n0 + 64, k0, c.e, pol_b);
+              tma_load_3d_hint(sb + 2 * B_BOX, &tmB1, &full_bar[stage], n0, k0, c.e, pol_b);
+              tma_load_3d_hint(sb + 3 * B_BOX, &tmB1, &full_bar[stage], n0 + 64, k0, c.e, pol_b);
             } else {
 #pragma unroll
               for (int i = 0; i < 4; ++i)
                 tma_load_3d_hint(sb + i * B_BOX, &tmB0, &full_bar[stage], n0 + 64 * i, k0, c.e,
-                                 stream);
+                                 pol_b);
             }
             issued_mask |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -332,7 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (ok)
             tma_gather4_hint(sa + lane * 4 * (BK * 2), &tmA, &full_bar[stage], k0, r4[0], r4[1],
-                             r4[2], r4[3], keep);
+                             r4[2], r4[3], pol_a);
         }
         if (!ok) {
           alive = false;
@@ -393,6 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp >= 2) {
     // ------------------------------------------------------ epilogue
+    if (EPI == kEpiScatter) zero_dropped_rows(g, warp, lane);
     const int q = warp & 3;               // TMEM lane quarter of this warp
     const int row = q * 32 + lane;        // row inside the tile
     int acc = 0;
@@ -407,7 +465,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
-      const size_t orow_off = (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
+                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[acc]);
@@ -531,10 +590,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
     const CUtensorMap* bmap = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
-    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal();
+    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal(),
+                   done = l2_policy_evict_first();
     for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
       const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
+      // The row block's last column block and the weight block's last row
+      // block read their operand for the last time.
+      const uint64_t pol_a = c.n_tile == g.n_tiles - 1 ? done : keep;
+      const uint64_t pol_b = c.m0 + PBM >= row_off[c.e + 1] ? done : stream;
       // this CTA's B half: gate / up for SwiGLU, else the column halves
       const int nb = (EPI == kEpiSwiglu) ? n0 : n0 + (int)rank * (BN / 2);
       const int my_m = c.m0 + (int)rank * BM;
@@ -562,9 +626,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             report_error(g.err, kDevTimeoutProducer);
           } else {
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-            if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, keep);
-            tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, stream);
-            tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, stream);
+            if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, pol_a);
+            tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, pol_b);
+            tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, pol_b);
             issued_mask |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           }
@@ -573,7 +637,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (ok)
             tma_gather4_pair(sa + lane * 4 * (BK * 2), &tmA, &full_bar[stage], k0, r4[0], r4[1],
-                             r4[2], r4[3], keep);
+                             r4[2], r4[3], pol_a);
         }
         if (!ok) {
           alive = false;
@@ -634,6 +698,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue (both)
+    if (EPI == kEpiScatter) zero_dropped_rows(g, warp, lane);
     const int q = warp & 3;
     const int row = (int)rank * BM + q * 32 + lane;  // row inside the pair tile
     int acc = 0;
@@ -648,7 +713,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
-      const size_t orow_off = (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
+                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
       tc_fence_before_sync();
       __syncwarp();
@@ -730,11 +796,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
-                                const int32_t* perm, int a_rows) {
+                                const int32_t* perm, int a_rows, const ScatterCombine* sc) {
   if (rows_max == 0) return cudaSuccess;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const bool gather = perm != nullptr;
-  if (gather && (epi == kEpiNone || a_rows <= 0)) return cudaErrorInvalidValue;
+  if (gather && (epi == kEpiNone || epi == kEpiScatter || a_rows <= 0)) return cudaErrorInvalidValue;
+  if ((epi == kEpiScatter) != (sc != nullptr)) return cudaErrorInvalidValue;
   CUtensorMap ta, tb0, tb1;
   const bool a_ok = gather ? encode_a(&ta, A, a_rows, K, 1) : encode_a(&ta, A, rows_max, K);
   if (!a_ok || !encode_b(&tb0, B0, E, K, N) ||
@@ -752,6 +819,10 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   g.N = N;
   g.rows_max = rows_max;
   g.n_tiles = ceil_div(N, out_cols);
+  g.rows = sc != nullptr ? sc->rows : nullptr;
+  g.gates = sc != nullptr ? sc->gates : nullptr;
+  g.dest = sc != nullptr ? sc->dest : nullptr;
+  g.T = sc != nullptr ? sc->T : 0;
   // Expert groups of 1024 rows or more on average: CTA pairs (M = 256 tiles,
   // a third less traffic per CTA); smaller groups: single CTAs (M = 128
   // tiles waste fewer rows at group edges).
@@ -764,6 +835,7 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
     switch (epi) {
       case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, g, pairs, s);
       case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, g, pairs, s);
       default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, g, pairs, s);
     }
   }
@@ -775,6 +847,7 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   switch (epi) {
     case kEpiSwiglu: return run_gemm<kEpiSwiglu, false>(ta, tb0, tb1, g, grid, s);
     case kEpiRelu: return run_gemm<kEpiRelu, false>(ta, tb0, tb1, g, grid, s);
+    case kEpiScatter: return run_gemm<kEpiScatter, false>(ta, tb0, tb1, g, grid, s);
     default: return run_gemm<kEpiNone, false>(ta, tb0, tb1, g, grid, s);
   }
 }

@@ -116,6 +116,39 @@ cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* per
                              offsets, y_perm, err, s);
 }
 
+// The experts and the combine: for top_k = 1 with bf16 experts the combine
+// is the down projection's epilogue (gate * row written straight into the
+// token's output row; tokens whose slot was dropped get a zero row), so no
+// y_perm is written and no combine kernel runs; otherwise the experts write
+// y_perm (in the workspace) and the combine kernel sums each token's rows.
+cudaError_t run_experts_combine(const moe_config_t& c, const void* x_perm,
+                                const int32_t* offsets, const int32_t* perm_token,
+                                const int32_t* dest, const float* gates, const void* W_in,
+                                const void* W_up, const void* W_out, void* output, void* ws,
+                                cudaStream_t s) {
+  const WsLayout L = workspace_layout(c);
+  if (c.top_k == 1 && c.expert_kind != MOE_EXPERT_LINEAR) {
+    int32_t* err = at<int32_t>(ws, L.ctrl);
+    const int rows_max = c.T;
+    __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
+    const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
+    cudaError_t e = launch_grouped_gemm(
+        epi, static_cast<const __nv_bfloat16*>(x_perm), rows_max, c.d,
+        static_cast<const __nv_bfloat16*>(W_in),
+        epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
+        offsets, hidden, err, s);
+    if (e != cudaSuccess) return e;
+    const ScatterCombine sc{perm_token, gates, dest, c.T};
+    return launch_grouped_gemm(kEpiScatter, hidden, rows_max, c.d_hidden,
+                               static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
+                               offsets, output, err, s, nullptr, 0, &sc);
+  }
+  void* y_perm = at<void>(ws, L.y_perm);
+  cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws, s);
+  if (e != cudaSuccess) return e;
+  return launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output, s);
+}
+
 }  // namespace
 
 namespace {
@@ -295,7 +328,7 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
   }
   MOE_ALIGNED16(x);
   MOE_ALIGNED16(x_perm);
-  MOE_REQUIRE(prob_mean);
+  if (sh == nullptr) MOE_REQUIRE(prob_mean);   // a sharded batch takes P from the records
   MOE_REQUIRE(counts);
   MOE_REQUIRE(offsets);
   MOE_REQUIRE(f);
@@ -306,8 +339,8 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
       return fail(MOE_ERR_INVALID_ARG, "shard: need 0 <= rank < world");
     if (sh->T_global < c.T || (int64_t)sh->T_global * c.top_k >= ((int64_t)1 << 31))
       return fail(MOE_ERR_INVALID_ARG, "shard: need T <= T_global and T_global * top_k < 2^31");
-    if (sh->all_counts == nullptr) return fail(MOE_ERR_INVALID_ARG, "shard->all_counts is NULL");
-    shard = ShardInfo{sh->rank, sh->world, sh->T_global, sh->all_counts};
+    if (sh->records == nullptr) return fail(MOE_ERR_INVALID_ARG, "shard->records is NULL");
+    shard = ShardInfo{sh->rank, sh->world, sh->T_global, sh->records};
   }
   if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = workspace_layout(c);
@@ -381,6 +414,76 @@ int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_ro
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_backward");
 }
 
+size_t moe_expert_backward_workspace_size(const moe_config_t* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return expert_backward_layout(*cfg).total;
+}
+
+int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                            const void* W_in, const void* W_up, const void* W_out,
+                            const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
+                            float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  const bool swiglu = c.expert_kind == MOE_EXPERT_SWIGLU;
+  const bool linear = c.expert_kind == MOE_EXPERT_LINEAR;
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(W_in);
+  MOE_REQUIRE(dW_in);
+  if (swiglu) {
+    MOE_REQUIRE(W_up);
+    MOE_REQUIRE(dW_up);
+  }
+  if (!linear) {
+    MOE_REQUIRE(W_out);
+    MOE_REQUIRE(dW_out);
+  }
+  if (c.T > 0) {
+    MOE_REQUIRE(x_perm);
+    MOE_REQUIRE(dy_perm);
+    MOE_REQUIRE(dx_perm);
+  }
+  MOE_ALIGNED16(x_perm);
+  MOE_ALIGNED16(dy_perm);
+  MOE_ALIGNED16(dx_perm);
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
+  MOE_ALIGNED16(dW_in);
+  MOE_ALIGNED16(dW_up);
+  MOE_ALIGNED16(dW_out);
+  if (ws == nullptr) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const size_t need = expert_backward_layout(c).total;
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) +
+                                       " bytes (moe_expert_backward_workspace_size)");
+  const cudaError_t e = launch_expert_backward(c, x_perm, offsets, W_in, W_up, W_out, dy_perm,
+                                               dx_perm, dW_in, dW_up, dW_out, ws,
+                                               reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_backward");
+}
+
+int moe_permute_backward(const moe_config_t* cfg, const float* dx_perm, const int32_t* dest,
+                         const float* dx_add, float* dx, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) {
+    MOE_REQUIRE(dx_perm);
+    MOE_REQUIRE(dest);
+    MOE_REQUIRE(dx);
+  }
+  MOE_ALIGNED16(dx_perm);
+  MOE_ALIGNED16(dx_add);
+  MOE_ALIGNED16(dx);
+  const cudaError_t e = launch_permute_backward(c, dx_perm, dest, dx_add, dx,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_permute_backward");
+}
+
 int moe_check_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, moe_stream_t stream) {
   if (ws == nullptr || ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace missing or too small");
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
@@ -440,6 +543,25 @@ int moe_dispatch_count(const moe_config_t* cfg, const int32_t* expert_indices, i
                                               at<int32_t>(ws, L.ctrl),
                                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch_count");
+}
+
+int moe_shard_record(const moe_config_t* cfg, const int32_t* expert_indices,
+                     const float* prob_mean, int32_t* record, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T > 0) MOE_REQUIRE(expert_indices);
+  MOE_REQUIRE(prob_mean);
+  MOE_REQUIRE(record);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  const cudaError_t e = launch_dispatch_count(c, expert_indices, record,
+                                              at<int32_t>(ws, L.chunk_counts),
+                                              at<int32_t>(ws, L.local_rank),
+                                              at<int32_t>(ws, L.ctrl),
+                                              reinterpret_cast<cudaStream_t>(stream), prob_mean);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_shard_record");
 }
 
 int moe_dispatch_shard(const moe_config_t* cfg, const moe_shard_t* shard, const void* x,
@@ -505,6 +627,37 @@ int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_gather");
 }
 
+int moe_expert_ffn_combine(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                           const int32_t* perm_token, const int32_t* dest, const float* gates,
+                           const void* W_in, const void* W_up, const void* W_out, void* output,
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(W_in);
+  if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
+  if (c.expert_kind != MOE_EXPERT_LINEAR) MOE_REQUIRE(W_out);
+  if (c.T > 0) {
+    MOE_REQUIRE(x_perm);
+    MOE_REQUIRE(perm_token);
+    MOE_REQUIRE(dest);
+    MOE_REQUIRE(gates);
+    MOE_REQUIRE(output);
+  }
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
+  MOE_ALIGNED16(x_perm);
+  MOE_ALIGNED16(output);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  if (c.T == 0) return MOE_OK;
+  const cudaError_t e = run_experts_combine(c, x_perm, offsets, perm_token, dest, gates, W_in,
+                                            W_up, W_out, output, ws,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_combine");
+}
+
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
                 const float* gates, void* output, moe_stream_t stream) {
   int st = check_config(cfg);
@@ -557,7 +710,6 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   int32_t* dest = at<int32_t>(ws, L.dest);
   int32_t* perm = at<int32_t>(ws, L.perm_token);
   void* x_perm = at<void>(ws, L.x_perm);
-  void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, P,
                                nullptr, at<float>(ws, L.router_part),
                                at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl), s);
@@ -570,10 +722,8 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   // The materialised permute (one copy of each kept row, ~38 us at the
   // Mixtral shape) is far cheaper than gathering A rows inside the GEMM,
   // which re-fetches them for every output column block.
-  e = run_experts(c, x_perm, nullptr, offs, W_in, W_up, W_out, y_perm, ws, s);
-  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts");
-  e = launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output, s);
-  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/combine");
+  e = run_experts_combine(c, x_perm, offs, perm, dest, gates, W_in, W_up, W_out, output, ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts+combine");
   return MOE_OK;
 }
 
@@ -607,22 +757,65 @@ namespace {
 constexpr size_t kNoAllocScratchFloats = 65536;
 static __device__ __align__(256) float g_route_scratch[kNoAllocScratchFloats];
 
-// Device address of g_route_scratch on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is asked of
-// the runtime once per device (with that device current) and cached.
+// The driver's cuCtxGetCurrent and cuCtxGetId, looked up once (nullptr if
+// missing).  A context's id is unique for the life of the process, so it
+// tells a context made by cudaDeviceReset from the one it replaced even if
+// the new handle has the old one's value.
+struct CtxIdFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxIdFns& ctx_id_fns() {
+  static const CtxIdFns fns = [] {
+    CtxIdFns f;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    return f;
+  }();
+  return fns;
+}
+
+// Id of the current context, or 0 if it cannot be read.
+unsigned long long current_ctx_id() {
+  const CtxIdFns& f = ctx_id_fns();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (f.get_current == nullptr || f.get_id == nullptr) return 0;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_route_scratch in the current device's context.  In
+// host code the array's name is only a host-side stand-in, so the address
+// is asked of the runtime (with that device current) the first time a
+// context is seen and cached per device with that context's id.  A new
+// context on the device (after cudaDeviceReset, which loads the module
+// again, so the array may move) has a new id and is looked up afresh; where
+// the id cannot be read, the address is looked up on every call.
 cudaError_t route_scratch_address(float** out) {
   static std::mutex mu;
   static float* cached[64] = {};
+  static unsigned long long cached_ctx[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  const unsigned long long ctx = current_ctx_id();
+  if (cached[dev] == nullptr || ctx == 0 || cached_ctx[dev] != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    e = cudaGetSymbolAddress(&p, g_route_scratch);   // makes the device's context current
     if (e != cudaSuccess) return e;
     cached[dev] = static_cast<float*>(p);
+    cached_ctx[dev] = current_ctx_id();
   }
   *out = cached[dev];
   return cudaSuccess;

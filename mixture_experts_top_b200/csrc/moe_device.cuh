@@ -93,7 +93,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 
 // --------------------------------------------------------------------- TMA --
 // Tiled tensor loads, completion signalled on an mbarrier (transaction bytes).
-// No multicast form is used anywhere in this library.
+// No load in this library uses multicast; the only multicast form is the
+// pair GEMM's tcgen05.commit, which arrives on both CTAs' mbarriers.
 
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -118,7 +119,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 }
 
 // L2 cache policies for TMA loads: rows reused by many tiles stay (evict
-// last); everything else keeps the normal policy.
+// last), weights keep the normal policy, and a block's last reader marks it
+// evict-first so that dead data does not crowd out live data.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -127,6 +129,12 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// For a block's last reader: the lines may leave L2 first once read.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 

@@ -117,11 +117,12 @@ cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const
                             int32_t* err, cudaStream_t s, int* tiles_out);
 
 // A batch split over `world` ranks in contiguous token blocks, rank order:
-// every rank's per-expert slot counts (world, E) on the device, and the
-// whole batch's token count.
+// every rank's exchange record (world, 2E+1) int32 on the device (E slot
+// counts, E probability means as fp32 bits, the token count), and the whole
+// batch's token count.
 struct ShardInfo {
   int rank, world, T_global;
-  const int32_t* all_counts;
+  const int32_t* records;
 };
 cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t* idx,
                             const float* prob_mean, int32_t* counts, int32_t* offsets,
@@ -129,10 +130,12 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
                             int32_t* local_rank, int32_t* err, cudaStream_t s,
                             const ShardInfo* shard = nullptr, int32_t* shard_prefix = nullptr);
-// The per-expert slot counts of `idx` (T, top_k) into counts (E).
+// The per-expert slot counts of `idx` (T, top_k) into counts (E); with
+// prob_mean != nullptr, counts is a (2E+1) exchange record: the counts,
+// the fp32 bits of prob_mean and T.
 cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int32_t* counts,
                                   int32_t* chunk_counts, int32_t* local_rank, int32_t* err,
-                                  cudaStream_t s);
+                                  cudaStream_t s, const float* prob_mean = nullptr);
 
 cudaError_t launch_combine(const moe_config_t& c, const float* y_perm, const int32_t* dest,
                            const float* gates, void* out, cudaStream_t s);
@@ -146,8 +149,16 @@ cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
 // offsets[e+1]) of A (rows_max, K) times B_e (K, N) -> out rows, with a fused
 // epilogue.  epi: 0 = none (fp32 output), 1 = ReLU (bf16 output), 2 = SwiGLU
 // (bf16 output; B0 = gate, B1 = up; each output column pairs one gate and
-// one up column).
-enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2 };
+// one up column), 3 = the top-1 combine (bf16 output rows of tokens: grouped
+// row r writes gates[t] * acc into row t = rows[r]; tokens with dest[t] < 0
+// get a zero row).
+enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2, kEpiScatter = 3 };
+struct ScatterCombine {
+  const int32_t* rows;   // (rows) token of each grouped row (perm_token)
+  const float* gates;    // (T) the single slot's gate
+  const int32_t* dest;   // (T) the single slot's grouped row, -1 if dropped
+  int T;
+};
 
 // perm != nullptr (ReLU / SwiGLU only): grouped row r of A is row perm[r] of
 // A, an (a_rows, K) tensor, fetched by TMA row gathers (the permute fused into
@@ -155,7 +166,37 @@ enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2 };
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
-                                const int32_t* perm = nullptr, int a_rows = 0);
+                                const int32_t* perm = nullptr, int a_rows = 0,
+                                const ScatterCombine* sc = nullptr);
+
+// Experts' backward (expert_backward.cu, grouped_gemm_bwd.cu).  The bf16
+// GEMMs work on a padded grouped layout: each expert's rows rounded up to a
+// multiple of kBwdPadRows, zero rows after its own.
+constexpr int kBwdPadRows = 128;
+// Rows of the padded layout for at most rows_max grouped rows.
+int expert_backward_pad_rows(int rows_max, int E);
+// Workspace of moe_expert_ffn_backward: error word; padded rows Xp (bf16),
+// dYp (bf16); pre-activations [A | B], their gradients [dA | dB] and H.
+struct ExpertBwdLayout {
+  size_t ctrl, xp, dyp, pre, dab, hid, total;
+};
+ExpertBwdLayout expert_backward_layout(const moe_config_t& c);
+cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
+                                   const int32_t* offsets, const void* W_in, const void* W_up,
+                                   const void* W_out, const float* dy_perm, float* dx_perm,
+                                   float* dW_in, float* dW_up, float* dW_out, void* ws,
+                                   cudaStream_t s);
+cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* offsets,
+                                         const __nv_bfloat16* xp, const __nv_bfloat16* dyp,
+                                         const __nv_bfloat16* W_in, const __nv_bfloat16* W_up,
+                                         const __nv_bfloat16* W_out, __nv_bfloat16* pre,
+                                         __nv_bfloat16* dab, __nv_bfloat16* hid, float* dx_perm,
+                                         float* dW_in, float* dW_up, float* dW_out, int32_t* err,
+                                         cudaStream_t s);
+// dx (T, d) = dx_add (or 0) + sum over kept slots j of dx_perm[dest[t, j]].
+cudaError_t launch_permute_backward(const moe_config_t& c, const float* dx_perm,
+                                    const int32_t* dest, const float* dx_add, float* dx,
+                                    cudaStream_t s);
 
 // Routing backward (backward.cu).
 int route_backward_chunks(int T);

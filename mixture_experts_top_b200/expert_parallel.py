@@ -128,7 +128,8 @@ def exchange_rows(sends, x_perm, y_perm, rank: int, world: int, ranges, compute,
     """The two all-to-alls over `group`.  sends = this rank's exchange_plan;
     compute(x_recv, slice_counts, y_recv) runs this rank's experts on the
     received rows (source order) and fills y_recv; the returned rows land in
-    y_perm[:R] in the order they were sent."""
+    y_perm[:R] in the order they were sent.  Returns (slice_counts, what
+    compute returned)."""
     import torch.distributed as dist
     dev = x_perm.device
     lo, hi = ranges[rank]
@@ -149,9 +150,9 @@ def exchange_rows(sends, x_perm, y_perm, rank: int, world: int, ranges, compute,
     dist.all_to_all_single(x_recv, x_perm[:R].contiguous(), recv_splits, send_splits, group=group)
     y_recv = torch.empty((sum(recv_splits),) + tuple(y_perm.shape[1:]), dtype=y_perm.dtype,
                          device=dev)
-    compute(x_recv, slice_counts, y_recv)
+    result = compute(x_recv, slice_counts, y_recv)
     dist.all_to_all_single(y_perm[:R], y_recv, send_splits, recv_splits, group=group)
-    return slice_counts
+    return slice_counts, result
 
 
 def ep_forward(cfg, rank: int, world: int, x, W_router, logit_bias, noise, W_in_local,
@@ -159,12 +160,29 @@ def ep_forward(cfg, rank: int, world: int, x, W_router, logit_bias, noise, W_in_
     """This rank's layer with the experts split over `world` ranks of a
     torch.distributed group: dispatch, all-to-all of the rows (and of the
     per-expert counts), the local experts, all-to-all back, combine.  aux and
-    the capacity are this rank's batch's, as in moe_forward."""
+    the capacity are this rank's batch's, as in moe_forward.
+
+    The device error words of both workspaces (this rank's routing and
+    dispatch, and its local experts) are read after the second all-to-all;
+    a nonzero code (a bounded wait that ran out, offsets that are not a
+    partition) raises api.MoeError instead of combining rows that may not
+    have been written."""
     st = ep_dispatch(cfg, x, W_router, logit_bias, noise, ws, world)
     ranges = plan(cfg.E, world)
     lo, hi = ranges[rank]
-    exchange_rows(st.sends, st.x_perm, st.y_perm, rank, world, ranges,
-                  lambda xr, sc, yr: ep_experts(cfg, hi - lo, xr, sc, W_in_local, W_up_local,
-                                                W_out_local, yr), group)
+    _, lws = exchange_rows(st.sends, st.x_perm, st.y_perm, rank, world, ranges,
+                           lambda xr, sc, yr: ep_experts(cfg, hi - lo, xr, sc, W_in_local,
+                                                         W_up_local, W_out_local, yr), group)
+    check_device_status({"experts": lws, "dispatch": ws})
     output = torch.empty((cfg.T, cfg.d_out), dtype=x.dtype, device=x.device)
     return ep_combine(cfg, st, output)
+
+
+def check_device_status(workspaces: dict) -> None:
+    """Raise api.MoeError if any workspace's device error word is set (each
+    read synchronises its stream and clears the word)."""
+    for name, w in workspaces.items():
+        code = api.moe_device_status(w)
+        if code != 0:
+            raise api.MoeError(api.MOE_ERR_DEVICE_CHECK, f"ep_forward ({name})",
+                               f"device error code {code}")

@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 18
+    assert len(names) == 23
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -137,9 +137,9 @@ def test_shard_and_gather_argument_checks(moe_lib):
     st = moe_lib.moe_dispatch_shard(ctypes.byref(cfg), None, FAKE, FAKE, FAKE, *outs, FAKE,
                                     FAKE, ws, None)
     assert st == api.MOE_ERR_INVALID_ARG and "shard" in moe_lib.moe_last_error_message().decode()
-    for rank, world, T_g, counts in [(2, 2, 128, FAKE), (-1, 2, 128, FAKE), (0, 0, 128, FAKE),
-                                     (0, 2, 32, FAKE), (0, 2, 128, None)]:
-        sh = api.MoeShard(rank, world, T_g, counts)
+    for rank, world, T_g, records in [(2, 2, 128, FAKE), (-1, 2, 128, FAKE), (0, 0, 128, FAKE),
+                                      (0, 2, 32, FAKE), (0, 2, 128, None)]:
+        sh = api.MoeShard(rank, world, T_g, records)
         st = moe_lib.moe_dispatch_shard(ctypes.byref(cfg), ctypes.byref(sh), FAKE, FAKE, FAKE,
                                         *outs, FAKE, FAKE, ws, None)
         assert st == api.MOE_ERR_INVALID_ARG, (rank, world, T_g)
@@ -147,6 +147,10 @@ def test_shard_and_gather_argument_checks(moe_lib):
         api.MOE_ERR_INVALID_ARG
     assert moe_lib.moe_dispatch_count(ctypes.byref(cfg), FAKE, FAKE, FAKE, ws - 1, None) == \
         api.MOE_ERR_WORKSPACE
+    assert moe_lib.moe_shard_record(ctypes.byref(cfg), FAKE, None, FAKE, FAKE, ws, None) == \
+        api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_shard_record(ctypes.byref(cfg), FAKE, FAKE, None, FAKE, ws, None) == \
+        api.MOE_ERR_INVALID_ARG
     # gather: perm_token required, x aligned
     st = moe_lib.moe_expert_ffn_gather(ctypes.byref(cfg), FAKE, None, FAKE, FAKE, FAKE, FAKE,
                                        FAKE, FAKE, ws, None)
@@ -189,6 +193,40 @@ def test_backward_argument_checks(moe_lib):
     # workspace too small
     assert moe_lib.moe_route_backward(ctypes.byref(cfg), *args, 0, FAKE, FAKE, None, None, FAKE,
                                       ws - 256, None) == api.MOE_ERR_WORKSPACE
+
+
+def test_expert_backward_argument_checks(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    n = moe_lib.moe_expert_backward_workspace_size(ctypes.byref(cfg))
+    # padded rows (T*k + E*127) of Xp, dYp, [A|B], [dA|dB] and H, bf16
+    rows = 64 * 2 + 8 * 127
+    assert n >= rows * (64 + 64 + 2 * 128 + 2 * 128 + 128) * 2 and n % 256 == 0
+    lin = api.make_config(64, 32, 0, 32, 8, 2, "linear", "f32")
+    assert 0 < moe_lib.moe_expert_backward_workspace_size(ctypes.byref(lin)) < n
+    ins = [FAKE] * 6                          # x_perm, offsets, W_in, W_up, W_out, dy_perm
+    outs = [FAKE] * 4                         # dx_perm, dW_in, dW_up, dW_out
+    # SwiGLU needs dW_up
+    st = moe_lib.moe_expert_ffn_backward(ctypes.byref(cfg), *ins, FAKE, FAKE, None, FAKE, FAKE,
+                                         n, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "dW_up" in moe_lib.moe_last_error_message().decode()
+    # misaligned gradient output
+    st = moe_lib.moe_expert_ffn_backward(ctypes.byref(cfg), *ins, FAKE + 4, FAKE, FAKE, FAKE,
+                                         FAKE, n, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "dx_perm" in moe_lib.moe_last_error_message().decode()
+    # workspace too small, misaligned
+    assert moe_lib.moe_expert_ffn_backward(ctypes.byref(cfg), *ins, *outs, FAKE, n - 256,
+                                           None) == api.MOE_ERR_WORKSPACE
+    assert moe_lib.moe_expert_ffn_backward(ctypes.byref(cfg), *ins, *outs, FAKE + 16, n,
+                                           None) == api.MOE_ERR_WORKSPACE
+    # linear experts: W_out, W_up and their gradients may be NULL; dW_in may not
+    st = moe_lib.moe_expert_ffn_backward(ctypes.byref(lin), FAKE, FAKE, FAKE, None, None, FAKE,
+                                         FAKE, None, None, None, FAKE, n, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "dW_in" in moe_lib.moe_last_error_message().decode()
+    # rows back to tokens
+    assert moe_lib.moe_permute_backward(ctypes.byref(cfg), None, FAKE, None, FAKE, None) == \
+        api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_permute_backward(ctypes.byref(cfg), FAKE, FAKE, FAKE + 8, FAKE, None) == \
+        api.MOE_ERR_INVALID_ARG
 
 
 def test_swiglu_needs_three_matrices(moe_lib):

@@ -55,9 +55,11 @@ def _worker(rank, world, port, E, out):
                 [int((x_recv[:, 0] == s).sum()) for s in range(world)]
             y_recv[:, :3] = x_recv
             y_recv[:, 3] = rank
+            return ("computed on", rank)
 
         sends = ep.exchange_plan(offsets, ranges)
-        ep.exchange_rows(sends, x_perm, y_perm, rank, world, ranges, compute)
+        _, result = ep.exchange_rows(sends, x_perm, y_perm, rank, world, ranges, compute)
+        seen["result"] = result == ("computed on", rank)
         back_ok = torch.equal(y_perm[:R, :3], x_perm[:R])
         holder = np.searchsorted([b for _, b in ranges], expert_of_row, side="right")
         holder_ok = np.array_equal(y_perm[:R, 3].numpy().astype(int), holder)
@@ -76,5 +78,6 @@ def test_exchange_rows_over_gloo(world, E):
         res = dict(out)
     for r in range(world):
         seen, back_ok, holder_ok, untouched = res[r]
-        assert seen == {"experts_ok": True, "sources_in_order": True, "counts": True}, (r, seen)
+        assert seen == {"experts_ok": True, "sources_in_order": True, "counts": True,
+                        "result": True}, (r, seen)
         assert back_ok and holder_ok and untouched, r

@@ -68,3 +68,50 @@ def test_combine_top1_gate_one_copies_row():
     cfg = api.make_config(T, 64, 64, d_out, 4, 1, "relu", "bf16")
     got = run_combine(cfg, y_perm, dest, np.ones((T, 1), np.float32))
     assert np.array_equal(got, f32_to_bf16_bits(y_perm[dest[:, 0]]))
+
+
+@pytest.mark.parametrize("name,k,cf", [("switch_relu", 1, 1.25), ("mixtral", 1, 0.5),
+                                       ("mixtral", 1, 0.0), ("switch_relu", 2, 1.0)])
+def test_expert_ffn_combine_equals_ffn_then_combine(name, k, cf):
+    """moe_expert_ffn_combine: at top_k = 1 the combine runs in the down
+    projection's epilogue (no y_perm, dropped tokens zeroed there); it must
+    give the bits of moe_expert_ffn followed by moe_combine, drops included.
+    At top_k = 2 it is those two calls."""
+    from gpu_util import cfg_of
+    from workloads import WORKLOADS, make_inputs
+    base = {"switch_relu": WORKLOADS["switch_relu"].replace(T=1500, d=256, d_hidden=512,
+                                                            d_out=256),
+            "mixtral": WORKLOADS["mixtral"].replace(T=900, d=256, d_hidden=384, d_out=264)}[name]
+    w = base.replace(top_k=k, capacity_factor=cf)
+    inp = make_inputs(w, seed=17)
+    cfg = cfg_of(w)
+    ws = api.alloc_workspace(cfg)
+    T, E = w.T, w.E
+    i32 = dict(dtype=torch.int32, device="cuda")
+    x = dev(inp["x"])
+    idx = torch.empty((T, k), **i32)
+    gates = torch.empty((T, k), device="cuda")
+    P = torch.empty(E, device="cuda")
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    dest, perm = torch.empty((T, k), **i32), torch.empty(T * k, **i32)
+    drop = torch.empty((T, k), dtype=torch.uint8, device="cuda")
+    f, aux = torch.empty(E, device="cuda"), torch.empty(1, device="cuda")
+    x_perm = torch.empty((T * k, w.d), dtype=torch.bfloat16, device="cuda")
+    api.moe_route(cfg, x, dev(inp["W_router"]), dev(inp["logit_bias"]), dev(inp["noise"]), idx,
+                  gates, P, None, ws)
+    api.moe_dispatch(cfg, x, idx, P, counts, offsets, dest, perm, drop, f, aux, x_perm, ws)
+    W = [dev(inp[key]) for key in ("W_in", "W_up", "W_out")]
+    y_perm = torch.empty((T * k, w.d_out), device="cuda")
+    api.moe_expert_ffn(cfg, x_perm, offsets, *W, y_perm, ws)
+    ref = torch.full((T, w.d_out), 3.0, dtype=torch.bfloat16, device="cuda")
+    api.moe_combine(cfg, y_perm, dest, gates, ref)
+    got = torch.full((T, w.d_out), 3.0, dtype=torch.bfloat16, device="cuda")
+    api.moe_expert_ffn_combine(cfg, x_perm, offsets, perm, dest, gates, *W, got, ws)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(ws) == 0
+    dropped = host(drop).all(axis=1)
+    if cf > 0 and k == 1:
+        assert dropped.any()
+    g, r = host(got), host(ref)
+    assert np.array_equal(g, r)
+    assert (bf16_to_f64(g[dropped]) == 0).all()

@@ -93,6 +93,28 @@ def test_forward_reduced_all_tokens(name):
             assert (bf16_to_f64(g["output"][dead]) == 0).all()
 
 
+def full_size_sample(w, tok, o, n_total=256):
+    """At least n_total comparable tokens (all of them if fewer): for every
+    expert a share of the tokens it kept, then tokens that had a slot
+    dropped, then random ones."""
+    rng = np.random.default_rng(1)
+    per = -(-n_total // w.E)
+    picks = []
+    kept = (o["drop_mask"] == 0)
+    for e in range(w.E):
+        on_e = np.flatnonzero(tok & ((o["expert_indices"] == e) & kept).any(axis=1))
+        if len(on_e):
+            picks.append(rng.choice(on_e, size=min(per, len(on_e)), replace=False))
+    dropped = np.flatnonzero(tok & (o["drop_mask"] == 1).any(axis=1))
+    picks.append(dropped[:16])
+    sample = np.unique(np.concatenate(picks)) if picks else np.zeros(0, np.int64)
+    rest = np.setdiff1d(np.flatnonzero(tok), sample)
+    need = max(0, n_total - len(sample))
+    if need and len(rest):
+        sample = np.union1d(sample, rng.choice(rest, size=min(need, len(rest)), replace=False))
+    return sample
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["decode", "switch_relu", "fine_grained", "mixtral"])
 def test_forward_full_size_sampled(name):
@@ -101,12 +123,8 @@ def test_forward_full_size_sampled(name):
     g = gpu_forward(w, inp)
     o = oracle_routing(w, inp)
     tok = check_routing(w, g, o)
-    rng = np.random.default_rng(1)
-    candidates = np.flatnonzero(tok)
-    # include tokens that had a slot dropped, if any
-    dropped = np.flatnonzero(tok & (o["drop_mask"] == 1).any(axis=1))
-    sample = np.unique(np.concatenate([rng.choice(candidates, size=min(24, len(candidates)),
-                                                  replace=False), dropped[:8]]))
+    sample = full_size_sample(w, tok, o)
+    assert len(sample) >= min(256, int(tok.sum()))
     weights = {k: inp[k] for k in ("W_in", "W_up", "W_out")}
     ref, rows = O.sampled_outputs(sample, inp["x"], w.dtype, w.kind, weights,
                                   o["expert_indices"], o["gates"], o["dest"], return_rows=True)
@@ -150,6 +168,43 @@ def test_forward_collapse_aux_near_E():
     g = gpu_forward(w, inp)
     assert (g["expert_indices"][:, 0] == 9).all()
     assert w.E - 1e-3 < float(g["aux_loss"][0]) <= w.E * (1 + 1e-6)
+
+
+def test_tiny_linear_zero_router_aux_is_exactly_one():
+    """The pages' small linear case with W_router = 0: every logit ties, so
+    indices are [0, 1] (lower index wins), gates are 1/2, and aux = 1.0
+    exactly (MLG Examples); the output is the oracle's within 1e-4."""
+    w = WORKLOADS["tiny_linear"]
+    inp = make_inputs(w, seed=0)
+    inp["W_router"] = np.zeros_like(inp["W_router"])
+    g = gpu_forward(w, inp)
+    assert float(g["aux_loss"][0]) == 1.0
+    assert (g["expert_indices"] == np.array([0, 1])).all()
+    assert (g["gates"] == 0.5).all()
+    o = O.moe_forward(inp["x"], inp["W_router"], {"W_in": inp["W_in"]}, top_k=2, kind="linear",
+                      dtype="f32", d_out=w.d_out)
+    assert o["aux_loss"] == 1.0
+    check_rows(w, g["output"], o["output"], o["Y"])
+
+
+def test_tiny_linear_top1_output_is_the_expert_matmul():
+    """The pages' small linear case with top_k = 1: every gate is exactly 1
+    and each token's output is x_t @ W_e of its expert, checked against a
+    plain einsum of the fp32 inputs in fp64 and against the oracle."""
+    w = WORKLOADS["tiny_linear"].replace(top_k=1)
+    inp = make_inputs(w, seed=0)
+    g = gpu_forward(w, inp)
+    assert (g["gates"] == 1.0).all()
+    o = O.moe_forward(inp["x"], inp["W_router"], {"W_in": inp["W_in"]}, top_k=1, kind="linear",
+                      dtype="f32", d_out=w.d_out)
+    amb = ambiguous_tokens(o["logits"], 1)
+    assert not amb.any()
+    assert np.array_equal(g["expert_indices"], o["expert_indices"])
+    e = g["expert_indices"][:, 0]
+    ref = np.einsum("td,tdo->to", inp["x"].astype(np.float64),
+                    inp["W_in"].astype(np.float64)[e])
+    assert np.abs(g["output"] - ref).max() <= REL_F32 * np.abs(ref).max()
+    check_rows(w, g["output"], o["output"], o["Y"])
 
 
 def test_forward_empty_batch():

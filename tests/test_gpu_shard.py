@@ -1,8 +1,8 @@
 """One batch split over ranks, each rank's calls run one after another on one
-GPU (no kernel waits on another rank's): moe_route and moe_dispatch_count per
-block of tokens, the exchange's arithmetic on the host (shard.combine_stats,
-which shard.exchange runs over a process group), then moe_dispatch_shard,
-moe_expert_ffn and moe_combine per block.
+GPU (no kernel waits on another rank's): shard.ShardStep per block of tokens
+-- moe_route and moe_shard_record, the all-gather of the records (here the
+records stacked in rank order, a stand-in for the collective used only in
+this test), then moe_dispatch_shard and moe_expert_ffn_combine.
 
 The result must be the single-batch layer's (moe_forward on all tokens): the
 same keep decisions with the capacity binding, the same f, the same aux on
@@ -38,46 +38,26 @@ def _run_shards(w, inp, blocks):
     W = [dev(inp[key]) for key in ("W_in", "W_up", "W_out")]
     Wr, bias = dev(inp["W_router"]), dev(inp["logit_bias"])
     starts = np.concatenate([[0], np.cumsum(blocks)])
-    ranks = []
+    steps, xs = [], []
     for r, n in enumerate(blocks):
-        cfg = cfg_of(w, T=n)
-        ws = api.alloc_workspace(cfg)
+        st = shard.ShardStep(cfg_of(w, T=n), r, len(blocks), w.T)
         x = dev(inp["x"][starts[r]:starts[r + 1]])
-        idx = torch.empty((n, w.top_k), dtype=torch.int32, device="cuda")
-        gates = torch.empty((n, w.top_k), dtype=torch.float32, device="cuda")
-        P = torch.empty(w.E, dtype=torch.float32, device="cuda")
-        api.moe_route(cfg, x, Wr, bias, None, idx, gates, P, None, ws)
-        counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
-        api.moe_dispatch_count(cfg, idx, counts, ws)
-        ranks.append(dict(cfg=cfg, ws=ws, x=x, idx=idx, gates=gates, P=P, counts=counts))
-    torch.cuda.synchronize()
-    all_counts, P, T_g = shard.combine_stats([d["counts"].cpu() for d in ranks],
-                                             [d["P"].cpu() for d in ranks], blocks)
-    assert T_g == w.T
-    all_counts, P = all_counts.cuda().contiguous(), P.cuda()
+        st.route(x, Wr, bias, None)
+        steps.append(st)
+        xs.append(x)
+    records = torch.stack([st.record for st in steps])
+    c, p, t = shard.unpack_records(host(records))
+    assert t.tolist() == list(blocks)
     outs = []
-    for r, d in enumerate(ranks):
-        cfg, n, k = d["cfg"], blocks[r], w.top_k
-        t = dict(counts=torch.empty(w.E, dtype=torch.int32, device="cuda"),
-                 offsets=torch.empty(w.E + 1, dtype=torch.int32, device="cuda"),
-                 dest=torch.empty((n, k), dtype=torch.int32, device="cuda"),
-                 perm=torch.empty(n * k, dtype=torch.int32, device="cuda"),
-                 drop=torch.empty((n, k), dtype=torch.uint8, device="cuda"),
-                 f=torch.empty(w.E, dtype=torch.float32, device="cuda"),
-                 aux=torch.empty(1, dtype=torch.float32, device="cuda"))
-        x_perm = torch.empty((n * k, w.d), dtype=d["x"].dtype, device="cuda")
-        api.moe_dispatch_shard(cfg, r, len(blocks), T_g, all_counts, d["x"], d["idx"], P,
-                               t["counts"], t["offsets"], t["dest"], t["perm"], t["drop"], t["f"],
-                               t["aux"], x_perm, d["ws"])
-        y_perm = torch.empty((n * k, w.d_out), dtype=torch.float32, device="cuda")
-        api.moe_expert_ffn(cfg, x_perm, t["offsets"], *W, y_perm, d["ws"])
-        out = torch.empty((n, w.d_out), dtype=d["x"].dtype, device="cuda")
-        api.moe_combine(cfg, y_perm, t["dest"], d["gates"], out)
+    for st, x in zip(steps, xs):
+        st.exchange(gather=lambda rec, out: out.copy_(records))
+        st.finish(x, *W)
         torch.cuda.synchronize()
-        assert api.moe_device_status(d["ws"]) == 0
-        res = {key: host(v) for key, v in t.items()}
-        res.update(output=host(out), idx=host(d["idx"]))
-        outs.append(res)
+        assert st.device_status() == 0
+        o = st.out
+        outs.append(dict(counts=host(o.counts), offsets=host(st.offsets), dest=host(st.dest),
+                         perm=host(st.perm), drop=host(o.drop_mask), f=host(st.f),
+                         aux=host(o.aux_loss), output=host(o.output), idx=host(o.expert_indices)))
     return outs
 
 
@@ -122,6 +102,21 @@ def test_sharded_batch_equals_single_batch(name, blocks):
     assert rel_close(outs[0]["f"], o["f"], 1e-6)
 
 
+def test_shard_record_layout():
+    """moe_shard_record: counts per expert, then moe_route's P as fp32 bits,
+    then T."""
+    w = REDUCED["fine_grained"]
+    inp = _inputs(w, seed=5)
+    cfg = cfg_of(w)
+    st = shard.ShardStep(cfg, 0, 1, w.T)
+    st.route(dev(inp["x"]), dev(inp["W_router"]), dev(inp["logit_bias"]), None)
+    torch.cuda.synchronize()
+    c, p, t = shard.unpack_records(host(st.record)[None, :])
+    idx = host(st.out.expert_indices)
+    assert np.array_equal(c[0], np.bincount(idx.ravel(), minlength=w.E))
+    assert np.array_equal(p[0], host(st.P)) and t[0] == w.T
+
+
 def test_shard_with_wrong_counts_is_reported():
     w = REDUCED["mixtral"]
     inp = _inputs(w, seed=3)
@@ -132,8 +127,9 @@ def test_shard_with_wrong_counts_is_reported():
     g = torch.empty((300, 2), dtype=torch.float32, device="cuda")
     P = torch.empty(w.E, dtype=torch.float32, device="cuda")
     api.moe_route(cfg, x, dev(inp["W_router"]), None, None, idx, g, P, None, ws)
-    wrong = torch.zeros((2, w.E), dtype=torch.int32, device="cuda")   # rank 0's row is not its counts
     E = w.E
+    wrong = torch.zeros((2, 2 * E + 1), dtype=torch.int32, device="cuda")
+    wrong[:, 2 * E] = 300                 # token counts add up; rank 0's counts are not its own
     t = [torch.empty(E, dtype=torch.int32, device="cuda"),
          torch.empty(E + 1, dtype=torch.int32, device="cuda"),
          torch.empty((300, 2), dtype=torch.int32, device="cuda"),
@@ -141,7 +137,15 @@ def test_shard_with_wrong_counts_is_reported():
          torch.empty((300, 2), dtype=torch.uint8, device="cuda"),
          torch.empty(E, dtype=torch.float32, device="cuda"),
          torch.empty(1, dtype=torch.float32, device="cuda")]
-    api.moe_dispatch_shard(cfg, 0, 2, 600, wrong, x, idx, P, *t,
+    api.moe_dispatch_shard(cfg, 0, 2, 600, wrong, x, idx, None, *t,
+                           torch.empty((600, w.d), dtype=torch.bfloat16, device="cuda"), ws)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(ws) == 4
+    # records whose token counts do not add up to T_global
+    right = torch.zeros((2, 2 * E + 1), dtype=torch.int32, device="cuda")
+    api.moe_shard_record(cfg, idx, P, right[0], ws)
+    right[1, 2 * E] = 299
+    api.moe_dispatch_shard(cfg, 0, 2, 600, right, x, idx, None, *t,
                            torch.empty((600, w.d), dtype=torch.bfloat16, device="cuda"), ws)
     torch.cuda.synchronize()
     assert api.moe_device_status(ws) == 4

@@ -1,8 +1,8 @@
 """A batch split over ranks (mixture_experts_top_b200/shard.py), on CPU.
 
-* combine_stats: the exchange's arithmetic in closed form;
-* exchange over two and three gloo ranks: every rank gets the same batch
-  statistics, equal to combine_stats of all ranks' inputs;
+* the exchange record's layout (E counts, E P bits, T) read back on the host;
+* gather_records over two and three gloo ranks: every rank gets every
+  rank's record, in rank order;
 * the reading the sharded dispatch implements: with each rank's slot
   positions offset by the earlier ranks' slots on the same expert and the
   capacity taken from the whole batch, the kept slots are exactly the
@@ -23,14 +23,13 @@ from mixture_experts_top_b200 import shard
 from oracle import moe_oracle as O
 
 
-def test_combine_stats_closed_form():
-    counts = [torch.tensor([3, 0, 1], dtype=torch.int32), torch.tensor([1, 2, 5], dtype=torch.int32)]
-    P = [torch.tensor([0.5, 0.25, 0.25]), torch.tensor([0.0, 1.0, 0.0])]
-    all_counts, Pg, T = shard.combine_stats(counts, P, [2, 6])
-    assert T == 8
-    assert all_counts.tolist() == [[3, 0, 1], [1, 2, 5]]
-    assert torch.allclose(Pg, torch.tensor([1.0 / 8, 6.5 / 8, 0.5 / 8]))
-    assert abs(float(Pg.sum()) - 1.0) < 1e-7
+def test_record_layout_round_trip():
+    counts = np.array([[3, 0, 1], [1, 2, 5]], np.int32)
+    P = np.array([[0.5, 0.25, 0.25], [0.0, 1.0, 0.0]], np.float32)
+    rec = np.concatenate([counts, P.view(np.int32), np.array([[2], [6]], np.int32)], axis=1)
+    assert rec.shape[1] == shard.record_ints(3)
+    c, p, t = shard.unpack_records(rec)
+    assert c.tolist() == counts.tolist() and np.array_equal(p, P) and t.tolist() == [2, 6]
 
 
 def _free_port():
@@ -49,26 +48,26 @@ def _worker(rank, world, port, out):
         P = torch.rand(E, generator=g)
         P = P / P.sum()
         T_local = 10 + 7 * rank
-        res = shard.exchange(counts, P, T_local)
-        out[rank] = (counts, P, T_local, res)
+        record = torch.cat([counts, P.view(torch.int32), torch.tensor([T_local], dtype=torch.int32)])
+        res = shard.gather_records(record)
+        out[rank] = (counts.numpy(), P.numpy(), T_local, res.numpy())
     finally:
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_exchange_over_gloo_ranks(world):
+def test_gather_records_over_gloo_ranks(world):
     port = _free_port()
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
-    ref = shard.combine_stats([res[r][0] for r in range(world)], [res[r][1] for r in range(world)],
-                              [res[r][2] for r in range(world)])
     for r in range(world):
-        all_counts, P, T = res[r][3]
-        assert torch.equal(all_counts, ref[0])
-        assert torch.equal(P, ref[1])
-        assert T == ref[2]
+        c, p, t = shard.unpack_records(res[r][3])
+        for src in range(world):
+            assert np.array_equal(c[src], res[src][0])
+            assert np.array_equal(p[src], res[src][1])
+            assert t[src] == res[src][2]
 
 
 def _sharded_keep(idx, E, cf, blocks):

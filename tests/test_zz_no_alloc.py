@@ -72,3 +72,50 @@ def test_route_noalloc_rejects_calls_beyond_its_scratch():
     st = lib.moe_route_noalloc(ctypes.byref(cfg), p, p, None, None, p, p, p, None, None)
     assert st == api.MOE_ERR_UNSUPPORTED
     assert "scratch" in lib.moe_last_error_message().decode()
+
+
+def test_route_noalloc_fills_its_scratch_exactly():
+    # ceil(T/32) * E = 1024 * 64 = 65536 floats: the whole fixed array, its
+    # last row of column sums included.
+    w = WORKLOADS["fine_grained"].with_tokens(32768)
+    assert -(-w.T // 32) * w.E == 65536
+    inp = make_inputs(w, seed=23, with_experts=False)
+    cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
+                          w.capacity_factor)
+    x, Wr, b, n = dev(inp["x"]), dev(inp["W_router"]), dev(inp["logit_bias"]), dev(inp["noise"])
+    idx0, g0, P0, L0 = _outputs(cfg)
+    api.moe_route_noalloc(cfg, x, Wr, b, n, idx0, g0, P0, L0)
+    ws = api.alloc_workspace(cfg)
+    idx1, g1, P1, L1 = _outputs(cfg)
+    api.moe_route(cfg, x, Wr, b, n, idx1, g1, P1, L1, ws)
+    torch.cuda.synchronize()
+    L1h = host(L1)
+    ok = ~ambiguous_tokens(L1h, w.top_k)
+    assert ok.mean() > 0.99
+    assert np.array_equal(host(idx0)[ok], host(idx1)[ok])
+    assert rel_close(host(g0)[ok], host(g1)[ok], REL_ROUTE)
+    assert rel_close(host(P0), host(P1), REL_ROUTE)
+    # the last CTA's row: tokens of the final 32-token tile were routed
+    assert np.all(host(idx0)[-32:] >= 0)
+
+
+def test_route_noalloc_against_the_oracle():
+    # fp32 tokens (the pages' small linear-expert case): logits within an fp32
+    # accumulation bound of the oracle's, indices identical outside near-ties,
+    # gates and P within 1e-5, on two calls in a row.
+    from oracle import moe_oracle as O
+    for w in (WORKLOADS["tiny_linear"], WORKLOADS["tiny_linear"].with_tokens(1000)):
+        inp = make_inputs(w, seed=29, with_experts=False)
+        cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
+                              w.capacity_factor)
+        idx, g, P, L = _outputs(cfg)
+        api.moe_route_noalloc(cfg, dev(inp["x"]), dev(inp["W_router"]), None, None, idx, g, P, L)
+        torch.cuda.synchronize()
+        ref = O.moe_route(inp["x"], inp["W_router"], w.top_k, w.dtype)
+        scale = np.abs(inp["x"].astype(np.float64)) @ np.abs(inp["W_router"].astype(np.float64))
+        bound = 2 * w.d * 2.0 ** -24 * scale + 2.0 ** -23 * np.abs(ref["logits"])
+        assert np.all(np.abs(host(L).astype(np.float64) - ref["logits"]) <= bound)
+        ok = ~ambiguous_tokens(ref["logits"], w.top_k)
+        assert np.array_equal(host(idx)[ok], ref["expert_indices"][ok])
+        assert rel_close(host(g)[ok], ref["gates"][ok], REL_ROUTE)
+        assert rel_close(host(P), ref["P"], REL_ROUTE)
