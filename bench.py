@@ -133,18 +133,19 @@ def fused_combine(w) -> bool:
 def launches_per_step(w, cfg, world: int = 1) -> int:
     """Kernels of this library launched by one timed step (route, dispatch,
     experts, combine), as the library picks them for this configuration:
-    route = weight split + tensor-core router + P mean (bf16, E <= 64) or
-    SIMT router + P mean; dispatch = count + scan + scatter; experts = up and
+    route = weight split + tensor-core router (its last tile writes P; bf16,
+    E <= 64) or SIMT router + P mean; dispatch = count (its last CTA runs
+    the scan) + scatter; experts = up and
     down GEMM (bf16) or the fp32 linear kernel; combine = 1, or 0 where it is
     fused into the down projection (top-1).  A rank of a split batch adds
     its exchange record (count + total)."""
     from mixture_experts_top_b200 import api as _api
     if w.T == 0:
         return 2                       # P mean and the dispatch scan only
-    route = 3 if _api.router_tc_width_supported(cfg) else 2
+    route = 2
     experts = 1 if w.kind == "linear" else 2
     record = 2 if world > 1 else 0
-    return route + record + 3 + experts + (0 if fused_combine(w) else 1)
+    return route + record + 2 + experts + (0 if fused_combine(w) else 1)
 
 
 # ------------------------------------------------------------- ranks (N>1) --
@@ -567,6 +568,7 @@ def extra_workload(name, steps, warmup, peaks, peak_src, base_inputs=None):
     rows = A.kept_rows(counts, w.capacity_factor, w.T, w.top_k)
     used = int((counts > 0).sum())
     regime = regime_of(ms / 1e3)
+    noisy = route_noisy_timing(w, lb, peaks) if w.noise else None
     res = {
         "workload": describe(w), "tokens_per_s": w.T / (ms / steps / 1e3),
         "ms_per_step": ms / steps,
@@ -577,6 +579,7 @@ def extra_workload(name, steps, warmup, peaks, peak_src, base_inputs=None):
         "rows": rows, "used_experts": used,
         "aux_loss": float(lb.layer.out.aux_loss.item()),
         "steps": steps, "warmup": warmup, "inputs_s": gen_s,
+        **({"route_noisy": noisy} if noisy else {}),
     }
     del lb, D
     torch.cuda.empty_cache()
@@ -770,6 +773,43 @@ def routing_backward(w, lb, peaks):
     return {"us": us, "GB/s": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / peaks["hbm_gbs"],
             "note": "moe_combine_backward + moe_route_backward (6 launches): dy read, expert rows "
                     "read and their gradients written, logits and dlogits, x read and dx written"}
+
+
+def route_noisy_timing(w, lb, peaks):
+    """The router with the noisy gate's noise made inside it (moe_route_noisy)
+    against the router fed a host-made noise tensor (moe_route), each back to
+    back on this workload's tokens."""
+    import torch
+    from mixture_experts_top_b200 import api
+    from mixture_experts_top_b200.api import router_tc_width_supported
+    D, o, cfg, stream = lb.D, lb.layer.out, lb.cfg, lb.stream
+    if D.get("W_noise") is None or not router_tc_width_supported(cfg):
+        return None
+    reps = 20
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for _ in range(reps):
+            fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / reps * 1e3
+
+    fused = timed(lambda: api.moe_route_noisy(
+        cfg, D["x"], D["W_router"], D["logit_bias"], D["W_noise"], 7, 0, 0, o.expert_indices,
+        o.gates, lb.P, None, None, lb.layer.ws))
+    host_noise = timed(lambda: api.moe_route(
+        cfg, D["x"], D["W_router"], D["logit_bias"], D["noise"], o.expert_indices, o.gates, lb.P,
+        None, lb.layer.ws))
+    nb = A.router_bytes(w.T, w.d, w.E, w.top_k, 2, False) + w.d * w.E * 4
+    return {"fused_us": fused, "host_noise_us": host_noise,
+            "fused_GB/s": nb / fused / 1e3, "frac_hbm": nb / fused / 1e3 / peaks["hbm_gbs"],
+            "note": "moe_route_noisy (noise logits from the router's own contraction, z and "
+                    "softplus in the logit pass; x, W_router and W_noise read, indices and gates "
+                    "written) vs moe_route reading a (T, E) noise tensor; back to back, 20 calls"}
 
 
 def experts_backward(w, lb, peaks):

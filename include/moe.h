@@ -168,6 +168,26 @@ int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise,
                    uint64_t offset, int64_t token_base, float* noise_out, void* ws,
                    size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route with the noisy gate's noise made inside the router: logits =
+ * x @ W_router (+ logit_bias) + z(token_base + t, e) * softplus((x @ W_noise)
+ * [t, e]), the noise exactly as moe_gate_noise draws it (same Philox stream,
+ * same fp32 noise logits, same fp64 softplus and product), so the results
+ * equal moe_gate_noise followed by moe_route bit for bit -- but the noise
+ * logits come out of the router's own tensor-core contraction (W_noise rides
+ * as three more bf16 terms of the B operand) and the (T, E) noise never
+ * reaches memory unless noise_out asks for it.  [PFD The code, `router`:
+ * the noisy top-k gate]
+ *   bf16 activations and E <= 64 only (MOE_ERR_UNSUPPORTED otherwise: fp32
+ *   tokens and wider gates take moe_gate_noise's noise into moe_route, or
+ *   noise of their own).
+ *   W_noise (d, E) fp32; seed, offset, token_base as in moe_gate_noise;
+ *   noise_out (T, E) fp32 out or NULL; the other arguments as in moe_route. */
+int moe_route_noisy(const moe_config_t* cfg, const void* x, const float* W_router,
+                    const float* logit_bias, const float* W_noise, uint64_t seed, uint64_t offset,
+                    int64_t token_base, int32_t* expert_indices, float* gates, float* prob_mean,
+                    float* logits_out, float* noise_out, void* ws, size_t ws_bytes,
+                    moe_stream_t stream);
+
 /* moe_route without a workspace.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for
  * example a plugin running inside a host program whose memory pool owns the
@@ -431,7 +451,7 @@ int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_ro
  *           (zeros for an expert without rows)
  * bf16 experts run on the tensor cores (bf16 operands, fp32 accumulation):
  * the rows are copied into a layout padded to 128 rows per expert, dY is
- * rounded to bf16, the forward's A and B are recomputed and kept as bf16,
+ * rounded to bf16, the forward's A and B are recomputed and kept in fp32,
  * dA, dB and H are rounded to bf16 between the GEMMs.  Linear experts run
  * in fp32.  Deterministic: no atomics, fixed summation orders. */
 size_t moe_expert_backward_workspace_size(const moe_config_t* cfg);

@@ -31,6 +31,9 @@ _SIGNATURES = {
     "moe_device_status": (ctypes.c_int, [_c_p, ctypes.c_size_t, _c_p, _c_p]),
     "moe_route": (ctypes.c_int, [_c_p] * 10 + [ctypes.c_size_t, _c_p]),
     "moe_route_noalloc": (ctypes.c_int, [_c_p] * 10),
+    "moe_route_noisy": (ctypes.c_int, [_c_p] * 5 + [ctypes.c_uint64, ctypes.c_uint64,
+                                                    ctypes.c_int64] + [_c_p] * 6
+                        + [ctypes.c_size_t, _c_p]),
     "moe_check_wait_timeout": (ctypes.c_int, [_c_p, ctypes.c_size_t, ctypes.c_uint32, _c_p]),
     "moe_expert_backward_workspace_size": (ctypes.c_size_t, [_c_p]),
     "moe_expert_ffn_backward": (ctypes.c_int, [_c_p] * 12 + [ctypes.c_size_t, _c_p]),
@@ -170,6 +173,16 @@ def moe_route(cfg, x, W_router, logit_bias, noise, expert_indices, gates, prob_m
         ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(noise),
         _ptr(expert_indices), _ptr(gates), _ptr(prob_mean), _ptr(logits_out), _ptr(ws),
         ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_noisy(cfg, x, W_router, logit_bias, W_noise, seed, offset, token_base,
+                    expert_indices, gates, prob_mean, logits_out, noise_out, ws,
+                    stream=None) -> None:
+    _check(load_library().moe_route_noisy(
+        ctypes.byref(cfg), _ptr(x), _ptr(W_router), _ptr(logit_bias), _ptr(W_noise), int(seed),
+        int(offset), int(token_base), _ptr(expert_indices), _ptr(gates), _ptr(prob_mean),
+        _ptr(logits_out), _ptr(noise_out), _ptr(ws), ws.numel(), _stream(stream)),
+        "moe_route_noisy")
 
 
 def moe_route_noalloc(cfg, x, W_router, logit_bias, noise, expert_indices, gates, prob_mean,

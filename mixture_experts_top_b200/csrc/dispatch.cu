@@ -12,15 +12,17 @@
 // then lands on grouped row offsets[e] + p, offsets being the exclusive scan
 // of kept_e = min(count_e, cap).
 //
-// Three launches, no atomics on data, no scheduling-dependent order:
+// Two launches, no atomics on data, no scheduling-dependent order:
 //   count   - one CTA per 256-token chunk; each warp ranks 32 tokens' slots
 //             with __match_any_sync (peers with the same expert) against a
 //             per-warp running histogram, then warps are offset by an
 //             exclusive scan over warps.  Writes the chunk histogram and each
 //             slot's rank inside its chunk.
-//   scan    - one CTA: per expert, exclusive scan of the chunk histograms over
-//             chunks (chunk bases) and the total count; kept, offsets, f and
-//             aux = E * sum f_e P_e (fp64, fixed-order butterfly).
+//   scan    - in the last chunk's CTA to finish (a counter in the workspace
+//             finds it; the result does not depend on which CTA it is): per
+//             expert, exclusive scan of the chunk histograms over chunks
+//             (chunk bases) and the total count; kept, offsets, f and aux = E
+//             * sum f_e P_e (fp64, fixed-order butterfly).
 //   scatter - one warp per token: dest, drop mask, perm_token, and the copy
 //             of x[t] into every kept grouped row with 16-byte vectors
 //             (skipped when x_perm is null: the up projection then gathers
@@ -34,10 +36,138 @@ namespace {
 constexpr int kCountWarps = kChunkTokens / 32;  // 8 warps, 32 tokens each
 constexpr int kMaxE = 256;
 
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Arguments of the scan (one CTA): per expert, the exclusive scan of the
+// chunk histograms over chunks (chunk bases) and the total; the capacity,
+// offsets, f and aux; and, for a rank of a sharded batch, the earlier ranks'
+// slots and the batch's P from the exchange records.
+struct ScanArgs {
+  const int32_t* chunk_counts;
+  int nchunks, E, T, k;
+  int64_t cap;
+  const float* prob_mean;
+  int32_t* chunk_base;
+  int32_t* counts;
+  int32_t* offsets;
+  float* f;
+  float* aux;
+  const int32_t* records;
+  int rank, world, T_global;
+  int32_t* prefix;
+  int32_t* err;
+};
+
+// The scan by the whole calling CTA (at least two warps).  The chunk
+// histograms are read through L2: they may have been written by other CTAs
+// of the same launch.
+__device__ void dispatch_scan_body(const ScanArgs& a) {
+  __shared__ int32_t s_counts[kMaxE];
+  __shared__ int32_t s_prefix[kMaxE];   // slots of earlier ranks (sharded batch), else 0
+  __shared__ int32_t s_total[kMaxE];    // slots of the whole batch
+  __shared__ float s_P[kMaxE];          // P_e of the batch (sharded) or prob_mean
+  const int E = a.E, nchunks = a.nchunks, T = a.T, k = a.k;
+  const int64_t cap = a.cap;
+  const int32_t* records = a.records;
+  const int rank = a.rank, world = a.world, T_global = a.T_global;
+  const int rec = 2 * E + 1;            // ints per exchange record
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nwarps) {
+    int carry = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < nchunks ? __ldcg(a.chunk_counts + (size_t)c * E + e) : 0;
+      const int incl = warp_inclusive_scan(v);
+      if (c < nchunks) a.chunk_base[(size_t)c * E + e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_counts[e] = carry;
+  }
+  // Sharded batch: this rank's tokens follow those of ranks 0..rank-1 in
+  // the batch order, so a slot's position on its expert is offset by their
+  // slots on it; the capacity, f and aux are those of the whole batch, and
+  // P_e is the token-weighted mean of the ranks' P_e, summed in fp64 in rank
+  // order and rounded once to fp32.
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int pre = 0, tot = 0;
+    float P = 0.f;
+    if (records != nullptr) {
+      double acc = 0.0;
+      for (int r = 0; r < world; ++r) {
+        const int32_t* rr = records + (size_t)r * rec;
+        const int v = rr[e];
+        if (r < rank) pre += v;
+        tot += v;
+        acc += (double)__int_as_float(rr[E + e]) * (double)rr[2 * E];
+      }
+      a.prefix[e] = pre;
+      P = T_global > 0 ? (float)(acc / (double)T_global) : 0.f;
+    } else {
+      P = a.prob_mean[e];
+    }
+    s_prefix[e] = pre;
+    s_total[e] = records != nullptr ? tot : 0;
+    s_P[e] = P;
+  }
+  __syncthreads();
+  if (records != nullptr) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      if (records[(size_t)rank * rec + e] != s_counts[e]) report_error(a.err, kDevBadShard);
+    if (threadIdx.x == 0) {
+      long long tokens = 0;
+      for (int r = 0; r < world; ++r) tokens += records[(size_t)r * rec + 2 * E];
+      if (tokens != (long long)T_global || records[(size_t)rank * rec + 2 * E] != T)
+        report_error(a.err, kDevBadShard);
+    }
+  }
+  if (warp == 0) {
+    int run = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int cnt = e < E ? s_counts[e] : 0;
+      const int64_t room = cap < 0 ? (int64_t)cnt : cap - (int64_t)(e < E ? s_prefix[e] : 0);
+      const int kept = room <= 0 ? 0 : (room < cnt ? (int)room : cnt);
+      const int incl = warp_inclusive_scan(kept);
+      if (e < E) {
+        a.offsets[e] = run + incl - kept;
+        a.counts[e] = cnt;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) a.offsets[E] = run;
+  } else if (warp == 1) {
+    const bool sharded = records != nullptr;
+    const double slots = (double)(sharded ? T_global : T) * (double)k;
+    double acc = 0.0;
+    for (int e = lane; e < E; e += 32) {
+      const double fe = slots > 0.0 ? (double)(sharded ? s_total[e] : s_counts[e]) / slots : 0.0;
+      a.f[e] = (float)fe;
+      acc += fe * (double)s_P[e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) a.aux[0] = (float)((double)E * acc);
+  }
+}
+
+// The scan alone (no chunks to count: T = 0).
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(const ScanArgs a) {
+  pdl_wait_and_release();
+  dispatch_scan_body(a);
+}
+
 __global__ void __launch_bounds__(kCountWarps * 32)
     dispatch_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                           int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
-                          int32_t* err) {
+                          int32_t* err, const ScanArgs scan, unsigned* __restrict__ done) {
   pdl_wait_and_release();
   __shared__ int32_t whist[kCountWarps][kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -84,108 +214,19 @@ __global__ void __launch_bounds__(kCountWarps * 32)
       if (e >= 0 && e < E) local_rank[s] += wbase[warp][e];
     }
   }
-}
-
-__device__ __forceinline__ int warp_inclusive_scan(int v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  return v;
-}
-
-__global__ void __launch_bounds__(1024)
-    dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E, int T,
-                         int k, int64_t cap, const float* __restrict__ prob_mean,
-                         int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
-                         int32_t* __restrict__ offsets, float* __restrict__ f,
-                         float* __restrict__ aux, const int32_t* __restrict__ records,
-                         int rank, int world, int T_global, int32_t* __restrict__ prefix,
-                         int32_t* err) {
-  pdl_wait_and_release();
-  __shared__ int32_t s_counts[kMaxE];
-  __shared__ int32_t s_prefix[kMaxE];   // slots of earlier ranks (sharded batch), else 0
-  __shared__ int32_t s_total[kMaxE];    // slots of the whole batch
-  __shared__ float s_P[kMaxE];          // P_e of the batch (sharded) or prob_mean
-  const int rec = 2 * E + 1;            // ints per exchange record
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nwarps) {
-    int carry = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < nchunks ? chunk_counts[(size_t)c * E + e] : 0;
-      const int incl = warp_inclusive_scan(v);
-      if (c < nchunks) chunk_base[(size_t)c * E + e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+  // With `done`, the last chunk's CTA to finish runs the scan (all chunk
+  // histograms are complete and visible by then), and leaves `done` at 0.
+  if (done != nullptr) {
+    __threadfence();
+    __syncthreads();
+    __shared__ int s_last;
+    if (threadIdx.x == 0) s_last = atomicAdd(done, 1u) == gridDim.x - 1u;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      dispatch_scan_body(scan);
+      if (threadIdx.x == 0) atomicExch(done, 0u);
     }
-    if (lane == 0) s_counts[e] = carry;
-  }
-  // Sharded batch: this rank's tokens follow those of ranks 0..rank-1 in
-  // the batch order, so a slot's position on its expert is offset by their
-  // slots on it; the capacity, f and aux are those of the whole batch, and
-  // P_e is the token-weighted mean of the ranks' P_e, summed in fp64 in rank
-  // order and rounded once to fp32.
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int pre = 0, tot = 0;
-    float P = 0.f;
-    if (records != nullptr) {
-      double acc = 0.0;
-      for (int r = 0; r < world; ++r) {
-        const int32_t* rr = records + (size_t)r * rec;
-        const int v = rr[e];
-        if (r < rank) pre += v;
-        tot += v;
-        acc += (double)__int_as_float(rr[E + e]) * (double)rr[2 * E];
-      }
-      prefix[e] = pre;
-      P = T_global > 0 ? (float)(acc / (double)T_global) : 0.f;
-    } else {
-      P = prob_mean[e];
-    }
-    s_prefix[e] = pre;
-    s_total[e] = records != nullptr ? tot : 0;
-    s_P[e] = P;
-  }
-  __syncthreads();
-  if (records != nullptr) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-      if (records[(size_t)rank * rec + e] != s_counts[e]) report_error(err, kDevBadShard);
-    if (threadIdx.x == 0) {
-      long long tokens = 0;
-      for (int r = 0; r < world; ++r) tokens += records[(size_t)r * rec + 2 * E];
-      if (tokens != (long long)T_global || records[(size_t)rank * rec + 2 * E] != T)
-        report_error(err, kDevBadShard);
-    }
-  }
-  if (warp == 0) {
-    int run = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int cnt = e < E ? s_counts[e] : 0;
-      const int64_t room = cap < 0 ? (int64_t)cnt : cap - (int64_t)(e < E ? s_prefix[e] : 0);
-      const int kept = room <= 0 ? 0 : (room < cnt ? (int)room : cnt);
-      const int incl = warp_inclusive_scan(kept);
-      if (e < E) {
-        offsets[e] = run + incl - kept;
-        counts[e] = cnt;
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) offsets[E] = run;
-  } else if (warp == 1) {
-    const bool sharded = records != nullptr;
-    const double slots = (double)(sharded ? T_global : T) * (double)k;
-    double acc = 0.0;
-    for (int e = lane; e < E; e += 32) {
-      const double fe = slots > 0.0 ? (double)(sharded ? s_total[e] : s_counts[e]) / slots : 0.0;
-      f[e] = (float)fe;
-      acc += fe * (double)s_P[e];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) aux[0] = (float)((double)E * acc);
   }
 }
 
@@ -242,22 +283,41 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
                             int32_t* local_rank, int32_t* err, cudaStream_t s,
-                            const ShardInfo* shard, int32_t* shard_prefix) {
+                            const ShardInfo* shard, int32_t* shard_prefix, unsigned* done) {
   const int nchunks = ceil_div(c.T, kChunkTokens);
   const int64_t cap = capacity_slots(c.capacity_factor, shard != nullptr ? shard->T_global : c.T,
                                      c.top_k, c.E);
+  ScanArgs sa;
+  sa.chunk_counts = chunk_counts;
+  sa.nchunks = nchunks;
+  sa.E = c.E;
+  sa.T = c.T;
+  sa.k = c.top_k;
+  sa.cap = cap;
+  sa.prob_mean = prob_mean;
+  sa.chunk_base = chunk_base;
+  sa.counts = counts;
+  sa.offsets = offsets;
+  sa.f = f;
+  sa.aux = aux;
+  sa.records = shard != nullptr ? shard->records : nullptr;
+  sa.rank = shard != nullptr ? shard->rank : 0;
+  sa.world = shard != nullptr ? shard->world : 1;
+  sa.T_global = shard != nullptr ? shard->T_global : c.T;
+  sa.prefix = shard != nullptr ? shard_prefix : nullptr;
+  sa.err = err;
+  cudaError_t e;
   if (nchunks > 0) {
-    cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
-                                  c.T, c.top_k, c.E, chunk_counts, local_rank, err);
+    // count, with the scan in the last chunk's CTA when `done` is given
+    e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx, c.T,
+                      c.top_k, c.E, chunk_counts, local_rank, err, sa, done);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = launch_kernel(
-      dispatch_scan_kernel, 1, 1024, 0, s, 0, chunk_counts, nchunks, c.E, c.T, c.top_k, cap,
-      prob_mean, chunk_base, counts, offsets, f, aux,
-      shard != nullptr ? shard->records : nullptr, shard != nullptr ? shard->rank : 0,
-      shard != nullptr ? shard->world : 1, shard != nullptr ? shard->T_global : c.T,
-      shard != nullptr ? shard_prefix : nullptr, err);
-  if (e != cudaSuccess || c.T == 0) return e;
+  if (nchunks == 0 || done == nullptr) {
+    e = launch_kernel(dispatch_scan_kernel, 1, 1024, 0, s, 0, sa);
+    if (e != cudaSuccess) return e;
+  }
+  if (c.T == 0) return cudaSuccess;
   const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
   return launch_kernel(elem == 2 ? dispatch_scatter_kernel<2> : dispatch_scatter_kernel<4>, blocks,
@@ -290,7 +350,8 @@ cudaError_t launch_dispatch_count(const moe_config_t& c, const int32_t* idx, int
   const int nchunks = ceil_div(c.T, kChunkTokens);
   if (nchunks > 0) {
     cudaError_t e = launch_kernel(dispatch_count_kernel, nchunks, kCountWarps * 32, 0, s, 0, idx,
-                                  c.T, c.top_k, c.E, chunk_counts, local_rank, err);
+                                  c.T, c.top_k, c.E, chunk_counts, local_rank, err, ScanArgs{},
+                                  (unsigned*)nullptr);
     if (e != cudaSuccess) return e;
   }
   return launch_kernel(dispatch_total_kernel, 1, 256, 0, s, 0, chunk_counts, nchunks, c.E,

@@ -211,7 +211,7 @@ ExpertBwdLayout expert_backward_layout(const moe_config_t& c) {
     const size_t wide = (c.expert_kind == MOE_EXPERT_SWIGLU ? 2 : 1) * DHp;
     L.xp = take(Rp * (size_t)c.d * 2);
     L.dyp = take(Rp * (size_t)c.d_out * 2);
-    L.pre = take(Rp * wide * 2);
+    L.pre = take(Rp * wide * 4);
     L.dab = take(Rp * wide * 2);
     L.hid = take(Rp * DHp * 2);
   }
@@ -256,7 +256,7 @@ cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
   return launch_expert_backward_gemms(
       c, offsets, xp, dyp, static_cast<const __nv_bfloat16*>(W_in),
       static_cast<const __nv_bfloat16*>(W_up), static_cast<const __nv_bfloat16*>(W_out),
-      reinterpret_cast<__nv_bfloat16*>(base + L.pre), reinterpret_cast<__nv_bfloat16*>(base + L.dab),
+      reinterpret_cast<float*>(base + L.pre), reinterpret_cast<__nv_bfloat16*>(base + L.dab),
       reinterpret_cast<__nv_bfloat16*>(base + L.hid), dx_perm, dW_in, dW_up, dW_out, err, s);
 }
 

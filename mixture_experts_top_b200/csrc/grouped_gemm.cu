@@ -36,10 +36,9 @@
 //    block (read from HBM once, reused from L2) across the expert's row blocks.
 //    Row tiles are re-read for every column block, so they are loaded with an
 //    evict-last L2 policy; weights keep the normal policy (an evict-first
-//    policy on all of them made CTAs that share a weight block re-read it
-//    from HBM).  The last reader of a block (a row block's last column block,
-//    a weight block's last row block) loads it evict-first, so that blocks
-//    no tile needs again leave L2 before live ones.
+//    policy on them made CTAs that share a weight block re-read it from HBM,
+//    and so did evict-first on only each block's last reader: 6.9 GB read
+//    per Mixtral step against 5.4 GB).
 //  * A tile that straddles two experts' rows reads the next expert's rows,
 //    computes them, and masks them at the store: no padding of the grouped
 //    layout is needed.
@@ -108,6 +107,9 @@ struct GemmArgs {
   const float* gates;
   const int32_t* dest;  // (T) slot of each token, -1 if dropped: that output row is zeroed
   int T;
+  // Pair kernel: [0] the next tile to hand out, [1] CTAs finished; both 0
+  // at launch and left at 0 by the last CTA to finish.
+  unsigned* sched;
 };
 
 struct TileCoord {
@@ -336,15 +338,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
-    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal(),
-                   done = l2_policy_evict_first();
+    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_normal();
     for (int tile = blockIdx.x; tile < total_tiles && alive; tile += gridDim.x) {
       const TileCoord c = decode_tile(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
-      // The row block's last column block and the weight block's last row
-      // block read their operand for the last time.
-      const uint64_t pol_a = c.n_tile == g.n_tiles - 1 ? done : keep;
-      const uint64_t pol_b = c.m0 + BM >= row_off[c.e + 1] ? done : stream;
       int r4[4] = {0, 0, 0, 0};
       if (GATHER) {
 #pragma unroll
@@ -498,22 +495,114 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // full barrier; the leader's commits are multicast to both CTAs' empty and
 // accumulator-full barriers; both CTAs' epilogue warps release an
 // accumulator by arriving on the leader's barrier.  No load is multicast.
+// Tiles are handed out dynamically, in order: the leader's producer claims
+// the next tile index from a counter in global memory and publishes it to
+// both CTAs through a small queue in shared memory (the peer's copy written
+// through distributed shared memory); every role of both CTAs takes its
+// tiles from that queue.  Pairs that run together therefore always work on
+// neighbouring tiles, which share weight and row blocks in L2, however far
+// apart their earlier tiles took them.
 // ---------------------------------------------------------------------------
 
 constexpr int PBM = 2 * BM;                       // rows per pair tile
+constexpr int kTileQ = 4;                         // tile indices published ahead
+// Readers of each published tile index: the leader's MMA thread, the peer's
+// producer, and the four epilogue warps of each CTA.
+constexpr int kTileQConsumers = 1 + 1 + 4 + 4;
 constexpr int P_STAGES = 6;
 constexpr int P_STAGE_BYTES = A_STAGE + B_STAGE / 2;  // 32 KiB
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES;
+constexpr int kTailBox = 32;                      // token rows per TMA box of a tail tile
+constexpr int kSwapMaxRows = PBM - 1;             // tail tiles of at most this many rows swap
+constexpr int kXbufStride = 33;                   // floats per column in the exchange buffer
+constexpr int P_XBUF_BYTES = 64 * kXbufStride * 4;   // SwiGLU tail: 64 columns x 32 tokens
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES + P_XBUF_BYTES;
 constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
+// A tail tile's instruction: A = the weights, MN-major (bit 15), B = the
+// tokens, K-major (bit 16 = 0), N = the tile's rows rounded up to 16.
+__device__ __forceinline__ uint32_t idesc_pair_swap(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
+}
+__device__ __forceinline__ int tail_n(int rows) { return (rows + 15) & ~15; }
+
+__device__ __forceinline__ void epilogue_bar_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps
+}
+
+// Epilogue of a tail tile (operands swapped): TMEM lane (q*32 + lane) of
+// this CTA is one output column, TMEM column j is token row m0 + j.  The
+// values are those of the normal tile, only transposed: column `col` of
+// grouped row m0 + j.  SwiGLU: this CTA's lanes 0-63 hold gate columns and
+// lanes 64-127 the matching up columns, which warps q = 2, 3 hand to warps
+// q = 0, 1 through shared memory.
+template <int EPI>
+__device__ __forceinline__ void store_tail_tile(uint32_t tacc, const TileCoord& c, int n0,
+                                                int rank, int q, int lane, float* xbuf,
+                                                const GemmArgs& g) {
+  const int nt = tail_n(c.rows);
+#pragma unroll 1
+  for (int j0 = 0; j0 < nt; j0 += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tacc + (uint32_t)j0, r);
+    tmem_ld_wait();
+    const int nvalid = min(32, c.rows - j0);
+    if (EPI == kEpiSwiglu) {
+      if (q >= 2) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xbuf[((q - 2) * 32 + lane) * kXbufStride + i] = __uint_as_float(r[i]);
+      }
+      epilogue_bar_sync();
+      if (q < 2) {
+        const int col = n0 + 64 * rank + q * 32 + lane;
+        if (col < g.N) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i < nvalid) {
+              const float gv = __uint_as_float(r[i]);
+              const float uv = xbuf[(q * 32 + lane) * kXbufStride + i];
+              out[(size_t)(c.m0 + j0 + i) * g.N + col] = __float2bfloat16_rn(silu_f(gv) * uv);
+            }
+          }
+        }
+      }
+      epilogue_bar_sync();
+    } else {
+      const int col = n0 + 128 * rank + q * 32 + lane;
+      if (col < g.N) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i >= nvalid) break;
+          const float v = __uint_as_float(r[i]);
+          const size_t m = (size_t)(c.m0 + j0 + i);
+          if (EPI == kEpiNone) {
+            static_cast<float*>(g.out)[m * g.N + col] = v;
+          } else if (EPI == kEpiRelu) {
+            static_cast<__nv_bfloat16*>(g.out)[m * g.N + col] = __float2bfloat16_rn(fmaxf(v, 0.f));
+          } else {   // kEpiScatter
+            const int tok = g.rows[m];
+            if (tok >= 0 && tok < g.T)
+              static_cast<__nv_bfloat16*>(g.out)[(size_t)tok * g.N + col] =
+                  __float2bfloat16_rn(g.gates[tok] * v);
+          }
+        }
+      }
+    }
+  }
+}
 
 template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
-                             const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
+                             const __grid_constant__ CUtensorMap tmB1,
+                             const __grid_constant__ CUtensorMap tmAt, const GemmArgs g) {
   pdl_wait_and_release();
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  // An expert's last row block with fewer than 256 rows runs as a tail tile
+  // (operands swapped, N = its rows): no MMA work on padding rows.
+  constexpr bool SWAP = !GATHER;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -522,14 +611,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tfull_bar = empty_bar + P_STAGES;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint64_t* drain_bar = tempty_bar + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
-  int* tile_prefix = reinterpret_cast<int*>(tmem_holder + 4);  // MAX_E + 1
+  uint64_t* tq_full = drain_bar + 1;         // [kTileQ] a tile index was published
+  uint64_t* tq_empty = tq_full + kTileQ;     // [kTileQ] (leader) every consumer has read it
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
+  int* tile_q = reinterpret_cast<int*>(tmem_holder + 4);         // kTileQ
+  int* tile_prefix = tile_q + kTileQ;                            // MAX_E + 1
   int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
+  float* xbuf = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES + AUX_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E;
   const uint32_t rank = cluster_cta_rank();   // 0 = leader, 1 = peer
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (warp == 0) {
     for (int e = lane; e <= E; e += 32) row_off[e] = g.offsets[e];
@@ -557,6 +649,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_map(&tmA);
       tma_prefetch_map(&tmB0);
       tma_prefetch_map(&tmB1);
+      if (SWAP) tma_prefetch_map(&tmAt);
     }
   } else if (warp == 1) {
     tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -571,6 +664,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tempty_bar[b], 8);  // one arrive per epilogue warp of both CTAs
     }
     mbar_init(drain_bar, 1);
+    for (int q = 0; q < kTileQ; ++q) {
+      mbar_init(&tq_full[q], 1);
+      mbar_init(&tq_empty[q], kTileQConsumers);
+    }
     fence_mbar_init();
   }
   tc_fence_before_sync();
@@ -590,29 +687,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t issued_mask = 0, last_phase = 0;
     bool alive = true;
     const CUtensorMap* bmap = (EPI == kEpiSwiglu && rank == 1) ? &tmB1 : &tmB0;
-    const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_normal(),
-                   done = l2_policy_evict_first();
-    for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
+    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_normal();
+    // Tiles are handed out in order: the leader claims the next index from
+    // the global counter (one claim ahead, so its latency hides behind a
+    // tile) and publishes it to both CTAs' queues; the peer reads it there.
+    unsigned next = 0;
+    if (rank == 0 && lane == 0) next = atomicAdd(&g.sched[0], 1u);
+    for (int i = 0; alive; ++i) {
+      const int slot = i & (kTileQ - 1);
+      const uint32_t qpar = (uint32_t)(i / kTileQ) & 1u;
+      int tile = total_tiles;
+      if (lane == 0) {
+        if (rank == 0) {
+          if (!mbar_wait(&tq_empty[slot], qpar ^ 1u)) {
+            report_error(g.err, kDevTimeoutProducer);
+            alive = false;
+          } else {
+            tile = next < (unsigned)total_tiles ? (int)next : total_tiles;
+            tile_q[slot] = tile;
+            st_cluster_u32(cluster_smem_addr(&tile_q[slot], 1), (uint32_t)tile);
+            mbar_arrive(&tq_full[slot]);
+            mbar_arrive_cluster(cluster_smem_addr(&tq_full[slot], 1));
+            if (tile < total_tiles) next = atomicAdd(&g.sched[0], 1u);
+          }
+        } else {
+          if (!mbar_wait_cluster(&tq_full[slot], qpar)) {
+            report_error(g.err, kDevTimeoutProducer);
+            alive = false;
+          } else {
+            tile = tile_q[slot];
+            mbar_arrive_cluster(cluster_smem_addr(&tq_empty[slot], 0));
+          }
+        }
+      }
+      if (GATHER) {
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+        alive = __shfl_sync(0xffffffffu, alive, 0);
+      }
+      if (!alive || tile >= total_tiles) break;
       const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
-      // The row block's last column block and the weight block's last row
-      // block read their operand for the last time.
-      const uint64_t pol_a = c.n_tile == g.n_tiles - 1 ? done : keep;
-      const uint64_t pol_b = c.m0 + PBM >= row_off[c.e + 1] ? done : stream;
       // this CTA's B half: gate / up for SwiGLU, else the column halves
       const int nb = (EPI == kEpiSwiglu) ? n0 : n0 + (int)rank * (BN / 2);
       const int my_m = c.m0 + (int)rank * BM;
+      // tail tile: this CTA's half of the tokens in 32-row boxes, and its 128
+      // weight columns (SwiGLU: 64 gate and the matching 64 up columns)
+      const bool swap = SWAP && c.rows <= kSwapMaxRows;
+      const int half = tail_n(c.rows) / 2;
+      const int nbox = swap ? (half + kTailBox - 1) / kTailBox : 0;
+      const uint32_t cta_bytes =
+          swap ? (uint32_t)(2 * B_BOX + nbox * kTailBox * BK * 2) : (uint32_t)P_STAGE_BYTES;
       int r4[4] = {0, 0, 0, 0};
       if (GATHER) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = my_m + 4 * lane + i;
+        for (int u = 0; u < 4; ++u) {
+          const int m = my_m + 4 * lane + u;
           int r = m < row_off[E] ? g.perm[m] : 0;   // rows past the last expert: any valid row
           if (r < 0 || r >= g.a_rows) {
             report_error(g.err, kDevBadPerm);
             r = 0;
           }
-          r4[i] = r;
+          r4[u] = r;
         }
       }
       for (int kb = 0; kb < num_kb; ++kb) {
@@ -625,10 +760,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) {
             report_error(g.err, kDevTimeoutProducer);
           } else {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-            if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, pol_a);
-            tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, pol_b);
-            tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, pol_b);
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * cta_bytes);
+            if (swap) {
+              for (int j = 0; j < nbox; ++j)
+                tma_load_2d_pair(sa + j * kTailBox * BK * 2, &tmAt, &full_bar[stage], k0,
+                                 c.m0 + (int)rank * half + j * kTailBox, pol_a);
+              if (EPI == kEpiSwiglu) {
+                tma_load_3d_pair(sb, &tmB0, &full_bar[stage], n0 + 64 * (int)rank, k0, c.e, pol_b);
+                tma_load_3d_pair(sb + B_BOX, &tmB1, &full_bar[stage], n0 + 64 * (int)rank, k0, c.e,
+                                 pol_b);
+              } else {
+                tma_load_3d_pair(sb, &tmB0, &full_bar[stage], nb, k0, c.e, pol_b);
+                tma_load_3d_pair(sb + B_BOX, &tmB0, &full_bar[stage], nb + 64, k0, c.e, pol_b);
+              }
+            } else {
+              if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, pol_a);
+              tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, pol_b);
+              tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, pol_b);
+            }
             issued_mask |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           }
@@ -661,13 +810,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool alive = true;
-    for (int tile = pair; tile < total_tiles && alive; tile += npairs) {
+    for (int i = 0; alive; ++i) {
+      const int slot = i & (kTileQ - 1);
+      if (!mbar_wait(&tq_full[slot], (uint32_t)(i / kTileQ) & 1u)) {
+        report_error(g.err, kDevTimeoutMma);
+        break;
+      }
+      const int tile = tile_q[slot];
+      mbar_arrive(&tq_empty[slot]);
+      if (tile >= total_tiles) break;
       if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u)) {
         report_error(g.err, kDevTimeoutMma);
         break;
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
+      const bool swap = SWAP && c.rows <= kSwapMaxRows;
+      const uint32_t idesc_swap = idesc_pair_swap(tail_n(c.rows));
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase)) {
           report_error(g.err, kDevTimeoutMma);
@@ -677,11 +837,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after_sync();
         const uint32_t sa = smem_u32(smem + stage * P_STAGE_BYTES);
         const uint32_t sb = sa + A_STAGE;
+        if (swap) {
+          // A = the weights (MN-major boxes at sb), B = the tokens (K-major at sa)
 #pragma unroll
-        for (int kk = 0; kk < BK / UK; ++kk) {
-          umma_bf16_ss_pair(d_tmem, desc_a_kmajor(sa + kk * UK * 2),
-                            desc_b_nmajor(sb + kk * UK * 128), kIdescPair,
-                            (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / UK; ++kk)
+            umma_bf16_ss_pair(d_tmem, desc_b_nmajor(sb + kk * UK * 128),
+                              desc_a_kmajor(sa + kk * UK * 2), idesc_swap,
+                              (kb | kk) != 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            umma_bf16_ss_pair(d_tmem, desc_a_kmajor(sa + kk * UK * 2),
+                              desc_b_nmajor(sb + kk * UK * 128), kIdescPair,
+                              (kb | kk) != 0 ? 1u : 0u);
         }
         umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
         if (++stage == P_STAGES) {
@@ -703,7 +871,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = (int)rank * BM + q * 32 + lane;  // row inside the pair tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < total_tiles; tile += npairs) {
+    for (int i = 0;; ++i) {
+      const int slot = i & (kTileQ - 1);
+      if (!mbar_wait_cluster(&tq_full[slot], (uint32_t)(i / kTileQ) & 1u)) {
+        report_error(g.err, kDevTimeoutEpilogue);
+        break;
+      }
+      const int tile = tile_q[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_smem_addr(&tq_empty[slot], 0));
+      if (tile >= total_tiles) break;
       const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
       if (!mbar_wait(&tfull_bar[acc], acc_phase)) {
@@ -712,10 +889,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      const bool valid = row < c.rows;
-      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
-                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
+      if (SWAP && c.rows <= kSwapMaxRows) {
+        store_tail_tile<EPI>(tacc, c, n0, (int)rank, q, lane, xbuf, g);
+      } else {
+        const bool valid = row < c.rows;
+        const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
+                                                   : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+        store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
+      }
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
@@ -731,6 +912,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+  // Every claim of this launch precedes its CTA's arrival here, so the last
+  // CTA to arrive puts the counter back to 0 for the next launch.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&g.sched[1], 1u) == gridDim.x - 1u) {
+      atomicExch(&g.sched[0], 0u);
+      atomicExch(&g.sched[1], 0u);
+    }
   }
 }
 
@@ -771,11 +961,11 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 
 template <int EPI, bool GATHER>
 cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                          const GemmArgs& g, int pairs, cudaStream_t s) {
+                          const CUtensorMap& at, const GemmArgs& g, int pairs, cudaStream_t s) {
   auto kern = grouped_gemm_pair_kernel<EPI, GATHER>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), P_SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, g);
+  return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, at, g);
 }
 
 }  // namespace
@@ -795,8 +985,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
-                                const int32_t* perm, int a_rows, const ScatterCombine* sc) {
+                                const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
+                                cudaStream_t s, const int32_t* perm, int a_rows,
+                                const ScatterCombine* sc) {
   if (rows_max == 0) return cudaSuccess;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const bool gather = perm != nullptr;
@@ -823,20 +1014,26 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   g.gates = sc != nullptr ? sc->gates : nullptr;
   g.dest = sc != nullptr ? sc->dest : nullptr;
   g.T = sc != nullptr ? sc->T : 0;
+  g.sched = sched;
   // Expert groups of 1024 rows or more on average: CTA pairs (M = 256 tiles,
   // a third less traffic per CTA); smaller groups: single CTAs (M = 128
   // tiles waste fewer rows at group edges).
   if (rows_max >= 1024 * E) {
+    if (sched == nullptr) return cudaErrorInvalidValue;
     const long max_pairs = (long)(ceil_div(rows_max, PBM) + E) * g.n_tiles;
     const int pairs = (int)std::min<long>((long)(device_sm_count() / 2), max_pairs);
+    // tail tiles' token rows: the same rows, 32-row boxes
+    CUtensorMap tat;
+    if (!(gather ? encode_a(&tat, A, a_rows, K, 1) : encode_a(&tat, A, rows_max, K, kTailBox)))
+      return cudaErrorInvalidValue;
     if (gather)
-      return epi == kEpiSwiglu ? run_gemm_pair<kEpiSwiglu, true>(ta, tb0, tb1, g, pairs, s)
-                               : run_gemm_pair<kEpiRelu, true>(ta, tb0, tb1, g, pairs, s);
+      return epi == kEpiSwiglu ? run_gemm_pair<kEpiSwiglu, true>(ta, tb0, tb1, tat, g, pairs, s)
+                               : run_gemm_pair<kEpiRelu, true>(ta, tb0, tb1, tat, g, pairs, s);
     switch (epi) {
-      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, g, pairs, s);
-      case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, g, pairs, s);
-      case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, g, pairs, s);
-      default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, tat, g, pairs, s);
+      case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, tat, g, pairs, s);
+      case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, tat, g, pairs, s);
+      default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, tat, g, pairs, s);
     }
   }
   const long max_tiles = (long)(ceil_div(rows_max, BM) + E) * g.n_tiles;

@@ -22,7 +22,7 @@
 // dB and H are zero too).  The four GEMMs (one kernel, the stage selected by
 // a template argument):
 //   kPre   (M rows, N hidden, K d)      pre = Xp [W_in | W_up]: A and B of
-//          the forward, recomputed, stored bf16 as [A | B] per row
+//          the forward, recomputed, stored fp32 as [A | B] per row
 //   kDH    (M rows, N hidden, K d_out)  dH = dYp W_out^T; the epilogue reads
 //          the row's pre-activations and writes dAB = [dA | dB] and H (bf16)
 //   kDX    (M rows, N d, K 2 hidden)    dX = dAB [W_in | W_up]^T, written as
@@ -102,7 +102,7 @@ struct BwdArgs {
   int d, DH, DHp, d_out;    // DHp: DH rounded up to 64
   int n_tiles;              // row-grouped stages: output-column blocks
   int rows_max;             // rows of the unpadded grouped buffers (T * top_k)
-  __nv_bfloat16* pre;       // (Rp, (1 + swiglu) DHp): [A | B] pre-activations
+  float* pre;               // (Rp, (1 + swiglu) DHp) fp32: [A | B] pre-activations
   __nv_bfloat16* dab;       // (Rp, (1 + swiglu) DHp): [dA | dB]
   __nv_bfloat16* hid;       // (Rp, DHp): H
   float* dx;                // (R, d): unpadded grouped rows
@@ -176,9 +176,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const Tile& t, int 
                                               const BwdArgs& g) {
   if (STAGE == kPre) {
     // row: padded row; columns [n0, n0 + 128) gate / up (SwiGLU) or
-    // [n0, n0 + 256) (ReLU) of the pre-activations, bf16.
+    // [n0, n0 + 256) (ReLU) of the pre-activations, kept in fp32.
     const size_t ld = (size_t)(g.swiglu ? 2 : 1) * g.DHp;
-    __nv_bfloat16* prow = g.pre + (size_t)(t.m0 + row) * ld;
+    float* prow = g.pre + (size_t)(t.m0 + row) * ld;
     const int halves = g.swiglu ? 2 : 1;
     const int per = BN / halves;
 #pragma unroll 1
@@ -188,23 +188,19 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const Tile& t, int 
         uint32_t r[32];
         tmem_ld_32x32b_x32(tacc + (uint32_t)(h * per + cc), r);
         tmem_ld_wait();
-        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int col = t.n0 + cc + v * 8;
+        for (int v = 0; v < 8; ++v) {
+          const int col = t.n0 + cc + v * 4;
           if (col < g.DHp)
             *reinterpret_cast<uint4*>(prow + (size_t)h * g.DHp + col) =
-                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
         }
       }
     }
   } else if (STAGE == kDH) {
     const size_t ld = (size_t)(g.swiglu ? 2 : 1) * g.DHp;
     const size_t r = (size_t)(t.m0 + row);
-    const __nv_bfloat16* prow = g.pre + r * ld;
+    const float* prow = g.pre + r * ld;
     __nv_bfloat16* drow = g.dab + r * ld;
     __nv_bfloat16* hrow = g.hid + r * (size_t)g.DHp;
 #pragma unroll 1
@@ -216,12 +212,18 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const Tile& t, int 
       for (int v = 0; v < 4; ++v) {
         const int col = t.n0 + cc + v * 8;
         if (col >= g.DHp) continue;
-        const uint4 av = *reinterpret_cast<const uint4*>(prow + col);
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-        uint32_t bw[4] = {0u, 0u, 0u, 0u};
-        if (g.swiglu) {
-          const uint4 bv = *reinterpret_cast<const uint4*>(prow + g.DHp + col);
-          bw[0] = bv.x; bw[1] = bv.y; bw[2] = bv.z; bw[3] = bv.w;
+        float av[8], bv[8];
+        {
+          const float4 a0 = *reinterpret_cast<const float4*>(prow + col);
+          const float4 a1 = *reinterpret_cast<const float4*>(prow + col + 4);
+          av[0] = a0.x; av[1] = a0.y; av[2] = a0.z; av[3] = a0.w;
+          av[4] = a1.x; av[5] = a1.y; av[6] = a1.z; av[7] = a1.w;
+          if (g.swiglu) {
+            const float4 b0 = *reinterpret_cast<const float4*>(prow + g.DHp + col);
+            const float4 b1 = *reinterpret_cast<const float4*>(prow + g.DHp + col + 4);
+            bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+            bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
+          }
         }
         uint32_t da[4], db[4], hh[4];
 #pragma unroll
@@ -229,10 +231,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const Tile& t, int 
           float dA2[2], dB2[2], H2[2];
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            const float a = __uint_as_float(hf ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
+            const float a = av[2 * i + hf];
             const float dh = __uint_as_float(acc[v * 8 + 2 * i + hf]);
             if (g.swiglu) {
-              const float b = __uint_as_float(hf ? (bw[i] & 0xFFFF0000u) : (bw[i] << 16));
+              const float b = bv[2 * i + hf];
               const float s = sigmoid_f(a);
               const float silu = a * s;
               dA2[hf] = dh * b * (s * (1.0f + a * (1.0f - s)));
@@ -579,7 +581,7 @@ int expert_backward_pad_rows(int rows_max, int E) {
 cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* offsets,
                                          const __nv_bfloat16* xp, const __nv_bfloat16* dyp,
                                          const __nv_bfloat16* W_in, const __nv_bfloat16* W_up,
-                                         const __nv_bfloat16* W_out, __nv_bfloat16* pre,
+                                         const __nv_bfloat16* W_out, float* pre,
                                          __nv_bfloat16* dab, __nv_bfloat16* hid, float* dx_perm,
                                          float* dW_in, float* dW_up, float* dW_out, int32_t* err,
                                          cudaStream_t s) {

@@ -104,16 +104,17 @@ cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* per
                                 static_cast<const float*>(W_in), static_cast<float*>(y_perm), err,
                                 s, perm);
   __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
+  unsigned* sched = at<unsigned>(ws, L.ctrl + kCtrlGemmSched);
   const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
   cudaError_t e = launch_grouped_gemm(
       epi, static_cast<const __nv_bfloat16*>(A), rows_max, c.d,
       static_cast<const __nv_bfloat16*>(W_in),
       epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
-      offsets, hidden, err, s, perm, c.T);
+      offsets, hidden, err, sched, s, perm, c.T);
   if (e != cudaSuccess) return e;
   return launch_grouped_gemm(kEpiNone, hidden, rows_max, c.d_hidden,
                              static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
-                             offsets, y_perm, err, s);
+                             offsets, y_perm, err, sched, s);
 }
 
 // The experts and the combine: for top_k = 1 with bf16 experts the combine
@@ -131,17 +132,18 @@ cudaError_t run_experts_combine(const moe_config_t& c, const void* x_perm,
     int32_t* err = at<int32_t>(ws, L.ctrl);
     const int rows_max = c.T;
     __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
+    unsigned* sched = at<unsigned>(ws, L.ctrl + kCtrlGemmSched);
     const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
     cudaError_t e = launch_grouped_gemm(
         epi, static_cast<const __nv_bfloat16*>(x_perm), rows_max, c.d,
         static_cast<const __nv_bfloat16*>(W_in),
         epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
-        offsets, hidden, err, s);
+        offsets, hidden, err, sched, s);
     if (e != cudaSuccess) return e;
     const ScatterCombine sc{perm_token, gates, dest, c.T};
     return launch_grouped_gemm(kEpiScatter, hidden, rows_max, c.d_hidden,
                                static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
-                               offsets, output, err, s, nullptr, 0, &sc);
+                               offsets, output, err, sched, s, nullptr, 0, &sc);
   }
   void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws, s);
@@ -188,7 +190,8 @@ WsLayout workspace_layout(const moe_config_t& c) {
   const size_t n_chunks = (size_t)std::max(1, ceil_div(c.T, kChunkTokens));
   L.ctrl = take(256);
   L.router_part = take(n_router * E * 4);
-  L.w_split = take((size_t)3 * (size_t)router_tc_width(c) * (size_t)c.d * 2);
+  L.w_split = take((size_t)6 * (size_t)router_tc_width(c) * (size_t)c.d * 2);
+  L.noise_z = take(router_tc_width(c) > 0 ? (size_t)c.T * E * 8 : 0);
   L.prob_mean = take(E * 4);
   L.chunk_counts = take(n_chunks * E * 4);
   L.chunk_base = take(n_chunks * E * 4);
@@ -303,7 +306,8 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* W_router,
   const cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates,
                                      prob_mean, logits_out, at<float>(ws, L.router_part),
                                      at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl),
-                                     reinterpret_cast<cudaStream_t>(stream));
+                                     reinterpret_cast<cudaStream_t>(stream),
+                                     at<unsigned>(ws, L.ctrl + kCtrlRouterDone));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
 }
 
@@ -349,7 +353,7 @@ int dispatch_entry(const moe_config_t* cfg, const moe_shard_t* sh, const void* x
       x_perm, at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
       at<int32_t>(ws, L.local_rank), at<int32_t>(ws, L.ctrl),
       reinterpret_cast<cudaStream_t>(stream), sh != nullptr ? &shard : nullptr,
-      at<int32_t>(ws, L.shard_prefix));
+      at<int32_t>(ws, L.shard_prefix), at<unsigned>(ws, L.ctrl + kCtrlDispatchDone));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, name);
 }
 
@@ -517,6 +521,43 @@ int moe_gate_noise(const moe_config_t* cfg, const void* x, const float* W_noise,
       noise_out, at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl),
       reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_gate_noise");
+}
+
+int moe_route_noisy(const moe_config_t* cfg, const void* x, const float* W_router,
+                    const float* logit_bias, const float* W_noise, uint64_t seed, uint64_t offset,
+                    int64_t token_base, int32_t* expert_indices, float* gates, float* prob_mean,
+                    float* logits_out, float* noise_out, void* ws, size_t ws_bytes,
+                    moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (router_tc_width(c) == 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_noisy: bf16 activations and E <= 64 only "
+                                     "(elsewhere: moe_gate_noise's noise into moe_route)");
+  if (c.T > 0) {
+    MOE_REQUIRE(x);
+    MOE_REQUIRE(expert_indices);
+    MOE_REQUIRE(gates);
+  }
+  MOE_ALIGNED16(x);
+  MOE_REQUIRE(W_router);
+  MOE_REQUIRE(W_noise);
+  MOE_REQUIRE(prob_mean);
+  if (token_base < 0) return fail(MOE_ERR_INVALID_ARG, "token_base must be >= 0");
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = workspace_layout(c);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int tiles = 0;
+  const cudaError_t e =
+      c.T > 0 ? launch_route_tc_noisy(c, static_cast<const __nv_bfloat16*>(x), W_router,
+                                      logit_bias, W_noise, seed, offset, (long long)token_base,
+                                      expert_indices, gates, logits_out, noise_out,
+                                      at<float>(ws, L.router_part),
+                                      at<__nv_bfloat16>(ws, L.w_split), at<double>(ws, L.noise_z),
+                                      at<int32_t>(ws, L.ctrl), s, &tiles, prob_mean,
+                                      at<unsigned>(ws, L.ctrl + kCtrlRouterDone))
+              : launch_prob_mean(at<float>(ws, L.router_part), 0, c.E, 0, prob_mean, s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_noisy");
 }
 
 int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* expert_indices,
@@ -712,12 +753,14 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   void* x_perm = at<void>(ws, L.x_perm);
   cudaError_t e = launch_route(c, x, W_router, logit_bias, noise, expert_indices, gates, P,
                                nullptr, at<float>(ws, L.router_part),
-                               at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl), s);
+                               at<__nv_bfloat16>(ws, L.w_split), at<int32_t>(ws, L.ctrl), s,
+                               at<unsigned>(ws, L.ctrl + kCtrlRouterDone));
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/route");
   e = launch_dispatch(c, x, expert_indices, P, cnt, offs, dest, perm, drop, at<float>(ws, L.f),
                       aux_loss, x_perm, at<int32_t>(ws, L.chunk_counts),
                       at<int32_t>(ws, L.chunk_base), at<int32_t>(ws, L.local_rank),
-                      at<int32_t>(ws, L.ctrl), s);
+                      at<int32_t>(ws, L.ctrl), s, nullptr, nullptr,
+                      at<unsigned>(ws, L.ctrl + kCtrlDispatchDone));
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/dispatch");
   // The materialised permute (one copy of each kept row, ~38 us at the
   // Mixtral shape) is far cheaper than gathering A rows inside the GEMM,

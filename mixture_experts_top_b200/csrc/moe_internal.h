@@ -25,7 +25,8 @@ constexpr int kChunkTokens = 256;
 struct WsLayout {
   size_t ctrl;           // int32 error word (+ padding)
   size_t router_part;    // (router CTAs, E) fp32 per-CTA column sums of probs
-  size_t w_split;        // (3, EP, d) bf16: W_router split for the tensor-core router
+  size_t w_split;        // (6, EP, d) bf16: W_router (and W_noise) split for the tensor-core router
+  size_t noise_z;        // (T, E) fp64: the noisy gate's draws (moe_route_noisy)
   size_t prob_mean;      // (E) fp32, moe_forward only
   size_t chunk_counts;   // (chunks, E) int32
   size_t chunk_base;     // (chunks, E) int32
@@ -96,25 +97,54 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 }
 
 // Launchers; each returns cudaSuccess or the launch error.
-// w_split (3 * router_tc_width(c) * d bf16) selects the tensor-core router
+// w_split (6 * router_tc_width(c) * d bf16) selects the tensor-core router
 // where router_tc_width(c) > 0; nullptr always runs the SIMT router.  err is
-// the workspace error word (may be nullptr with w_split == nullptr).
+// the workspace error word and done its tile counter (both may be nullptr
+// with w_split == nullptr).
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
-                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s);
+                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s,
+                         unsigned* done = nullptr);
+// The workspace's control block (first 256 bytes, cleared by
+// moe_workspace_init): the error word at byte 0, the router's tile counter
+// at byte kCtrlRouterDone, the pair GEMM's tile counter (two unsigned) at
+// byte kCtrlGemmSched and the dispatch count's chunk counter at byte
+// kCtrlDispatchDone, each on its own 64-byte line.  The kernels leave every
+// counter at 0.
+constexpr size_t kCtrlRouterDone = 64;
+constexpr size_t kCtrlGemmSched = 128;
+constexpr size_t kCtrlDispatchDone = 192;
 // The noisy gate's noise (router_tc.cu): noise_out (T, E) fp32 =
 // z(token_base + t, e) * softplus(x @ W_noise); bf16 x and E <= 64 only.
 cudaError_t launch_gate_noise(const moe_config_t& c, const __nv_bfloat16* x, const float* W_noise,
                               uint64_t seed, uint64_t offset, long long token_base,
                               float* noise_out, __nv_bfloat16* w_split, int32_t* err,
                               cudaStream_t s);
-// Tensor-core router (router_tc.cu): logits, softmax, top-k, gates and one
-// row of probability column sums per 128-token tile; *tiles_out = rows.
+// Tensor-core router (router_tc.cu): logits, softmax, top-k, gates, one row
+// of probability column sums per 128-token tile (*tiles_out = rows) and,
+// from the last tile to finish, P_e into prob_mean; `done` is a counter that
+// must be 0 before the launch and is 0 again after it.
 cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W_router,
                             const float* bias, const float* noise, int32_t* idx, float* gates,
                             float* logits_out, float* router_part, __nv_bfloat16* w_split,
-                            int32_t* err, cudaStream_t s, int* tiles_out);
+                            int32_t* err, cudaStream_t s, int* tiles_out, float* prob_mean,
+                            unsigned* done);
+
+// The tensor-core router with the noisy gate's noise made in the kernel:
+// noise = z(token_base + t, e) * softplus(x @ W_noise) added after the bias;
+// noise_out (T, E) fp32 or nullptr receives the noise drawn.  w_split holds
+// 6 * router_tc_width(c) * d bf16, noise_z (T, E) fp64 the draws z.
+cudaError_t launch_route_tc_noisy(const moe_config_t& c, const __nv_bfloat16* x,
+                                  const float* W_router, const float* bias, const float* W_noise,
+                                  uint64_t seed, uint64_t offset, long long token_base,
+                                  int32_t* idx, float* gates, float* logits_out, float* noise_out,
+                                  float* router_part, __nv_bfloat16* w_split, double* noise_z,
+                                  int32_t* err, cudaStream_t s, int* tiles_out, float* prob_mean,
+                                  unsigned* done);
+// P_e = (the column-sum rows of router_part added in fp64) / T (router.cu).
+cudaError_t launch_prob_mean(const float* router_part, int rows, int E, int T, float* prob_mean,
+                             cudaStream_t s);
 
 // A batch split over `world` ranks in contiguous token blocks, rank order:
 // every rank's exchange record (world, 2E+1) int32 on the device (E slot
@@ -129,7 +159,8 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
                             int32_t* dest, int32_t* perm_token, uint8_t* drop_mask, float* f,
                             float* aux, void* x_perm, int32_t* chunk_counts, int32_t* chunk_base,
                             int32_t* local_rank, int32_t* err, cudaStream_t s,
-                            const ShardInfo* shard = nullptr, int32_t* shard_prefix = nullptr);
+                            const ShardInfo* shard = nullptr, int32_t* shard_prefix = nullptr,
+                            unsigned* done = nullptr);
 // The per-expert slot counts of `idx` (T, top_k) into counts (E); with
 // prob_mean != nullptr, counts is a (2E+1) exchange record: the counts,
 // the fp32 bits of prob_mean and T.
@@ -163,10 +194,12 @@ struct ScatterCombine {
 // perm != nullptr (ReLU / SwiGLU only): grouped row r of A is row perm[r] of
 // A, an (a_rows, K) tensor, fetched by TMA row gathers (the permute fused into
 // the up projection's operand load).
+// sched: the workspace's tile counter (two unsigned, 0 before the launch and
+// left at 0), used where the CTA-pair kernel runs.
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
-                                const int32_t* offsets, void* out, int32_t* err, cudaStream_t s,
-                                const int32_t* perm = nullptr, int a_rows = 0,
+                                const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
+                                cudaStream_t s, const int32_t* perm = nullptr, int a_rows = 0,
                                 const ScatterCombine* sc = nullptr);
 
 // Experts' backward (expert_backward.cu, grouped_gemm_bwd.cu).  The bf16
@@ -176,7 +209,8 @@ constexpr int kBwdPadRows = 128;
 // Rows of the padded layout for at most rows_max grouped rows.
 int expert_backward_pad_rows(int rows_max, int E);
 // Workspace of moe_expert_ffn_backward: error word; padded rows Xp (bf16),
-// dYp (bf16); pre-activations [A | B], their gradients [dA | dB] and H.
+// dYp (bf16); pre-activations [A | B] (fp32), their gradients [dA | dB] and
+// H (bf16).
 struct ExpertBwdLayout {
   size_t ctrl, xp, dyp, pre, dab, hid, total;
 };
@@ -189,7 +223,7 @@ cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
 cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* offsets,
                                          const __nv_bfloat16* xp, const __nv_bfloat16* dyp,
                                          const __nv_bfloat16* W_in, const __nv_bfloat16* W_up,
-                                         const __nv_bfloat16* W_out, __nv_bfloat16* pre,
+                                         const __nv_bfloat16* W_out, float* pre,
                                          __nv_bfloat16* dab, __nv_bfloat16* hid, float* dx_perm,
                                          float* dW_in, float* dW_up, float* dW_out, int32_t* err,
                                          cudaStream_t s);

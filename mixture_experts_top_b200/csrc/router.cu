@@ -418,16 +418,23 @@ cudaError_t dispatch_router(const RouterArgs<XT>& a, cudaStream_t s, int* tiles)
 
 }  // namespace
 
+cudaError_t launch_prob_mean(const float* router_part, int rows, int E, int T, float* prob_mean,
+                             cudaStream_t s) {
+  return launch_kernel(prob_mean_kernel, 1, 256, 0, s, 0, router_part, rows, E, T, prob_mean);
+}
+
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* W_router,
                          const float* bias, const float* noise, int32_t* idx, float* gates,
                          float* prob_mean, float* logits_out, float* router_part,
-                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s) {
+                         __nv_bfloat16* w_split, int32_t* err, cudaStream_t s, unsigned* done) {
   int tiles = 0;  // token tiles; each writes one row of router_part
   if (c.T > 0) {
     cudaError_t e;
-    if (w_split != nullptr && router_tc_width(c) > 0) {
-      e = launch_route_tc(c, static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
-                          gates, logits_out, router_part, w_split, err, s, &tiles);
+    if (w_split != nullptr && done != nullptr && router_tc_width(c) > 0) {
+      // the tensor-core router writes P itself (its last tile)
+      return launch_route_tc(c, static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
+                             gates, logits_out, router_part, w_split, err, s, &tiles, prob_mean,
+                             done);
     } else if (c.act_dtype == MOE_BF16) {
       RouterArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(x), W_router, bias, noise, idx,
                                   gates, logits_out, router_part, c.T, c.d, c.E, c.top_k};

@@ -70,34 +70,53 @@ constexpr int TTHREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 accumulate a
 constexpr int kCoopBatch = 8;  // elements per thread per round of the logit pass
 constexpr int kMaxTopK = 8;    // largest top_k the library accepts
 
-template <int EP>
+// kModeRoute: the router.  kModeLogits: the contraction and the rank-ordered
+// sum only, written to logits_out (the noisy gate's noise logits).
+// kModeNoisy: the router with the noisy gate's noise made in the kernel: the
+// B operand carries W_noise's three terms after W_router's, so each token's
+// noise logits come out of the same contraction, and noise = z * softplus(
+// noise logit) is formed in the logit pass (the (T, E) noise never reaches
+// memory unless asked for).
+enum TcMode { kModeRoute = 0, kModeLogits = 1, kModeNoisy = 2 };
+
+template <int EP, int MODE>
 struct TcShape {
   static_assert(EP == 16 || EP == 32 || EP == 64, "EP is 16, 32 or 64");
-  static constexpr int ST = EP == 16 ? 4 : (EP == 32 ? 3 : 2);   // two CTAs per SM
+  static constexpr bool NOISY = MODE == kModeNoisy;
+  static constexpr int TERMS = NOISY ? 6 : 3;                    // hi, mid, lo (x2 noisy)
+  static constexpr int ST = NOISY ? (EP == 16 ? 3 : 2) : (EP == 16 ? 4 : (EP == 32 ? 3 : 2));
   static constexpr int X_BYTES = TBM * TBK * 2;                  // 16 KiB
   static constexpr int W_PART = EP * TBK * 2;                    // one term's box
-  static constexpr int STAGE = X_BYTES + 3 * W_PART;
-  static constexpr int LGS = EP + 4;                             // padded logit row (floats)
+  static constexpr int STAGE = X_BYTES + TERMS * W_PART;
+  static constexpr int LOGW = NOISY ? 2 * EP : EP;               // a token's logits (+ noise logits)
+  static constexpr int LGS = LOGW + 4;                           // padded logit row (floats)
   static constexpr int PIPE = ST * STAGE;
   static constexpr int LG_BYTES = TBM * LGS * 4;
   static constexpr int MAIN = PIPE > LG_BYTES ? PIPE : LG_BYTES;
   static constexpr int AUX = 256;                                // barriers, TMEM address
   static constexpr int SMEM = 1024 + MAIN + EP * 4 + AUX;
-  // One MMA covers the three terms: B is the 3 EP rows (hi, mid, lo) of the
-  // stage, so an accumulator is 3 EP columns.  Two accumulators alternate
-  // (one when 2 x 3 EP columns would not leave room for a second CTA).
-  static constexpr int N = 3 * EP;
-  static constexpr int NBUF = EP <= 32 ? 2 : 1;
+  // B is the TERMS * EP rows of the stage (W's hi, mid, lo, then W_noise's),
+  // so an accumulator is TERMS * EP columns, issued as one MMA (or two of half
+  // the width where that exceeds the instruction's 256).  Up to four
+  // accumulators rotate within 256 columns (the MMA runs ahead of the
+  // registers' block sums by that many blocks): four at EP = 16, two at
+  // EP = 32, one at EP = 64 or with the noise terms at EP > 16.
+  static constexpr int N = TERMS * EP;
+  static constexpr int NMMA = N <= 256 ? N : N / 2;
+  static constexpr int MMAS = N / NMMA;
+  static constexpr int NBUF = N > 128 ? 1 : (256 / N >= 4 ? 4 : 2);
   static constexpr int G = 1;   // 64-wide d blocks summed per accumulator before it is read
   static constexpr int FG = EP / 8;  // lanes per token in the finishing pass (8 experts each)
   static constexpr uint32_t TMEM_COLS = NBUF * N <= 32 ? 32u : NBUF * N <= 64 ? 64u
-                                        : NBUF * N <= 128 ? 128u : 256u;
+                                        : NBUF * N <= 128 ? 128u : NBUF * N <= 256 ? 256u : 512u;
+  static constexpr int CTAS_PER_SM = TMEM_COLS > 256 ? 1 : 2;
   // kind::f16: D fp32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 =
   // 1), A and B K-major (bits 15, 16 = 0), N >> 3 at 17, M >> 4 at 24.
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(N >> 3) << 17) | ((uint32_t)(TBM >> 4) << 24);
-  static_assert(NBUF * N <= 256 && N % 16 == 0, "accumulators fit half of tensor memory");
-  static_assert((2 * ST + 5) * 8 + 4 <= AUX, "barriers fit");
+                                    ((uint32_t)(NMMA >> 3) << 17) | ((uint32_t)(TBM >> 4) << 24);
+  static_assert(NBUF * N <= 512 && NMMA % 16 == 0 && NMMA * MMAS == N, "accumulators fit");
+  static_assert((NMMA * 128) % 1024 == 0, "second MMA's B starts on an 8-row group");
+  static_assert((2 * ST + 2 * NBUF + 1) * 8 + 4 <= AUX, "barriers fit");
 };
 
 // K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024
@@ -117,15 +136,93 @@ struct TcArgs {
   float* part;
   int32_t* err;
   int T, d, E, k;
+  // kModeNoisy: the noise's Philox key and stream, the batch index of this
+  // call's first token, and an optional (T, E) copy of the noise drawn.
+  uint64_t seed, offset;
+  long long token_base;
+  float* noise_out;
+  const double* noise_z;   // (T, E) the draws z, made before the router runs
+  // kModeRoute / kModeNoisy: P_e, written by the last tile to finish, which
+  // it finds with a counter that starts at 0 and is left at 0.
+  float* prob_mean;
+  unsigned* done;
 };
 
+// Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): ten rounds over a 4-word counter, the key
+// advanced by the two Weyl constants between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
+  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
+    const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
+    const uint64_t y0 = hi1 ^ x[1] ^ k0, y2 = hi0 ^ x[3] ^ k1;
+    x[0] = y0;
+    x[1] = lo1;
+    x[2] = y2;
+    x[3] = lo0;
+  }
+}
+
+// The noisy gate's noise of batch token t and expert e from its noise logit
+// l: z * softplus(l), z the standard normal drawn from Philox4x64-10 of the
+// counter (t, e, offset, 0) under the key (seed, 0): two words to u = ((w >>
+// 11) + 1/2) 2^-53 and z = sqrt(-2 ln u0) cos(2 pi u1) (Box-Muller), in
+// fp64; softplus(l) = max(l, 0) + log1p(exp(-|l|)) in fp64; one rounding.
+__device__ __forceinline__ double gate_noise_z(uint64_t seed, uint64_t offset, long long t,
+                                               int e) {
+  uint64_t w[4] = {(uint64_t)t, (uint64_t)e, offset, 0ull};
+  philox4x64_10(w, seed, 0ull);
+  const double u0 = ((double)(w[0] >> 11) + 0.5) * 0x1.0p-53;
+  const double u1 = ((double)(w[1] >> 11) + 0.5) * 0x1.0p-53;
+  return sqrt(-2.0 * log(u0)) * cos(2.0 * 3.141592653589793 * u1);
+}
+__device__ __forceinline__ float gate_noise_from_z(double z, float l) {
+  const double ld = (double)l;
+  const double sp = fmax(ld, 0.0) + log1p(exp(-fabs(ld)));
+  return (float)(z * sp);
+}
+__device__ __forceinline__ float gate_noise_value(uint64_t seed, uint64_t offset, long long t,
+                                                  int e, float l) {
+  return gate_noise_from_z(gate_noise_z(seed, offset, t, e), l);
+}
+
 // (d, E) fp32 -> (3, EP, d) bf16 terms hi, mid, lo with w = hi + mid + lo.
-// One block per 64 rows of d, transposed through shared memory.
+// One block per 64 rows of d, transposed through shared memory; blockIdx.y
+// = 1 splits W2 into the next three planes.
+// With z_out, the blocks of blockIdx.y = 2 instead draw the noisy gate's
+// z for every (token, expert) of the call (they depend on neither input).
+struct NoiseDraw {
+  double* z_out;          // (T, E) or nullptr
+  uint64_t seed, offset;
+  long long token_base;
+  int T;
+};
+
 __global__ void __launch_bounds__(256)
-    split_router_weights_kernel(const float* __restrict__ W, int d, int E, int EP,
-                                __nv_bfloat16* __restrict__ out) {
+    split_router_weights_kernel(const float* __restrict__ W1, const float* __restrict__ W2, int d,
+                                int E, int EP, __nv_bfloat16* __restrict__ out_base,
+                                const NoiseDraw nd) {
   pdl_wait_and_release();
+  if (blockIdx.y == 2) {
+    const long long n = (long long)nd.T * E;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+      const long long t = i / E;
+      nd.z_out[i] = gate_noise_z(nd.seed, nd.offset, nd.token_base + t, (int)(i - t * E));
+    }
+    return;
+  }
+  if ((int)blockIdx.x * TBK >= d) return;
   __shared__ float tile[TBK][65];
+  const float* __restrict__ W = blockIdx.y == 0 ? W1 : W2;
+  __nv_bfloat16* __restrict__ out = out_base + (size_t)blockIdx.y * 3 * EP * d;
   const int k0 = blockIdx.x * TBK;
   for (int i = threadIdx.x; i < TBK * E; i += blockDim.x) {
     const int kk = i / E, e = i - kk * E;
@@ -147,14 +244,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// LOGITS_ONLY: the contraction and the rank-ordered sum only, written to
-// a.logits_out (the noisy gate's noise logits); no top-k, gates or sums.
-template <int EP, bool LOGITS_ONLY>
-__global__ void __launch_bounds__(TTHREADS, 2)
+template <int EP, int MODE>
+__global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const TcArgs a) {
   pdl_wait_and_release();
-  using S = TcShape<EP>;
+  using S = TcShape<EP, MODE>;
+  constexpr bool LOGITS_ONLY = MODE == kModeLogits;
+  constexpr bool NOISY = MODE == kModeNoisy;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -163,8 +260,8 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S::MAIN + EP * 4);
   uint64_t* empty_bar = full_bar + S::ST;
   uint64_t* tfull_bar = empty_bar + S::ST;   // [NBUF] accumulator written
-  uint64_t* tempty_bar = tfull_bar + 2;      // [NBUF] accumulator read
-  uint64_t* drain_bar = tempty_bar + 2;
+  uint64_t* tempty_bar = tfull_bar + S::NBUF;  // [NBUF] accumulator read
+  uint64_t* drain_bar = tempty_bar + S::NBUF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -190,7 +287,7 @@ __global__ void __launch_bounds__(TTHREADS, 2)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < S::NBUF; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 128);
     }
@@ -244,9 +341,11 @@ __global__ void __launch_bounds__(TTHREADS, 2)
       const uint32_t acc = tmem + (uint32_t)(b * S::N);
 #pragma unroll
       for (int kk = 0; kk < TBK / TUK; ++kk)
-        umma_bf16_ss(acc, desc_kmajor_sw128(sx + kk * TUK * 2),
-                     desc_kmajor_sw128(sw + kk * TUK * 2), S::IDESC,
-                     (!first || kk != 0) ? 1u : 0u);
+#pragma unroll
+        for (int m = 0; m < S::MMAS; ++m)
+          umma_bf16_ss(acc + (uint32_t)(m * S::NMMA), desc_kmajor_sw128(sx + kk * TUK * 2),
+                       desc_kmajor_sw128(sw + m * S::NMMA * 128 + kk * TUK * 2), S::IDESC,
+                       (!first || kk != 0) ? 1u : 0u);
       umma_commit(&empty_bar[stage]);   // frees the stage once these MMAs finish
       if ((c % S::G) == S::G - 1 || c == nchunks - 1)
         umma_commit(&tfull_bar[b]);     // this group's sums are ready
@@ -261,8 +360,11 @@ __global__ void __launch_bounds__(TTHREADS, 2)
     // ------------------------------- per-block sums -> fp32 registers -> smem
     const int q = warp & 3;                 // TMEM lanes 32q .. 32q + 31
     float acc[EP];
+    float nacc[NOISY ? EP : 1];
 #pragma unroll
     for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int e = 0; e < (NOISY ? EP : 1); ++e) nacc[e] = 0.f;
     const int ngroups = (nchunks + S::G - 1) / S::G;
     for (int gi = 0; gi < ngroups; ++gi) {
       const int b = gi % S::NBUF;
@@ -285,6 +387,17 @@ __global__ void __launch_bounds__(TTHREADS, 2)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           acc[c0 + j] += __uint_as_float(hi[j]) + (__uint_as_float(mid[j]) + __uint_as_float(lo[j]));
+        if (NOISY) {
+          // columns [3 EP, 6 EP): W_noise's terms, summed the same way
+          tmem_ld_32x32b_x16(taddr + (uint32_t)(3 * EP + c0), hi);
+          tmem_ld_32x32b_x16(taddr + (uint32_t)(4 * EP + c0), mid);
+          tmem_ld_32x32b_x16(taddr + (uint32_t)(5 * EP + c0), lo);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            nacc[(c0 + j) % (NOISY ? EP : 1)] +=
+                __uint_as_float(hi[j]) + (__uint_as_float(mid[j]) + __uint_as_float(lo[j]));
+        }
       }
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[b]);
@@ -293,6 +406,13 @@ __global__ void __launch_bounds__(TTHREADS, 2)
 #pragma unroll
     for (int e = 0; e < EP; e += 4)
       *reinterpret_cast<float4*>(my + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+    if (NOISY) {
+#pragma unroll
+      for (int e = 0; e < (NOISY ? EP : 1); e += 4)
+        *reinterpret_cast<float4*>(my + EP + e) =
+            make_float4(nacc[e], nacc[(e + 1) % (NOISY ? EP : 1)], nacc[(e + 2) % (NOISY ? EP : 1)],
+                        nacc[(e + 3) % (NOISY ? EP : 1)]);
+    }
   }
   __syncwarp();
   cluster.sync();  // every CTA's partial logits are complete and visible
@@ -310,29 +430,34 @@ __global__ void __launch_bounds__(TTHREADS, 2)
   {
     const int n = rpc * EP;
     for (int base = threadIdx.x; base < n; base += TTHREADS * kCoopBatch) {
-      float acc[kCoopBatch], bv[kCoopBatch], nv[kCoopBatch];
+      float acc[kCoopBatch], bv[kCoopBatch], nv[kCoopBatch], nl[kCoopBatch];
 #pragma unroll
       for (int u = 0; u < kCoopBatch; ++u) {
         const int i = base + u * TTHREADS;
         acc[u] = 0.f;
         bv[u] = 0.f;
         nv[u] = 0.f;
+        nl[u] = 0.f;
         const int r = r0 + i / EP, e = i % EP, t = t_base + r;
         if (i < n && e < E && t < T) {
           if (a.bias != nullptr) bv[u] = a.bias[e];
-          if (a.noise != nullptr) nv[u] = a.noise[(size_t)t * E + e];
+          if (!NOISY && a.noise != nullptr) nv[u] = a.noise[(size_t)t * E + e];
         }
       }
       for (int sp = 0; sp < nsplit; ++sp) {
         const float* src = cluster.map_shared_rank(lg, sp);
-        float pv[kCoopBatch];
+        float pv[kCoopBatch], pn[kCoopBatch];
 #pragma unroll
         for (int u = 0; u < kCoopBatch; ++u) {
           const int i = base + u * TTHREADS;
           pv[u] = i < n ? src[(r0 + i / EP) * S::LGS + i % EP] : 0.f;
+          pn[u] = (NOISY && i < n) ? src[(r0 + i / EP) * S::LGS + EP + i % EP] : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < kCoopBatch; ++u) acc[u] += pv[u];
+        for (int u = 0; u < kCoopBatch; ++u) {
+          acc[u] += pv[u];
+          nl[u] += pn[u];
+        }
       }
 #pragma unroll
       for (int u = 0; u < kCoopBatch; ++u) {
@@ -341,8 +466,14 @@ __global__ void __launch_bounds__(TTHREADS, 2)
           const int r = r0 + i / EP, e = i % EP, t = t_base + r;
           float v = acc[u];
           if (e < E && t < T) {
+            if (NOISY) {
+              // the noise of this token and expert from its noise logit and
+              // its draw (drawn ahead by the weight-split launch)
+              nv[u] = gate_noise_from_z(__ldcg(a.noise_z + (size_t)t * E + e), nl[u]);
+              if (a.noise_out != nullptr) a.noise_out[(size_t)t * E + e] = nv[u];
+            }
             if (a.bias != nullptr) v = __fadd_rn(v, bv[u]);
-            if (a.noise != nullptr) v = __fadd_rn(v, nv[u]);
+            if (NOISY || a.noise != nullptr) v = __fadd_rn(v, nv[u]);
             if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = v;
           }
           lg[r * S::LGS + e] = v;
@@ -447,10 +578,44 @@ __global__ void __launch_bounds__(TTHREADS, 2)
     csum[threadIdx.x] = v;
   }
   cluster.sync();
-  if (rank == 0 && (int)threadIdx.x < E) {
-    float v = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) v += cluster.map_shared_rank(csum, sp)[threadIdx.x];
-    a.part[(size_t)tile * E + threadIdx.x] = v;
+  if (rank == 0) {
+    if ((int)threadIdx.x < E) {
+      float v = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) v += cluster.map_shared_rank(csum, sp)[threadIdx.x];
+      a.part[(size_t)tile * E + threadIdx.x] = v;
+      __threadfence();
+    }
+    // The last tile to finish turns the rows into P_e = (sum over rows in
+    // fp64) / T: 256 fixed groups (group g of expert e adds rows g, g +
+    // groups, ... in order; then the groups in order), whichever CTA is last.
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const unsigned ntiles = gridDim.x / (unsigned)nsplit;
+      s_last = atomicAdd(a.done, 1u) == ntiles - 1u;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      double* red = reinterpret_cast<double*>(lg);   // no CTA reads lg any more
+      const int nrows = (int)(gridDim.x / (unsigned)nsplit);
+      const int groups = max(1, 256 / E);
+      for (int v = threadIdx.x; v < 256; v += TTHREADS) {
+        const int e = v % E, g = v / E;
+        double acc = 0.0;
+        if (g < groups)
+          for (int b = g; b < nrows; b += groups) acc += (double)__ldcg(a.part + (size_t)b * E + e);
+        red[v] = acc;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < E; e += TTHREADS) {
+        double sum = 0.0;
+        for (int gg = 0; gg < groups; ++gg)
+          if (gg * E + e < 256) sum += red[gg * E + e];
+        a.prob_mean[e] = T > 0 ? (float)(sum / (double)T) : 0.f;
+      }
+      if (threadIdx.x == 0) *a.done = 0u;            // ready for the next launch
+    }
   }
 teardown:
   cluster.sync();  // peers keep their shared memory until every read of it is done
@@ -483,27 +648,37 @@ bool encode_bf16(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* di
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EP, bool LOGITS_ONLY = false>
+// W2: kModeNoisy's second weight matrix (W_noise), split into planes 3-5.
+template <int EP, int MODE>
 cudaError_t run_router_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W,
-                          const TcArgs& a, __nv_bfloat16* w_split, cudaStream_t s, int* tiles_out) {
-  using S = TcShape<EP>;
+                          const float* W2, const TcArgs& a, __nv_bfloat16* w_split,
+                          cudaStream_t s, int* tiles_out) {
+  using S = TcShape<EP, MODE>;
   const int chunks = ceil_div(c.d, TBK);
-  cudaError_t e = launch_kernel(split_router_weights_kernel, chunks, 256, 0, s, 0, W, c.d, c.E,
-                                EP, w_split);
+  // kModeNoisy: a third plane of blocks draws z for every (token, expert)
+  const NoiseDraw nd{const_cast<double*>(a.noise_z), a.seed, a.offset, a.token_base, c.T};
+  const int zblocks = S::NOISY ? (int)std::min<long long>(((long long)c.T * c.E + 255) / 256,
+                                                          (long long)device_sm_count() * 4)
+                               : 0;
+  cudaError_t e = launch_kernel(split_router_weights_kernel,
+                                dim3(std::max(chunks, zblocks), S::TERMS / 3 + (S::NOISY ? 1 : 0)),
+                                256, 0, s, 0, W, W2, c.d, c.E, EP, w_split, nd);
   if (e != cudaSuccess) return e;
   CUtensorMap tx, tw;
   const cuuint64_t xd[2] = {(cuuint64_t)c.d, (cuuint64_t)c.T};
   const cuuint64_t xs[1] = {(cuuint64_t)c.d * 2};
   const cuuint32_t xb[2] = {TBK, TBM};
-  const cuuint64_t wd[3] = {(cuuint64_t)c.d, (cuuint64_t)EP, 3};
+  const cuuint64_t wd[3] = {(cuuint64_t)c.d, (cuuint64_t)EP, (cuuint64_t)S::TERMS};
   const cuuint64_t wstr[2] = {(cuuint64_t)c.d * 2, (cuuint64_t)EP * (cuuint64_t)c.d * 2};
-  const cuuint32_t wb[3] = {TBK, EP, 3};
+  const cuuint32_t wb[3] = {TBK, EP, (cuuint32_t)S::TERMS};
   if (!encode_bf16(&tx, x, 2, xd, xs, xb) || !encode_bf16(&tw, w_split, 3, wd, wstr, wb))
     return cudaErrorInvalidValue;
   const int tiles = ceil_div(c.T, TBM);
+  // the same split for every mode, so that the noisy router sums the logits
+  // in the same order as the plain one
   const int nsplit = tc_splits(tiles, chunks);
   *tiles_out = tiles;
-  auto kern = router_tc_kernel<EP, LOGITS_ONLY>;
+  auto kern = router_tc_kernel<EP, MODE>;
   e = ensure_smem_limit(reinterpret_cast<const void*>(kern), S::SMEM);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, tiles * nsplit, TTHREADS, S::SMEM, s, nsplit, tx, tw, a);
@@ -514,46 +689,41 @@ cudaError_t run_router_tc(const moe_config_t& c, const __nv_bfloat16* x, const f
 cudaError_t launch_route_tc(const moe_config_t& c, const __nv_bfloat16* x, const float* W_router,
                             const float* bias, const float* noise, int32_t* idx, float* gates,
                             float* logits_out, float* router_part, __nv_bfloat16* w_split,
-                            int32_t* err, cudaStream_t s, int* tiles_out) {
+                            int32_t* err, cudaStream_t s, int* tiles_out, float* prob_mean,
+                            unsigned* done) {
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
-  const TcArgs a{bias, noise, idx, gates, logits_out, router_part, err, c.T, c.d, c.E, c.top_k};
+  const TcArgs a{bias, noise, idx, gates, logits_out, router_part, err, c.T, c.d, c.E, c.top_k,
+                 0, 0, 0, nullptr, nullptr, prob_mean, done};
   switch (router_tc_width(c)) {
-    case 16: return run_router_tc<16>(c, x, W_router, a, w_split, s, tiles_out);
-    case 32: return run_router_tc<32>(c, x, W_router, a, w_split, s, tiles_out);
-    case 64: return run_router_tc<64>(c, x, W_router, a, w_split, s, tiles_out);
+    case 16: return run_router_tc<16, kModeRoute>(c, x, W_router, W_router, a, w_split, s, tiles_out);
+    case 32: return run_router_tc<32, kModeRoute>(c, x, W_router, W_router, a, w_split, s, tiles_out);
+    case 64: return run_router_tc<64, kModeRoute>(c, x, W_router, W_router, a, w_split, s, tiles_out);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_route_tc_noisy(const moe_config_t& c, const __nv_bfloat16* x,
+                                  const float* W_router, const float* bias, const float* W_noise,
+                                  uint64_t seed, uint64_t offset, long long token_base,
+                                  int32_t* idx, float* gates, float* logits_out, float* noise_out,
+                                  float* router_part, __nv_bfloat16* w_split, double* noise_z,
+                                  int32_t* err, cudaStream_t s, int* tiles_out, float* prob_mean,
+                                  unsigned* done) {
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  const TcArgs a{bias, nullptr, idx, gates, logits_out, router_part, err, c.T, c.d, c.E, c.top_k,
+                 seed, offset, token_base, noise_out, noise_z, prob_mean, done};
+  switch (router_tc_width(c)) {
+    case 16: return run_router_tc<16, kModeNoisy>(c, x, W_router, W_noise, a, w_split, s, tiles_out);
+    case 32: return run_router_tc<32, kModeNoisy>(c, x, W_router, W_noise, a, w_split, s, tiles_out);
+    case 64: return run_router_tc<64, kModeNoisy>(c, x, W_router, W_noise, a, w_split, s, tiles_out);
     default: return cudaErrorInvalidValue;
   }
 }
 
 namespace {
 
-// Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
-// easy as 1, 2, 3", SC 2011): ten rounds over a 4-word counter, the key
-// advanced by the two Weyl constants between rounds.
-__device__ __forceinline__ void philox4x64_10(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
-  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
-  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += W0;
-      k1 += W1;
-    }
-    const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
-    const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
-    const uint64_t y0 = hi1 ^ x[1] ^ k0, y2 = hi0 ^ x[3] ^ k1;
-    x[0] = y0;
-    x[1] = lo1;
-    x[2] = y2;
-    x[3] = lo0;
-  }
-}
-
-// In place: noise logits l (T, E) -> z(t, e) * softplus(l), z the standard
-// normal of the batch token token_base + t and expert e: Philox4x64-10 of the
-// counter (token, e, offset, 0) under the key (seed, 0), two words to
-// u = ((w >> 11) + 1/2) 2^-53 and z = sqrt(-2 ln u0) cos(2 pi u1) in fp64;
-// softplus(l) = max(l, 0) + log1p(exp(-|l|)) in fp64; one rounding to fp32.
+// In place: noise logits l (T, E) -> z(token_base + t, e) * softplus(l)
+// (gate_noise_value), one thread per element.
 __global__ void __launch_bounds__(256)
     gate_noise_kernel(float* __restrict__ buf, long long n, int E, uint64_t seed, uint64_t offset,
                       long long token_base) {
@@ -562,14 +732,7 @@ __global__ void __launch_bounds__(256)
        i += (long long)gridDim.x * blockDim.x) {
     const long long t = i / E;
     const int e = (int)(i - t * E);
-    uint64_t w[4] = {(uint64_t)(t + token_base), (uint64_t)e, offset, 0ull};
-    philox4x64_10(w, seed, 0ull);
-    const double u0 = ((double)(w[0] >> 11) + 0.5) * 0x1.0p-53;
-    const double u1 = ((double)(w[1] >> 11) + 0.5) * 0x1.0p-53;
-    const double z = sqrt(-2.0 * log(u0)) * cos(2.0 * 3.141592653589793 * u1);
-    const double l = (double)buf[i];
-    const double sp = fmax(l, 0.0) + log1p(exp(-fabs(l)));
-    buf[i] = (float)(z * sp);
+    buf[i] = gate_noise_value(seed, offset, t + token_base, e, buf[i]);
   }
 }
 
@@ -582,13 +745,13 @@ cudaError_t launch_gate_noise(const moe_config_t& c, const __nv_bfloat16* x, con
   if (c.T == 0) return cudaSuccess;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const TcArgs a{nullptr, nullptr, nullptr, nullptr, noise_out, nullptr, err, c.T, c.d, c.E,
-                 c.top_k};
+                 c.top_k, 0, 0, 0, nullptr, nullptr, nullptr, nullptr};
   int tiles = 0;
   cudaError_t e;
   switch (router_tc_width(c)) {
-    case 16: e = run_router_tc<16, true>(c, x, W_noise, a, w_split, s, &tiles); break;
-    case 32: e = run_router_tc<32, true>(c, x, W_noise, a, w_split, s, &tiles); break;
-    case 64: e = run_router_tc<64, true>(c, x, W_noise, a, w_split, s, &tiles); break;
+    case 16: e = run_router_tc<16, kModeLogits>(c, x, W_noise, W_noise, a, w_split, s, &tiles); break;
+    case 32: e = run_router_tc<32, kModeLogits>(c, x, W_noise, W_noise, a, w_split, s, &tiles); break;
+    case 64: e = run_router_tc<64, kModeLogits>(c, x, W_noise, W_noise, a, w_split, s, &tiles); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 23
+    assert len(names) == 24
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -121,12 +121,13 @@ def test_row_tensors_must_be_16_byte_aligned(moe_lib):
 
 
 def test_workspace_holds_the_split_router_weights(moe_lib):
-    """bf16 with E <= 64 adds 3 * EP * d bf16 for the tensor-core router."""
+    """bf16 with E <= 64 adds 6 * EP * d bf16 for the tensor-core router
+    (W_router's three terms, and W_noise's for the fused noisy router)."""
     a = api.make_config(64, 4096, 128, 64, 8, 2, "swiglu", "bf16")
     b = api.make_config(64, 4096, 128, 64, 100, 2, "swiglu", "bf16")   # E > 64: SIMT router
     c = api.make_config(64, 4096, 128, 64, 16, 2, "swiglu", "bf16")
     na, nb, nc = (moe_lib.moe_workspace_size(ctypes.byref(x)) for x in (a, b, c))
-    assert na >= 3 * 16 * 4096 * 2 and nc >= 3 * 16 * 4096 * 2
+    assert na >= 6 * 16 * 4096 * 2 and nc >= 6 * 16 * 4096 * 2
     assert nb > 0
 
 
@@ -173,6 +174,14 @@ def test_gate_noise_argument_checks(moe_lib):
     ws2 = moe_lib.moe_workspace_size(ctypes.byref(wide))
     assert moe_lib.moe_gate_noise(ctypes.byref(wide), FAKE, FAKE, 1, 0, 0, FAKE, FAKE, ws2,
                                   None) == api.MOE_ERR_UNSUPPORTED
+    # the fused noisy router: same limits, W_noise required
+    outs = [FAKE, FAKE, FAKE, None, None]   # indices, gates, P, logits_out, noise_out
+    assert moe_lib.moe_route_noisy(ctypes.byref(wide), FAKE, FAKE, None, FAKE, 1, 0, 0, *outs,
+                                   FAKE, ws2, None) == api.MOE_ERR_UNSUPPORTED
+    assert moe_lib.moe_route_noisy(ctypes.byref(cfg), FAKE, FAKE, None, None, 1, 0, 0, *outs,
+                                   FAKE, ws, None) == api.MOE_ERR_INVALID_ARG
+    assert moe_lib.moe_route_noisy(ctypes.byref(cfg), FAKE, FAKE, None, FAKE, 1, 0, -2, *outs,
+                                   FAKE, ws, None) == api.MOE_ERR_INVALID_ARG
 
 
 def test_backward_argument_checks(moe_lib):
@@ -198,9 +207,9 @@ def test_backward_argument_checks(moe_lib):
 def test_expert_backward_argument_checks(moe_lib):
     cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
     n = moe_lib.moe_expert_backward_workspace_size(ctypes.byref(cfg))
-    # padded rows (T*k + E*127) of Xp, dYp, [A|B], [dA|dB] and H, bf16
+    # padded rows (T*k + E*127) of Xp, dYp, [dA|dB] and H in bf16, [A|B] in fp32
     rows = 64 * 2 + 8 * 127
-    assert n >= rows * (64 + 64 + 2 * 128 + 2 * 128 + 128) * 2 and n % 256 == 0
+    assert n >= rows * ((64 + 64 + 2 * 128 + 128) * 2 + 2 * 128 * 4) and n % 256 == 0
     lin = api.make_config(64, 32, 0, 32, 8, 2, "linear", "f32")
     assert 0 < moe_lib.moe_expert_backward_workspace_size(ctypes.byref(lin)) < n
     ins = [FAKE] * 6                          # x_perm, offsets, W_in, W_up, W_out, dy_perm

