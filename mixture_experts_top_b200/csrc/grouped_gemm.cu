@@ -511,98 +511,17 @@ constexpr int kTileQ = 4;                         // tile indices published ahea
 constexpr int kTileQConsumers = 1 + 1 + 4 + 4;
 constexpr int P_STAGES = 6;
 constexpr int P_STAGE_BYTES = A_STAGE + B_STAGE / 2;  // 32 KiB
-constexpr int kTailBox = 32;                      // token rows per TMA box of a tail tile
-constexpr int kSwapMaxRows = PBM - 1;             // tail tiles of at most this many rows swap
-constexpr int kXbufStride = 33;                   // floats per column in the exchange buffer
-constexpr int P_XBUF_BYTES = 64 * kXbufStride * 4;   // SwiGLU tail: 64 columns x 32 tokens
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES + P_XBUF_BYTES;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES;
 constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
-// A tail tile's instruction: A = the weights, MN-major (bit 15), B = the
-// tokens, K-major (bit 16 = 0), N = the tile's rows rounded up to 16.
-__device__ __forceinline__ uint32_t idesc_pair_swap(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
-}
-__device__ __forceinline__ int tail_n(int rows) { return (rows + 15) & ~15; }
-
-__device__ __forceinline__ void epilogue_bar_sync() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps
-}
-
-// Epilogue of a tail tile (operands swapped): TMEM lane (q*32 + lane) of
-// this CTA is one output column, TMEM column j is token row m0 + j.  The
-// values are those of the normal tile, only transposed: column `col` of
-// grouped row m0 + j.  SwiGLU: this CTA's lanes 0-63 hold gate columns and
-// lanes 64-127 the matching up columns, which warps q = 2, 3 hand to warps
-// q = 0, 1 through shared memory.
-template <int EPI>
-__device__ __forceinline__ void store_tail_tile(uint32_t tacc, const TileCoord& c, int n0,
-                                                int rank, int q, int lane, float* xbuf,
-                                                const GemmArgs& g) {
-  const int nt = tail_n(c.rows);
-#pragma unroll 1
-  for (int j0 = 0; j0 < nt; j0 += 32) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(tacc + (uint32_t)j0, r);
-    tmem_ld_wait();
-    const int nvalid = min(32, c.rows - j0);
-    if (EPI == kEpiSwiglu) {
-      if (q >= 2) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) xbuf[((q - 2) * 32 + lane) * kXbufStride + i] = __uint_as_float(r[i]);
-      }
-      epilogue_bar_sync();
-      if (q < 2) {
-        const int col = n0 + 64 * rank + q * 32 + lane;
-        if (col < g.N) {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nvalid) {
-              const float gv = __uint_as_float(r[i]);
-              const float uv = xbuf[(q * 32 + lane) * kXbufStride + i];
-              out[(size_t)(c.m0 + j0 + i) * g.N + col] = __float2bfloat16_rn(silu_f(gv) * uv);
-            }
-          }
-        }
-      }
-      epilogue_bar_sync();
-    } else {
-      const int col = n0 + 128 * rank + q * 32 + lane;
-      if (col < g.N) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i >= nvalid) break;
-          const float v = __uint_as_float(r[i]);
-          const size_t m = (size_t)(c.m0 + j0 + i);
-          if (EPI == kEpiNone) {
-            static_cast<float*>(g.out)[m * g.N + col] = v;
-          } else if (EPI == kEpiRelu) {
-            static_cast<__nv_bfloat16*>(g.out)[m * g.N + col] = __float2bfloat16_rn(fmaxf(v, 0.f));
-          } else {   // kEpiScatter
-            const int tok = g.rows[m];
-            if (tok >= 0 && tok < g.T)
-              static_cast<__nv_bfloat16*>(g.out)[(size_t)tok * g.N + col] =
-                  __float2bfloat16_rn(g.gates[tok] * v);
-          }
-        }
-      }
-    }
-  }
-}
 
 template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB0,
-                             const __grid_constant__ CUtensorMap tmB1,
-                             const __grid_constant__ CUtensorMap tmAt, const GemmArgs g) {
+                             const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
   pdl_wait_and_release();
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
-  // An expert's last row block with fewer than 256 rows runs as a tail tile
-  // (operands swapped, N = its rows): no MMA work on padding rows.
-  constexpr bool SWAP = !GATHER;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -617,7 +536,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int* tile_q = reinterpret_cast<int*>(tmem_holder + 4);         // kTileQ
   int* tile_prefix = tile_q + kTileQ;                            // MAX_E + 1
   int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
-  float* xbuf = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES + AUX_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E;
@@ -649,7 +567,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_map(&tmA);
       tma_prefetch_map(&tmB0);
       tma_prefetch_map(&tmB1);
-      if (SWAP) tma_prefetch_map(&tmAt);
     }
   } else if (warp == 1) {
     tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -730,13 +647,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // this CTA's B half: gate / up for SwiGLU, else the column halves
       const int nb = (EPI == kEpiSwiglu) ? n0 : n0 + (int)rank * (BN / 2);
       const int my_m = c.m0 + (int)rank * BM;
-      // tail tile: this CTA's half of the tokens in 32-row boxes, and its 128
-      // weight columns (SwiGLU: 64 gate and the matching 64 up columns)
-      const bool swap = SWAP && c.rows <= kSwapMaxRows;
-      const int half = tail_n(c.rows) / 2;
-      const int nbox = swap ? (half + kTailBox - 1) / kTailBox : 0;
-      const uint32_t cta_bytes =
-          swap ? (uint32_t)(2 * B_BOX + nbox * kTailBox * BK * 2) : (uint32_t)P_STAGE_BYTES;
       int r4[4] = {0, 0, 0, 0};
       if (GATHER) {
 #pragma unroll
@@ -760,24 +670,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) {
             report_error(g.err, kDevTimeoutProducer);
           } else {
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * cta_bytes);
-            if (swap) {
-              for (int j = 0; j < nbox; ++j)
-                tma_load_2d_pair(sa + j * kTailBox * BK * 2, &tmAt, &full_bar[stage], k0,
-                                 c.m0 + (int)rank * half + j * kTailBox, pol_a);
-              if (EPI == kEpiSwiglu) {
-                tma_load_3d_pair(sb, &tmB0, &full_bar[stage], n0 + 64 * (int)rank, k0, c.e, pol_b);
-                tma_load_3d_pair(sb + B_BOX, &tmB1, &full_bar[stage], n0 + 64 * (int)rank, k0, c.e,
-                                 pol_b);
-              } else {
-                tma_load_3d_pair(sb, &tmB0, &full_bar[stage], nb, k0, c.e, pol_b);
-                tma_load_3d_pair(sb + B_BOX, &tmB0, &full_bar[stage], nb + 64, k0, c.e, pol_b);
-              }
-            } else {
-              if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, pol_a);
-              tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, pol_b);
-              tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, pol_b);
-            }
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
+            if (!GATHER) tma_load_2d_pair(sa, &tmA, &full_bar[stage], k0, my_m, pol_a);
+            tma_load_3d_pair(sb, bmap, &full_bar[stage], nb, k0, c.e, pol_b);
+            tma_load_3d_pair(sb + B_BOX, bmap, &full_bar[stage], nb + 64, k0, c.e, pol_b);
             issued_mask |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
           }
@@ -825,9 +721,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-      const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
-      const bool swap = SWAP && c.rows <= kSwapMaxRows;
-      const uint32_t idesc_swap = idesc_pair_swap(tail_n(c.rows));
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase)) {
           report_error(g.err, kDevTimeoutMma);
@@ -837,20 +730,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after_sync();
         const uint32_t sa = smem_u32(smem + stage * P_STAGE_BYTES);
         const uint32_t sb = sa + A_STAGE;
-        if (swap) {
-          // A = the weights (MN-major boxes at sb), B = the tokens (K-major at sa)
 #pragma unroll
-          for (int kk = 0; kk < BK / UK; ++kk)
-            umma_bf16_ss_pair(d_tmem, desc_b_nmajor(sb + kk * UK * 128),
-                              desc_a_kmajor(sa + kk * UK * 2), idesc_swap,
-                              (kb | kk) != 0 ? 1u : 0u);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < BK / UK; ++kk)
-            umma_bf16_ss_pair(d_tmem, desc_a_kmajor(sa + kk * UK * 2),
-                              desc_b_nmajor(sb + kk * UK * 128), kIdescPair,
-                              (kb | kk) != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BK / UK; ++kk)
+          umma_bf16_ss_pair(d_tmem, desc_a_kmajor(sa + kk * UK * 2),
+                            desc_b_nmajor(sb + kk * UK * 128), kIdescPair,
+                            (kb | kk) != 0 ? 1u : 0u);
         umma_commit_pair(&empty_bar[stage], 0x3);  // frees the stage in both CTAs
         if (++stage == P_STAGES) {
           stage = 0;
@@ -889,14 +773,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      if (SWAP && c.rows <= kSwapMaxRows) {
-        store_tail_tile<EPI>(tacc, c, n0, (int)rank, q, lane, xbuf, g);
-      } else {
-        const bool valid = row < c.rows;
-        const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
-                                                   : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
-        store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
-      }
+      const bool valid = row < c.rows;
+      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
+                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
@@ -961,11 +841,11 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 
 template <int EPI, bool GATHER>
 cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                          const CUtensorMap& at, const GemmArgs& g, int pairs, cudaStream_t s) {
+                          const GemmArgs& g, int pairs, cudaStream_t s) {
   auto kern = grouped_gemm_pair_kernel<EPI, GATHER>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), P_SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, at, g);
+  return launch_kernel(kern, 2 * pairs, NUM_THREADS, P_SMEM_BYTES, s, 2, a, b0, b1, g);
 }
 
 }  // namespace
@@ -1022,18 +902,14 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
     if (sched == nullptr) return cudaErrorInvalidValue;
     const long max_pairs = (long)(ceil_div(rows_max, PBM) + E) * g.n_tiles;
     const int pairs = (int)std::min<long>((long)(device_sm_count() / 2), max_pairs);
-    // tail tiles' token rows: the same rows, 32-row boxes
-    CUtensorMap tat;
-    if (!(gather ? encode_a(&tat, A, a_rows, K, 1) : encode_a(&tat, A, rows_max, K, kTailBox)))
-      return cudaErrorInvalidValue;
     if (gather)
-      return epi == kEpiSwiglu ? run_gemm_pair<kEpiSwiglu, true>(ta, tb0, tb1, tat, g, pairs, s)
-                               : run_gemm_pair<kEpiRelu, true>(ta, tb0, tb1, tat, g, pairs, s);
+      return epi == kEpiSwiglu ? run_gemm_pair<kEpiSwiglu, true>(ta, tb0, tb1, g, pairs, s)
+                               : run_gemm_pair<kEpiRelu, true>(ta, tb0, tb1, g, pairs, s);
     switch (epi) {
-      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, tat, g, pairs, s);
-      case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, tat, g, pairs, s);
-      case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, tat, g, pairs, s);
-      default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, tat, g, pairs, s);
+      case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, g, pairs, s);
+      default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, g, pairs, s);
     }
   }
   const long max_tiles = (long)(ceil_div(rows_max, BM) + E) * g.n_tiles;
