@@ -29,7 +29,8 @@
 //    d contiguous (a K-major operand), rows E..EP-1 zero; EP = E padded to
 //    16, 32 or 64 (the MMA's N).
 //  * A thread-block cluster of S CTAs (S = 1..8) owns a tile of 128 tokens;
-//    CTA r of the cluster takes 1/S of the contraction range d.  192 threads:
+//    CTA r of the cluster takes every S-th 64-wide block of d, from block r
+//    (the cluster reads runs of S * 128 bytes of each token row).  192 threads:
 //    warp 0 lane 0 issues TMA copies (x box 64 (d) x 128 (tokens) and the
 //    three W boxes 64 (d) x EP, 128-byte swizzle) into a ring of stages;
 //    warp 1 lane 0 issues, per 64-wide d block, 4 tcgen05.mma M128 x N x K16
@@ -45,12 +46,14 @@
 //    [r 128/S, (r+1) 128/S) of the tile.  All its threads add the S partial
 //    logit rows in rank order through distributed shared memory, then the
 //    bias and the noise (coalesced, consecutive experts on consecutive
-//    threads); then a group of EP/8 lanes per token (8 experts a lane): top-k
-//    by k rounds of a group-wide maximum of 64-bit keys (order-preserving
-//    logit bits, then the complemented expert index, so the lower index wins
-//    ties), the softmax (its maximum is the first top-k logit) and the gates.  Each CTA then adds its tokens' probabilities per
-//    expert in token order, and rank 0 adds the S sums in rank order into the
-//    tile's row of column sums (the fp64 mean over rows is router.cu's).
+//    threads); then a group of EP/8 lanes per token (8 experts a lane): each
+//    lane sorts its 64-bit keys (order-preserving logit bits, then the
+//    complemented expert index, so the lower index wins ties) once, top-k
+//    takes k rounds of a group-wide maximum of the lanes' first keys, then
+//    the softmax (its maximum is the first top-k logit) and the gates.  Each
+//    CTA then adds its tokens' probabilities per expert in token order, and
+//    rank 0 adds the S sums in rank order into the tile's row of column sums;
+//    the last tile to finish reduces the rows to P in fp64.
 //  * Every mbarrier wait is bounded; on expiry the error word is set, the
 //    copies in flight are drained and tensor memory is freed.
 #include <cooperative_groups.h>
@@ -69,6 +72,7 @@ constexpr int TUK = 16;        // d per tcgen05.mma (kind::f16)
 constexpr int TTHREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 accumulate and finish
 constexpr int kCoopBatch = 8;  // elements per thread per round of the logit pass
 constexpr int kMaxTopK = 8;    // largest top_k the library accepts
+constexpr int kSplitLoads = TBK * 64 / 256;  // W loads per thread of the split (E <= 64)
 
 // kModeRoute: the router.  kModeLogits: the contraction and the rank-ordered
 // sum only, written to logits_out (the noisy gate's noise logits).
@@ -193,6 +197,23 @@ __device__ __forceinline__ float gate_noise_value(uint64_t seed, uint64_t offset
   return gate_noise_from_z(gate_noise_z(seed, offset, t, e), l);
 }
 
+// Sorts 8 keys into descending order: a 19-comparator, depth-6 network
+// (checked on all 256 zero-one inputs, which by the zero-one principle
+// covers every input).
+__device__ __forceinline__ void cmpx_desc(uint64_t& a, uint64_t& b) {
+  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+__device__ __forceinline__ void sort8_desc(uint64_t (&v)[8]) {
+  cmpx_desc(v[0], v[2]); cmpx_desc(v[1], v[3]); cmpx_desc(v[4], v[6]); cmpx_desc(v[5], v[7]);
+  cmpx_desc(v[0], v[4]); cmpx_desc(v[1], v[5]); cmpx_desc(v[2], v[6]); cmpx_desc(v[3], v[7]);
+  cmpx_desc(v[0], v[1]); cmpx_desc(v[2], v[3]); cmpx_desc(v[4], v[5]); cmpx_desc(v[6], v[7]);
+  cmpx_desc(v[2], v[4]); cmpx_desc(v[3], v[5]);
+  cmpx_desc(v[1], v[4]); cmpx_desc(v[3], v[6]);
+  cmpx_desc(v[1], v[2]); cmpx_desc(v[3], v[4]); cmpx_desc(v[5], v[6]);
+}
+
 // (d, E) fp32 -> (3, EP, d) bf16 terms hi, mid, lo with w = hi + mid + lo.
 // One block per 64 rows of d, transposed through shared memory; blockIdx.y
 // = 1 splits W2 into the next three planes.
@@ -224,9 +245,25 @@ __global__ void __launch_bounds__(256)
   const float* __restrict__ W = blockIdx.y == 0 ? W1 : W2;
   __nv_bfloat16* __restrict__ out = out_base + (size_t)blockIdx.y * 3 * EP * d;
   const int k0 = blockIdx.x * TBK;
-  for (int i = threadIdx.x; i < TBK * E; i += blockDim.x) {
-    const int kk = i / E, e = i - kk * E;
-    tile[kk][e] = (k0 + kk < d) ? W[(size_t)(k0 + kk) * E + e] : 0.f;
+  // The block's 64 rows of W are contiguous: up to 16 loads per thread, all
+  // issued before the first is used, so their latencies overlap.
+  {
+    const float* __restrict__ src = W + (size_t)k0 * E;
+    const int n = min(TBK, d - k0) * E;
+    float v[kSplitLoads];
+#pragma unroll
+    for (int j = 0; j < kSplitLoads; ++j) {
+      const int i = threadIdx.x + j * 256;
+      v[j] = i < n ? __ldg(src + i) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kSplitLoads; ++j) {
+      const int i = threadIdx.x + j * 256;
+      if (i < TBK * E) {
+        const int kk = i / E;
+        tile[kk][i - kk * E] = v[j];
+      }
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < EP * TBK; i += blockDim.x) {
@@ -248,7 +285,6 @@ template <int EP, int MODE>
 __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const TcArgs a) {
-  pdl_wait_and_release();
   using S = TcShape<EP, MODE>;
   constexpr bool LOGITS_ONLY = MODE == kModeLogits;
   constexpr bool NOISY = MODE == kModeNoisy;
@@ -272,9 +308,11 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
   const int tile = blockIdx.x / nsplit;
   const int t_base = tile * TBM;
   const int total_chunks = (a.d + TBK - 1) / TBK;
-  const int per = (total_chunks + nsplit - 1) / nsplit;
-  const int c_begin = min(rank * per, total_chunks);
-  const int nchunks = min(per, total_chunks - c_begin);
+  // CTA r takes the 64-wide d blocks r, r + S, r + 2S, ...: the S CTAs of a
+  // tile read neighbouring 128-byte pieces of the same token rows at about
+  // the same time, so HBM sees runs of S * 128 bytes instead of scattered
+  // 128-byte reads.
+  const int nchunks = rank < total_chunks ? (total_chunks - rank + nsplit - 1) / nsplit : 0;
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmX);
@@ -298,6 +336,9 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  // The set-up above reads no input, so it overlaps the previous kernel's
+  // tail; every read of x, W and the outputs' buffers comes after this.
+  pdl_wait_and_release();
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -309,7 +350,7 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
         break;
       }
       uint8_t* sx = smem + stage * S::STAGE;
-      const int k0 = (c_begin + c) * TBK;
+      const int k0 = (rank + c * nsplit) * TBK;
       mbar_arrive_expect_tx(&full_bar[stage], S::STAGE);
       tma_load_2d(sx, &tmX, &full_bar[stage], k0, t_base);
       tma_load_3d(sx + S::X_BYTES, &tmW, &full_bar[stage], k0, 0, 0);
@@ -485,13 +526,15 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
 
   if (LOGITS_ONLY) goto teardown;
   // ------------------------------ finishing, a group of G lanes per token
-  // Each lane of a group holds 8 consecutive experts' logits.  Top-k: k
-  // rounds of a group-wide maximum of 64-bit keys (order-preserving logit
-  // bits, then the complemented expert index, so the lower index wins ties;
-  // -0 and +0 are one key); the lane that holds the winner zeroes its key.
-  // Softmax: the maximum is the first top-k logit; the exponentials are
-  // summed per lane, then over the group.  The probabilities overwrite the
-  // token's logit row, and the group's first lane writes indices and gates.
+  // Each lane of a group holds 8 consecutive experts' logits as 64-bit keys
+  // (order-preserving logit bits, then the complemented expert index, so the
+  // lower index wins ties; -0 and +0 are one key; absent experts are 0),
+  // sorted once in descending order by a 19-comparator network.  Top-k: k
+  // rounds of a group-wide maximum of the lanes' first keys; the lane that
+  // held the winner drops it.  Softmax: the maximum is the first top-k
+  // logit; the exponentials are summed per lane, then over the group, and
+  // scaled by the sum's reciprocal.  The probabilities overwrite the token's
+  // logit row, and the group's first lane writes indices and gates.
   {
     constexpr int G = S::FG;                         // lanes per token
     const int lane_in = lane & (G - 1);
@@ -512,7 +555,6 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
         L[4] = v1.x; L[5] = v1.y; L[6] = v1.z; L[7] = v1.w;
       }
       const int e0 = lane_in * 8;
-      // The 8 keys of this lane, made once; a taken expert's key becomes 0.
       uint64_t key[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -520,6 +562,7 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
         key[q] = e < E ? ((uint64_t)ordered_key(L[q]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e)
                        : 0ull;
       }
+      sort8_desc(key);
       float vals[kMaxTopK];
       int ids[kMaxTopK];
 #pragma unroll
@@ -529,14 +572,14 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
         if (j < k) {
           uint64_t best = key[0];
 #pragma unroll
-          for (int q = 1; q < 8; ++q) best = key[q] > best ? key[q] : best;
-#pragma unroll
           for (int o = 1; o < G; o <<= 1) {
             const uint64_t other = __shfl_xor_sync(gmask, best, o);
             best = other > best ? other : best;
           }
+          const bool pop = key[0] == best;   // keys are distinct but for absent experts
 #pragma unroll
-          for (int q = 0; q < 8; ++q) key[q] = key[q] == best ? 0ull : key[q];
+          for (int q = 0; q < 7; ++q) key[q] = pop ? key[q + 1] : key[q];
+          key[7] = pop ? 0ull : key[7];
           const uint32_t kb = (uint32_t)(best >> 32);
           vals[j] = __uint_as_float((kb & 0x80000000u) ? (kb & 0x7FFFFFFFu) : ~kb);
           ids[j] = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
@@ -549,9 +592,10 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
       float sum = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
 #pragma unroll
       for (int o = 1; o < G; o <<= 1) sum += __shfl_xor_sync(gmask, sum, o);
-      *reinterpret_cast<float4*>(row) = make_float4(p[0] / sum, p[1] / sum, p[2] / sum, p[3] / sum);
+      const float inv = __frcp_rn(sum);
+      *reinterpret_cast<float4*>(row) = make_float4(p[0] * inv, p[1] * inv, p[2] * inv, p[3] * inv);
       *reinterpret_cast<float4*>(row + 4) =
-          make_float4(p[4] / sum, p[5] / sum, p[6] / sum, p[7] / sum);
+          make_float4(p[4] * inv, p[5] * inv, p[6] * inv, p[7] * inv);
       if (lane_in == 0) {
         float ex[kMaxTopK];
         float sk = 0.f;
@@ -560,11 +604,12 @@ __global__ void __launch_bounds__(TTHREADS, TcShape<EP, MODE>::CTAS_PER_SM)
           ex[j] = j < k ? expf(vals[j] - vals[0]) : 0.f;
           sk += ex[j];
         }
+        const float skinv = __frcp_rn(sk);
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j)
           if (j < k) {
             a.idx[(size_t)t * k + j] = ids[j];
-            a.gates[(size_t)t * k + j] = ex[j] / sk;
+            a.gates[(size_t)t * k + j] = ex[j] * skinv;
           }
       }
     }
