@@ -450,7 +450,7 @@ int moe_route_backward(const moe_config_t* cfg, const void* x, const float* W_ro
  *           NULL where the weight is NULL; every expert's block is written
  *           (zeros for an expert without rows)
  * bf16 experts run on the tensor cores (bf16 operands, fp32 accumulation):
- * the rows are copied into a layout padded to 128 rows per expert, dY is
+ * the rows are copied into a layout padded to 64 rows per expert, dY is
  * rounded to bf16, the forward's A and B are recomputed and kept in fp32,
  * dA, dB and H are rounded to bf16 between the GEMMs.  Linear experts run
  * in fp32.  Deterministic: no atomics, fixed summation orders. */

@@ -12,7 +12,7 @@
 // shards: an idle expert learns nothing).
 //
 //   pack            - padded layout for the bf16 GEMMs: expert e's rows start
-//                     at p_e = sum over e' < e of ceil(rows_e' / 128) * 128;
+//                     at p_e = sum over e' < e of ceil(rows_e' / 64) * 64;
 //                     Xp = x_perm rows, dYp = dy_perm rows rounded to bf16,
 //                     zero rows after each expert's rows
 //   linear backward - fp32 experts (x @ W): dx_perm = dy_perm W_e^T and

@@ -205,7 +205,7 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
 // Experts' backward (expert_backward.cu, grouped_gemm_bwd.cu).  The bf16
 // GEMMs work on a padded grouped layout: each expert's rows rounded up to a
 // multiple of kBwdPadRows, zero rows after its own.
-constexpr int kBwdPadRows = 128;
+constexpr int kBwdPadRows = 64;
 // Rows of the padded layout for at most rows_max grouped rows.
 int expert_backward_pad_rows(int rows_max, int E);
 // Workspace of moe_expert_ffn_backward: error word; padded rows Xp (bf16),

@@ -207,8 +207,8 @@ def test_backward_argument_checks(moe_lib):
 def test_expert_backward_argument_checks(moe_lib):
     cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
     n = moe_lib.moe_expert_backward_workspace_size(ctypes.byref(cfg))
-    # padded rows (T*k + E*127) of Xp, dYp, [dA|dB] and H in bf16, [A|B] in fp32
-    rows = 64 * 2 + 8 * 127
+    # padded rows (T*k + E*63) of Xp, dYp, [dA|dB] and H in bf16, [A|B] in fp32
+    rows = 64 * 2 + 8 * 63
     assert n >= rows * ((64 + 64 + 2 * 128 + 128) * 2 + 2 * 128 * 4) and n % 256 == 0
     lin = api.make_config(64, 32, 0, 32, 8, 2, "linear", "f32")
     assert 0 < moe_lib.moe_expert_backward_workspace_size(ctypes.byref(lin)) < n

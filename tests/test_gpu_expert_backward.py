@@ -44,7 +44,7 @@ CASES = {
     "switch_relu": WORKLOADS["switch_relu"].replace(T=1024, d=256, d_hidden=512, d_out=256),
     "tiny_linear": WORKLOADS["tiny_linear"],
     # d and d_out not multiples of the 256-column tile, rows of one expert
-    # spanning several 128-row tiles
+    # spanning several 256-row tiles
     "ragged": WORKLOADS["mixtral"].replace(T=700, d=200, d_hidden=136, d_out=72, E=5, top_k=2),
 }
 
