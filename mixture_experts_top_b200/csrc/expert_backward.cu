@@ -211,7 +211,9 @@ ExpertBwdLayout expert_backward_layout(const moe_config_t& c) {
     const size_t wide = (c.expert_kind == MOE_EXPERT_SWIGLU ? 2 : 1) * DHp;
     L.xp = take(Rp * (size_t)c.d * 2);
     L.dyp = take(Rp * (size_t)c.d_out * 2);
-    L.pre = take(Rp * wide * 4);
+    // pre-activations in blocks of kBwdPreBlock hidden units (grouped_gemm_bwd.cu)
+    const size_t pre_cols = (size_t)ceil_div(c.d_hidden, kBwdPreBlock) * kBwdPreBlock;
+    L.pre = take(Rp * (c.expert_kind == MOE_EXPERT_SWIGLU ? 2 : 1) * pre_cols * 4);
     L.dab = take(Rp * wide * 2);
     L.hid = take(Rp * DHp * 2);
   }

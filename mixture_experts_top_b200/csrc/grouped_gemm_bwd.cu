@@ -26,7 +26,9 @@
 // other operand on N, so that the epilogue's lanes run along the weight
 // dimension and every global access of a warp is one contiguous run:
 //   kPre   M = hidden units of W_in, then of W_up; N = the expert's rows;
-//          K = d.  pre^T = [W_in | W_up]^T Xp^T, stored fp32 as [A | B] per row
+//          K = d.  pre^T = [W_in | W_up]^T Xp^T, stored fp32 in blocks of 256
+//          hidden units (each block's rows one after another), the tiles dH
+//          reads back
 //   kDH    M = hidden units; N = rows; K = d_out.  dH^T = W_out dYp^T; the
 //          epilogue reads the rows' pre-activations and writes dAB = [dA | dB]
 //          and H (bf16)
@@ -45,7 +47,9 @@
 // B200 design as in grouped_gemm.cu's pair kernel: persistent, one CTA pair
 // per two SMs, warp 0 TMA producer (each CTA loads its 128 weight rows and
 // its half of the N operand), warp 1 of the leader issues the pair MMAs and
-// owns tensor memory, warps 2-5 of both CTAs are the epilogue; 6 stages of
+// owns tensor memory, warps 2-9 of both CTAs are the epilogue (two per
+// tensor-memory lane quarter, each on half of the tile's columns; warps 2-5
+// for kWgrad); 6 stages of
 // 32 KiB (5 for kWgrad, whose epilogue stages its output in shared memory),
 // two 256-column accumulators; every wait bounded (the error word records a
 // timeout, copies and MMAs are drained and tensor memory is freed).
@@ -59,6 +63,7 @@ namespace {
 
 constexpr int BM = 128;                        // weight rows per CTA
 constexpr int PM = 2 * BM;                     // weight rows per pair tile (UMMA M)
+static_assert(PM == kBwdPreBlock, "the stored pre-activations are blocked by the pair tile");
 constexpr int BK = 64;
 constexpr int BN = 256;                        // tile columns, at most (UMMA N)
 constexpr int UK = 16;
@@ -66,7 +71,6 @@ constexpr int A_STAGE = BM * BK * 2;           // 16 KiB: this CTA's weight rows
 constexpr int B_STAGE = (BN / 2) * BK * 2;     // 16 KiB: this CTA's half of N
 constexpr int BOX64 = 64 * BK * 2;             // one 64 x 64 box: 8 KiB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
-constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_E = 256;
 constexpr int AUX_BYTES = 6144;                // barriers, tmem address, offsets, tile table
@@ -79,6 +83,12 @@ template <int STAGE>
 struct Cfg {
   static constexpr int STAGES = STAGE == kWgrad ? 5 : 6;
   static constexpr int OUT = STAGE == kWgrad ? OUT_BYTES : 0;
+  // Epilogue warps per CTA: the row stages use two per tensor-memory lane
+  // quarter, each taking half of the tile's columns, so twice as many of
+  // the epilogue's global accesses are in flight; kWgrad keeps four (its
+  // output boxes take shared memory).
+  static constexpr int EPI_WARPS = STAGE == kWgrad ? 4 : 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int SMEM = STAGES * STAGE_BYTES + OUT + 1024 + AUX_BYTES;
   // Instruction descriptor, kind::f16 (bf16 x bf16 -> fp32), M = 256: D fp32
   // (bit 4), A bf16 (7-9 = 1), B bf16 (10-12 = 1), A major at bit 15 and B
@@ -116,7 +126,9 @@ struct BwdArgs {
   int d, DH, DHp, d_out;    // DHp: DH rounded up to 64
   int m_tiles;              // row stages: M tiles per weight matrix
   int rows_max;             // rows of the unpadded grouped buffers (T * top_k)
-  float* pre;               // (Rp, (1 + swiglu) DHp) fp32: [A | B] pre-activations
+  int Rp;                   // rows of the padded layout
+  float* pre;               // fp32 pre-activations A, B in blocks of 256 hidden units:
+                            // block (p, mt) is (Rp, 256), p = 0 A, 1 B
   __nv_bfloat16* dab;       // (Rp, (1 + swiglu) DHp): [dA | dB]
   __nv_bfloat16* hid;       // (Rp, DHp): H
   float* dx;                // (R, d): unpadded grouped rows
@@ -195,32 +207,33 @@ __device__ __forceinline__ Tile decode(int tile, const int* prefix, const int* p
 // expert at a time; at each of them the warp touches 32 consecutive weight
 // indices of one row.
 template <int STAGE>
-__device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int mrow,
-                                              const int* poff, const int* row_off,
+__device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int mrow, int c_begin,
+                                              int c_end, const int* poff, const int* row_off,
                                               const BwdArgs& g) {
   const int m = t.m0 + mrow;
   const size_t wide = (size_t)(g.swiglu ? 2 : 1) * g.DHp;
   const int prow0 = poff[t.e] + t.n0;    // padded row of the tile's first column
 #pragma unroll 1
-  for (int c0 = 0; c0 < t.n; c0 += 32) {
+  for (int c0 = c_begin; c0 < c_end; c0 += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
     tmem_ld_wait();
     if (STAGE == kPre) {
-      if (m < g.DHp) {
-        float* base = g.pre + (size_t)t.p * g.DHp + m + (size_t)(prow0 + c0) * wide;
+      // the tile's block: its 256 hidden units of every row, one 1 KB run per
+      // row, so the pair's warps write (and dH's read) whole runs in order
+      float* base = g.pre + ((size_t)(t.p * g.m_tiles + t.m0 / PM) * g.Rp + prow0 + c0) * PM + mrow;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) base[(size_t)j * wide] = __uint_as_float(r[j]);
-      }
+      for (int j = 0; j < 32; ++j) base[(size_t)j * PM] = __uint_as_float(r[j]);
     } else if (STAGE == kDH) {
       if (m < g.DHp) {
         const size_t row = (size_t)(prow0 + c0);
-        const float* pa = g.pre + row * wide + m;
+        const float* pa = g.pre + ((size_t)(t.m0 / PM) * g.Rp + row) * PM + mrow;
+        const float* pb = g.pre + ((size_t)(g.m_tiles + t.m0 / PM) * g.Rp + row) * PM + mrow;
         float av[32], bv[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          av[j] = pa[(size_t)j * wide];
-          bv[j] = g.swiglu ? pa[(size_t)j * wide + g.DHp] : 0.f;
+          av[j] = pa[(size_t)j * PM];
+          bv[j] = g.swiglu ? pb[(size_t)j * PM] : 0.f;
         }
         __nv_bfloat16* da = g.dab + row * wide + m;
         __nv_bfloat16* hh = g.hid + row * (size_t)g.DHp + m;
@@ -298,7 +311,7 @@ __device__ __forceinline__ void epilogue_wgrad(uint32_t tacc, const Tile& t, int
 // Tensor maps: A and A1 (kDX: W_up beside W_in; kWgrad: Xp beside H), B and
 // B1 (kWgrad: [dA | dB] beside dYp), O0..O2 (kWgrad: dW_out, dW_in, dW_up).
 template <int STAGE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<STAGE>::THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
@@ -383,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 8);  // one arrive per epilogue warp of both CTAs
+      mbar_init(&tempty_bar[b], 2 * C::EPI_WARPS);  // one arrive per epilogue warp of both CTAs
     }
     mbar_init(drain_bar, 1);
     fence_mbar_init();
@@ -513,7 +526,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue (both)
-    const int q = warp & 3;
+    const int q = warp & 3;                       // tensor-memory lanes 32q .. 32q + 31
+    const int half = (warp - 2) / 4;              // row stages: which half of the columns
     const int mrow = rank * BM + q * 32 + lane;   // weight row inside the pair tile
     uint8_t* my_out = out_stage + q * 2 * OUT_BOX;
     int nbox = 0;
@@ -531,7 +545,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         epilogue_wgrad(tacc, t, rank, q, lane, my_out, nbox,
                        t.p == 0 ? &tmO0 : (t.p == 1 ? &tmO1 : &tmO2));
       else
-        epilogue_rows<STAGE>(tacc, t, mrow, poff, row_off, g);
+        epilogue_rows<STAGE>(tacc, t, mrow, half * (t.n / 2), (half + 1) * (t.n / 2), poff,
+                             row_off, g);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
@@ -597,8 +612,8 @@ cudaError_t run_stage(const CUtensorMap& a, const CUtensorMap& a1, const CUtenso
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), Cfg<STAGE>::SMEM);
   if (e != cudaSuccess) return e;
   const int pairs = (int)std::max(1L, std::min<long>(device_sm_count() / 2, tiles));
-  return launch_kernel(kern, 2 * pairs, NUM_THREADS, Cfg<STAGE>::SMEM, s, 2, a, a1, b, b1, o0, o1,
-                       o2, g);
+  return launch_kernel(kern, 2 * pairs, Cfg<STAGE>::THREADS, Cfg<STAGE>::SMEM, s, 2, a, a1, b, b1,
+                       o0, o1, o2, g);
 }
 
 }  // namespace
@@ -631,6 +646,7 @@ cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* o
   g.DHp = DHp;
   g.d_out = d_out;
   g.rows_max = c.T * c.top_k;
+  g.Rp = Rp;
   g.pre = pre;
   g.dab = dab;
   g.hid = hid;

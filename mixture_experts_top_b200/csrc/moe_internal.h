@@ -206,6 +206,8 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
 // GEMMs work on a padded grouped layout: each expert's rows rounded up to a
 // multiple of kBwdPadRows, zero rows after its own.
 constexpr int kBwdPadRows = 64;
+// Hidden units per block of the backward's stored pre-activations (the M of a pair tile).
+constexpr int kBwdPreBlock = 256;
 // Rows of the padded layout for at most rows_max grouped rows.
 int expert_backward_pad_rows(int rows_max, int E);
 // Workspace of moe_expert_ffn_backward: error word; padded rows Xp (bf16),
