@@ -279,6 +279,141 @@ __global__ void __launch_bounds__(256)
   if (do_bias) dbias_part[(size_t)chunk * E + threadIdx.x] = bacc;
 }
 
+// dx for E <= 16 and d a multiple of 4: a thread owns 4 consecutive columns
+// and keeps their 4 rows of W (4 x E values) in registers; CTA row y walks
+// a contiguous range of tokens, their logit gradients staged 256 tokens at
+// a time in shared memory (read by the whole warp from one address), and
+// writes each token's 4 columns as one 16-byte store, so a warp writes 512
+// contiguous bytes per token.  The arithmetic is route_dx_kernel's: e in
+// increasing order from 0.
+template <int EMAX>
+__global__ void __launch_bounds__(256)
+    route_dx_narrow_kernel(const float* __restrict__ dlogits, const float* __restrict__ W, int T,
+                           int d, int E, float* __restrict__ dx) {
+  pdl_wait_and_release();
+  __shared__ float dls[256 * EMAX];
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  const bool active = c < d;
+  float w[4][EMAX];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) w[i][e] = (active && e < E) ? W[(size_t)(c + i) * E + e] : 0.f;
+  const int t0 = (int)((long long)T * blockIdx.y / gridDim.y);
+  const int t1 = (int)((long long)T * (blockIdx.y + 1) / gridDim.y);
+  for (int tb = t0; tb < t1; tb += 256) {
+    const int n = min(256, t1 - tb);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n * E; i += blockDim.x) dls[i] = dlogits[(size_t)tb * E + i];
+    __syncthreads();
+    if (!active) continue;
+    for (int tt = 0; tt < n; ++tt) {
+      const float* g = dls + tt * E;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (e < E) {
+          const float ge = g[e];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = fmaf(ge, w[i][e], acc[i]);
+        }
+      *reinterpret_cast<float4*>(dx + (size_t)(tb + tt) * d + c) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void load_cols(const __nv_bfloat16* p, float* v, int n) {
+  // n = 4 or 8 consecutive bf16 values (8 or 16 bytes)
+  if (n == 8) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(q.x << 16);
+    v[1] = __uint_as_float(q.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(q.y << 16);
+    v[3] = __uint_as_float(q.y & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load_cols(const float* p, float* v, int n) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  if (n == 8) {
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// Partial dW and dbias over one chunk of tokens for E <= 16 and d a
+// multiple of CPT: a thread owns CPT consecutive columns of x and keeps
+// CPT x E accumulators, reading x straight from global memory (a warp reads
+// 32 * CPT contiguous elements of a row) with kDwAhead tokens' loads in
+// flight; the chunk's logit gradients are staged 256 tokens at a time in
+// shared memory.  The arithmetic is route_dw_partial_kernel's: tokens of the
+// chunk in increasing order, each an fp32 FMA.
+constexpr int kDwAhead = 4;
+template <typename XT, int EMAX, int CPT>
+__global__ void __launch_bounds__(256)
+    route_dw_narrow_kernel(const XT* __restrict__ x, const float* __restrict__ dlogits, int T,
+                           int d, int E, int nchunks, float* __restrict__ dw_part,
+                           float* __restrict__ dbias_part) {
+  pdl_wait_and_release();
+  __shared__ float dls[256 * EMAX];
+  const int chunk = blockIdx.y;
+  const int t0 = (int)((long long)T * chunk / nchunks);
+  const int t1 = (int)((long long)T * (chunk + 1) / nchunks);
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * CPT;
+  const bool active = c < d;
+  const bool do_bias = blockIdx.x == 0 && (int)threadIdx.x < E;
+  float acc[CPT][EMAX];
+#pragma unroll
+  for (int i = 0; i < CPT; ++i)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[i][e] = 0.f;
+  float bacc = 0.f;
+  for (int tb = t0; tb < t1; tb += 256) {
+    const int n = min(256, t1 - tb);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n * E; i += blockDim.x) dls[i] = dlogits[(size_t)tb * E + i];
+    __syncthreads();
+    if (do_bias)
+      for (int tt = 0; tt < n; ++tt) bacc += dls[tt * E + threadIdx.x];
+    if (!active) continue;
+    for (int tt0 = 0; tt0 < n; tt0 += kDwAhead) {
+      float xv[kDwAhead][CPT];
+#pragma unroll
+      for (int u = 0; u < kDwAhead; ++u)
+        if (tt0 + u < n) load_cols(x + (size_t)(tb + tt0 + u) * d + c, xv[u], CPT);
+#pragma unroll
+      for (int u = 0; u < kDwAhead; ++u)
+        if (tt0 + u < n) {
+          const float* g = dls + (tt0 + u) * E;
+#pragma unroll
+          for (int e = 0; e < EMAX; ++e)
+            if (e < E) {
+              const float ge = g[e];
+#pragma unroll
+              for (int i = 0; i < CPT; ++i) acc[i][e] = fmaf(xv[u][i], ge, acc[i][e]);
+            }
+        }
+    }
+  }
+  const long long total = (long long)d * E;
+  if (active)
+#pragma unroll
+    for (int i = 0; i < CPT; ++i)
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (e < E) dw_part[(size_t)chunk * total + (size_t)(c + i) * E + e] = acc[i][e];
+  if (do_bias) dbias_part[(size_t)chunk * E + threadIdx.x] = bacc;
+}
+
 // Chunks added in increasing order.
 __global__ void __launch_bounds__(256)
     route_dw_reduce_kernel(const float* __restrict__ dw_part, const float* __restrict__ dbias_part,
@@ -301,7 +436,13 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-int route_backward_chunks(int T) { return std::max(1, std::min(16, ceil_div(T, 128))); }
+// Token chunks of the dW partial sums: up to 128 of at least 64 tokens where
+// E <= 16 (the narrow kernels: enough CTAs to stream x at HBM rate, and the
+// partials stay small), else up to 16 of at least 128 tokens.
+int route_backward_chunks(int T, int E) {
+  return E <= 16 ? std::max(1, std::min(128, ceil_div(T, 64)))
+                 : std::max(1, std::min(16, ceil_div(T, 128)));
+}
 
 cudaError_t launch_combine_backward(const moe_config_t& c, const void* dy, const float* y_perm,
                                     const int32_t* dest, const float* gates, float* dy_perm,
@@ -335,11 +476,45 @@ cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const fl
                                 dgates, f, daux, c.T, c.E, c.top_k,
                                 (double)c.E / (double)T_batch, dlogits);
   if (e != cudaSuccess) return e;
-  e = launch_kernel(route_dx_kernel,
-                    dim3((unsigned)ceil_div(c.d, 256), (unsigned)std::min(ceil_div(c.T, kTg), 65535)),
-                    256, 0, s, 0, dlogits, W, c.T, c.d, c.E, dx);
+  const bool narrow = c.E <= 16;
+  if (narrow && c.d % 4 == 0) {
+    const dim3 grid((unsigned)ceil_div(c.d, 1024),
+                    (unsigned)std::max(1, std::min(ceil_div(c.T, 16), 2 * device_sm_count())));
+    e = c.E <= 8 ? launch_kernel(route_dx_narrow_kernel<8>, grid, 256, 0, s, 0, dlogits, W, c.T,
+                                 c.d, c.E, dx)
+                 : launch_kernel(route_dx_narrow_kernel<16>, grid, 256, 0, s, 0, dlogits, W, c.T,
+                                 c.d, c.E, dx);
+  } else {
+    e = launch_kernel(route_dx_kernel,
+                      dim3((unsigned)ceil_div(c.d, 256),
+                           (unsigned)std::min(ceil_div(c.T, kTg), 65535)),
+                      256, 0, s, 0, dlogits, W, c.T, c.d, c.E, dx);
+  }
   if (e != cudaSuccess) return e;
-  const int nchunks = route_backward_chunks(c.T);
+  const int nchunks = route_backward_chunks(c.T, c.E);
+  if (narrow && c.d % 8 == 0) {
+    // E <= 8: 8 columns a thread; E <= 16: 4
+    const int cpt = c.E <= 8 ? 8 : 4;
+    const dim3 ngrid((unsigned)ceil_div(c.d, 256 * cpt), (unsigned)nchunks);
+    if (c.act_dtype == MOE_BF16) {
+      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+      e = c.E <= 8 ? launch_kernel(route_dw_narrow_kernel<__nv_bfloat16, 8, 8>, ngrid, 256, 0, s,
+                                   0, xb, dlogits, c.T, c.d, c.E, nchunks, dw_part, dbias_part)
+                   : launch_kernel(route_dw_narrow_kernel<__nv_bfloat16, 16, 4>, ngrid, 256, 0, s,
+                                   0, xb, dlogits, c.T, c.d, c.E, nchunks, dw_part, dbias_part);
+    } else {
+      const float* xf = static_cast<const float*>(x);
+      e = c.E <= 8 ? launch_kernel(route_dw_narrow_kernel<float, 8, 8>, ngrid, 256, 0, s, 0, xf,
+                                   dlogits, c.T, c.d, c.E, nchunks, dw_part, dbias_part)
+                   : launch_kernel(route_dw_narrow_kernel<float, 16, 4>, ngrid, 256, 0, s, 0, xf,
+                                   dlogits, c.T, c.d, c.E, nchunks, dw_part, dbias_part);
+    }
+    if (e != cudaSuccess) return e;
+    const int rblocks =
+        (int)std::min<long long>((total + 255) / 256, (long long)device_sm_count() * 8);
+    return launch_kernel(route_dw_reduce_kernel, rblocks, 256, 0, s, 0, dw_part, dbias_part, total,
+                         c.E, nchunks, dW, dbias);
+  }
   const dim3 grid((unsigned)ceil_div(c.d, kCt), (unsigned)nchunks);
   const size_t dsm = (size_t)kTs * c.E * sizeof(float);
   const int ept = c.E <= 8 ? 2 : c.E <= 16 ? 4 : c.E <= 32 ? 8 : c.E <= 64 ? 16 : c.E <= 128 ? 32 : 64;

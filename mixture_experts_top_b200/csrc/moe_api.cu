@@ -206,7 +206,7 @@ WsLayout workspace_layout(const moe_config_t& c) {
   L.x_perm = take(Tk * (size_t)c.d * s);
   L.hidden = take(c.expert_kind == MOE_EXPERT_LINEAR ? 0 : Tk * (size_t)c.d_hidden * 2);
   L.y_perm = take(Tk * (size_t)c.d_out * 4);
-  const size_t nch = (size_t)route_backward_chunks(c.T);
+  const size_t nch = (size_t)route_backward_chunks(c.T, c.E);
   L.dlogits = take((size_t)c.T * E * 4);
   L.dw_part = take(nch * (size_t)c.d * E * 4);
   L.dbias_part = take(nch * E * 4);

@@ -235,7 +235,7 @@ cudaError_t launch_permute_backward(const moe_config_t& c, const float* dx_perm,
                                     cudaStream_t s);
 
 // Routing backward (backward.cu).
-int route_backward_chunks(int T);
+int route_backward_chunks(int T, int E);
 cudaError_t launch_combine_backward(const moe_config_t& c, const void* dy, const float* y_perm,
                                     const int32_t* dest, const float* gates, float* dy_perm,
                                     float* dgates, cudaStream_t s);
