@@ -397,6 +397,37 @@ class LayerBench:
         self._evs = evs
         return start.elapsed_time(end), sum(e[2].elapsed_time(e[3]) for e in evs) / steps
 
+    def graph_timed(self, steps, warmup):
+        """The same step captured once as a CUDA graph and replayed `steps`
+        times (the host enqueues one graph instead of each launch, which is
+        what bounds the small configurations): device ms for all steps, or
+        (None, reason) where the capture is refused."""
+        import torch
+        try:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                self.step()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.step()
+            for _ in range(warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record()
+            for _ in range(steps):
+                g.replay()
+            end.record()
+            torch.cuda.synchronize()
+            del g
+            return start.elapsed_time(end), None
+        except Exception as exc:   # reported in the line, not raised
+            torch.cuda.synchronize()
+            return None, f"{type(exc).__name__}: {exc}"[:200]
+
     def stage_breakdown(self, steps, barrier):
         """The same steps again with an event between every two stages
         (diagnostic, outside the timed region): mean ms per stage."""
@@ -562,6 +593,7 @@ def extra_workload(name, steps, warmup, peaks, peak_src, base_inputs=None):
     stage_ms = lb.stage_breakdown(steps, sync)
     stage_ms[2] = expert_ms
     e2e_ms, h2d, d2h = lb.e2e(steps, warmup, sync)
+    graph_ms, graph_err = lb.graph_timed(steps, warmup)
     if lb.device_status() != 0:
         raise RuntimeError(f"{name}: device error word set")
     counts = lb.layer.out.counts.cpu().numpy()
@@ -574,6 +606,9 @@ def extra_workload(name, steps, warmup, peaks, peak_src, base_inputs=None):
         "ms_per_step": ms / steps,
         "e2e_tokens_per_s": w.T / (e2e_ms / steps / 1e3),
         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "graph": ({"tokens_per_s": w.T / (graph_ms / steps / 1e3), "ms_per_step": graph_ms / steps,
+                   "note": "the same step captured once as a CUDA graph and replayed"}
+                  if graph_ms is not None else {"unavailable": graph_err}),
         "experts": gemm_roofline(w, rows, used, expert_ms, peaks, peak_src, regime),
         "stages": stage_rooflines(w, rows, stage_ms, peaks["hbm_gbs"]),
         "rows": rows, "used_experts": used,
@@ -644,6 +679,12 @@ def run_ours(args, rank, world):
         return 0
 
     extras = {}
+    if world == 1:
+        graph_ms, graph_err = lb.graph_timed(args.steps, args.warmup)
+        extras["graph"] = ({"tokens_per_s": T / (graph_ms / args.steps / 1e3),
+                            "ms_per_step": graph_ms / args.steps,
+                            "note": "the same step captured once as a CUDA graph and replayed"}
+                           if graph_ms is not None else {"unavailable": graph_err})
     # The noisy gate's noise made on the device (moe_gate_noise), timed on
     # its own: the workload recipe hands the router a host-made noise tensor,
     # so this is not part of the step above.

@@ -294,21 +294,50 @@ __global__ void __launch_bounds__(256)
   __shared__ float dls[256 * EMAX];
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   const bool active = c < d;
+  // this thread's 4 rows of W are 4 E contiguous floats
   float w[4][EMAX];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) w[i][e] = (active && e < E) ? W[(size_t)(c + i) * E + e] : 0.f;
+    for (int e = 0; e < EMAX; ++e) w[i][e] = 0.f;
+  if (active) {
+    const float* src = W + (size_t)c * E;
+    if (E % 4 == 0 && (reinterpret_cast<uintptr_t>(W) & 15u) == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < EMAX / 4; ++q)
+          if (4 * q < E) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(src + i * E) + q);
+            w[i][4 * q] = v.x; w[i][4 * q + 1] = v.y; w[i][4 * q + 2] = v.z; w[i][4 * q + 3] = v.w;
+          }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e < E) w[i][e] = __ldg(src + i * E + e);
+    }
+  }
   const int t0 = (int)((long long)T * blockIdx.y / gridDim.y);
   const int t1 = (int)((long long)T * (blockIdx.y + 1) / gridDim.y);
   for (int tb = t0; tb < t1; tb += 256) {
     const int n = min(256, t1 - tb);
     __syncthreads();
-    for (int i = threadIdx.x; i < n * E; i += blockDim.x) dls[i] = dlogits[(size_t)tb * E + i];
+    // rows padded to EMAX, so a token's gradients are EMAX / 4 aligned vector loads
+    for (int i = threadIdx.x; i < n * EMAX; i += blockDim.x) {
+      const int tt = i / EMAX, e = i % EMAX;
+      dls[i] = e < E ? dlogits[(size_t)(tb + tt) * E + e] : 0.f;
+    }
     __syncthreads();
     if (!active) continue;
     for (int tt = 0; tt < n; ++tt) {
-      const float* g = dls + tt * E;
+      float g[EMAX];
+#pragma unroll
+      for (int q = 0; q < EMAX / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(dls + tt * EMAX)[q];
+        g[4 * q] = v.x; g[4 * q + 1] = v.y; g[4 * q + 2] = v.z; g[4 * q + 3] = v.w;
+      }
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < EMAX; ++e)
@@ -357,7 +386,7 @@ __device__ __forceinline__ void load_cols(const float* p, float* v, int n) {
 // flight; the chunk's logit gradients are staged 256 tokens at a time in
 // shared memory.  The arithmetic is route_dw_partial_kernel's: tokens of the
 // chunk in increasing order, each an fp32 FMA.
-constexpr int kDwAhead = 4;
+constexpr int kDwAhead = 2;
 template <typename XT, int EMAX, int CPT>
 __global__ void __launch_bounds__(256)
     route_dw_narrow_kernel(const XT* __restrict__ x, const float* __restrict__ dlogits, int T,
@@ -380,28 +409,46 @@ __global__ void __launch_bounds__(256)
   for (int tb = t0; tb < t1; tb += 256) {
     const int n = min(256, t1 - tb);
     __syncthreads();
-    for (int i = threadIdx.x; i < n * E; i += blockDim.x) dls[i] = dlogits[(size_t)tb * E + i];
+    // rows padded to EMAX, so a token's gradients are EMAX / 4 aligned vector loads
+    for (int i = threadIdx.x; i < n * EMAX; i += blockDim.x) {
+      const int tt = i / EMAX, e = i % EMAX;
+      dls[i] = e < E ? dlogits[(size_t)(tb + tt) * E + e] : 0.f;
+    }
     __syncthreads();
     if (do_bias)
-      for (int tt = 0; tt < n; ++tt) bacc += dls[tt * E + threadIdx.x];
+      for (int tt = 0; tt < n; ++tt) bacc += dls[tt * EMAX + threadIdx.x];
     if (!active) continue;
-    for (int tt0 = 0; tt0 < n; tt0 += kDwAhead) {
-      float xv[kDwAhead][CPT];
+    // the next kDwAhead tokens' x is loaded while the current ones are used
+    float xv[2][kDwAhead][CPT];
 #pragma unroll
-      for (int u = 0; u < kDwAhead; ++u)
-        if (tt0 + u < n) load_cols(x + (size_t)(tb + tt0 + u) * d + c, xv[u], CPT);
+    for (int u = 0; u < kDwAhead; ++u)
+      if (u < n) load_cols(x + (size_t)(tb + u) * d + c, xv[0][u], CPT);
+    for (int tt0 = 0; tt0 < n; tt0 += 2 * kDwAhead) {
 #pragma unroll
-      for (int u = 0; u < kDwAhead; ++u)
-        if (tt0 + u < n) {
-          const float* g = dls + (tt0 + u) * E;
+      for (int half = 0; half < 2; ++half) {
+        const int base = tt0 + half * kDwAhead;
+        if (base >= n) break;
+        const int nb = base + kDwAhead;
 #pragma unroll
-          for (int e = 0; e < EMAX; ++e)
-            if (e < E) {
-              const float ge = g[e];
+        for (int u = 0; u < kDwAhead; ++u)
+          if (nb + u < n) load_cols(x + (size_t)(tb + nb + u) * d + c, xv[half ^ 1][u], CPT);
 #pragma unroll
-              for (int i = 0; i < CPT; ++i) acc[i][e] = fmaf(xv[u][i], ge, acc[i][e]);
+        for (int u = 0; u < kDwAhead; ++u)
+          if (base + u < n) {
+            float g[EMAX];
+#pragma unroll
+            for (int q = 0; q < EMAX / 4; ++q) {
+              const float4 v = reinterpret_cast<const float4*>(dls + (base + u) * EMAX)[q];
+              g[4 * q] = v.x; g[4 * q + 1] = v.y; g[4 * q + 2] = v.z; g[4 * q + 3] = v.w;
             }
-        }
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e)
+              if (e < E) {
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) acc[i][e] = fmaf(xv[half][u][i], g[e], acc[i][e]);
+              }
+          }
+      }
     }
   }
   const long long total = (long long)d * E;
@@ -422,8 +469,17 @@ __global__ void __launch_bounds__(256)
   pdl_wait_and_release();
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
+    // 16 chunks' loads in flight at a time, added in chunk order
     float v = 0.f;
-    for (int c = 0; c < nchunks; ++c) v += dw_part[(size_t)c * total + i];
+    for (int c0 = 0; c0 < nchunks; c0 += 16) {
+      float t[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        t[u] = c0 + u < nchunks ? dw_part[(size_t)(c0 + u) * total + i] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (c0 + u < nchunks) v += t[u];
+    }
     dW[i] = v;
   }
   if (dbias != nullptr && blockIdx.x == 0)
@@ -477,9 +533,13 @@ cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const fl
                                 (double)c.E / (double)T_batch, dlogits);
   if (e != cudaSuccess) return e;
   const bool narrow = c.E <= 16;
-  if (narrow && c.d % 4 == 0) {
-    const dim3 grid((unsigned)ceil_div(c.d, 1024),
-                    (unsigned)std::max(1, std::min(ceil_div(c.T, 16), 2 * device_sm_count())));
+  if (narrow && c.d % 8 == 0) {
+    // about two CTAs per SM in all: each CTA loads its columns of W once, so
+    // the rows of CTAs share that cost over as many tokens as possible
+    const int gx = ceil_div(c.d, 1024);
+    const dim3 grid((unsigned)gx, (unsigned)std::max(
+                                      1, std::min(ceil_div(c.T, 16),
+                                                  ceil_div(2 * device_sm_count(), gx))));
     e = c.E <= 8 ? launch_kernel(route_dx_narrow_kernel<8>, grid, 256, 0, s, 0, dlogits, W, c.T,
                                  c.d, c.E, dx)
                  : launch_kernel(route_dx_narrow_kernel<16>, grid, 256, 0, s, 0, dlogits, W, c.T,
@@ -493,7 +553,7 @@ cudaError_t launch_route_backward(const moe_config_t& c, const void* x, const fl
   if (e != cudaSuccess) return e;
   const int nchunks = route_backward_chunks(c.T, c.E);
   if (narrow && c.d % 8 == 0) {
-    // E <= 8: 8 columns a thread; E <= 16: 4
+    // E <= 8: 8 columns a thread; E <= 16: 4 (64 accumulators either way)
     const int cpt = c.E <= 8 ? 8 : 4;
     const dim3 ngrid((unsigned)ceil_div(c.d, 256 * cpt), (unsigned)nchunks);
     if (c.act_dtype == MOE_BF16) {
