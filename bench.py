@@ -886,6 +886,33 @@ def experts_backward(w, lb, peaks):
     if api.moe_device_status(bws) != 0:
         raise RuntimeError("experts' backward: device error word set")
     ms = ev[0].elapsed_time(ev[1]) / reps
+
+    # Training forward (the experts' rows and, kept in bws, their
+    # pre-activations) against the plain forward, then the backward that
+    # takes the kept pre-activations instead of recomputing them.
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ev[0].record(stream)
+        for _ in range(reps):
+            fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / reps
+
+    saved = None
+    if w.kind != "linear":
+        fwd_ms = timed(lambda: api.moe_expert_ffn(cfg, lb.x_perm, lb.offsets, D["W_in"],
+                                                  D["W_up"], D["W_out"], lb.y_perm, lb.layer.ws))
+        train_ms = timed(lambda: api.moe_expert_ffn_train(cfg, lb.x_perm, lb.offsets, D["W_in"],
+                                                          D["W_up"], D["W_out"], lb.y_perm,
+                                                          lb.layer.ws, bws))
+        saved_ms = timed(lambda: api.moe_expert_ffn_backward_saved(
+            cfg, lb.x_perm, lb.offsets, D["W_in"], D["W_up"], D["W_out"], dyp, dxp, dWi, dWu, dWo,
+            bws))
+        saved = (fwd_ms, train_ms, saved_ms)
+    if api.moe_device_status(bws) != 0 or lb.device_status() != 0:
+        raise RuntimeError("experts' backward: device error word set")
     counts = o.counts.cpu().numpy()
     rows = A.kept_rows(counts, w.capacity_factor, T, k)
     mats = A.MATRICES[w.kind]
@@ -895,12 +922,22 @@ def experts_backward(w, lb, peaks):
     ach = algo / (ms / 1e3) / 1e12
     del dyp, dxp, dWi, dWu, dWo, bws
     torch.cuda.empty_cache()
-    return {"ms": ms, "TFLOP/s": ach, "frac_of_burst": ach / peaks["bf16_tflops"],
-            "algorithmic_flops": algo, "executed_flops": executed,
-            "note": "moe_expert_ffn_backward (pack, recompute of the pre-activations, dH with "
-                    "the activation backward fused, dX, weight gradients): algorithmic FLOPs = "
-                    "the dgrad and wgrad products (2x the forward's), executed adds the "
-                    "recomputed up projection; back to back, 5 calls"}
+    res = {"ms": ms, "TFLOP/s": ach, "frac_of_burst": ach / peaks["bf16_tflops"],
+           "algorithmic_flops": algo, "executed_flops": executed,
+           "note": "moe_expert_ffn_backward (pack, recompute of the pre-activations, dH with "
+                   "the activation backward fused, dX, weight gradients): algorithmic FLOPs = "
+                   "the dgrad and wgrad products (2x the forward's), executed adds the "
+                   "recomputed up projection; back to back, 5 calls"}
+    if saved is not None:
+        fwd_ms, train_ms, saved_ms = saved
+        ach_s = algo / (saved_ms / 1e3) / 1e12
+        res["saved"] = {
+            "ms": saved_ms, "TFLOP/s": ach_s, "frac_of_burst": ach_s / peaks["bf16_tflops"],
+            "forward_experts_ms": fwd_ms, "train_forward_experts_ms": train_ms,
+            "note": "moe_expert_ffn_train (the forward's experts keeping their fp32 "
+                    "pre-activations in the backward workspace) against moe_expert_ffn, and "
+                    "moe_expert_ffn_backward_saved (no recompute); back to back, 5 calls each"}
+    return res
 
 
 def cpu_baseline(w, tokens):

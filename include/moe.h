@@ -460,6 +460,30 @@ int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const i
                             const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
                             float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Training forward of the experts and the backward that uses what it kept.
+ * moe_expert_ffn_train: moe_expert_ffn (same arguments and the same y_perm,
+ *   bit for bit) that also writes every kept row's fp32 pre-activations, A =
+ *   X W_in (and B = X W_up for SwiGLU), into bwd_ws, the workspace of
+ *   moe_expert_ffn_backward (bwd_ws_bytes >= moe_expert_backward_workspace_size;
+ *   the same offsets must be given to the backward).  bf16 experts only
+ *   (MOE_ERR_UNSUPPORTED for linear experts, which have no pre-activations).
+ * moe_expert_ffn_backward_saved: moe_expert_ffn_backward with the same
+ *   arguments, taking A and B from ws (written there by
+ *   moe_expert_ffn_train on the same x_perm, offsets and weights) instead
+ *   of recomputing them: a quarter of the backward's tensor work less, for
+ *   (R_max + 63 E) x (1 + SwiGLU) x d_hidden fp32 written by the forward.
+ *   The results equal moe_expert_ffn_backward's up to the order in which the
+ *   tensor cores sum A and B. */
+int moe_expert_ffn_train(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                         const void* W_in, const void* W_up, const void* W_out, void* y_perm,
+                         void* ws, size_t ws_bytes, void* bwd_ws, size_t bwd_ws_bytes,
+                         moe_stream_t stream);
+int moe_expert_ffn_backward_saved(const moe_config_t* cfg, const void* x_perm,
+                                  const int32_t* offsets, const void* W_in, const void* W_up,
+                                  const void* W_out, const float* dy_perm, float* dx_perm,
+                                  float* dW_in, float* dW_up, float* dW_out, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream);
+
 /* moe_permute_backward: the grouped rows' input gradients back to their
  * tokens, dx[t] = dx_add[t] + sum over kept slots j (j increasing) of
  * dx_perm[dest[t, j]] (each token's input feeds its kept rows; [MLG

@@ -37,6 +37,9 @@ _SIGNATURES = {
     "moe_check_wait_timeout": (ctypes.c_int, [_c_p, ctypes.c_size_t, ctypes.c_uint32, _c_p]),
     "moe_expert_backward_workspace_size": (ctypes.c_size_t, [_c_p]),
     "moe_expert_ffn_backward": (ctypes.c_int, [_c_p] * 12 + [ctypes.c_size_t, _c_p]),
+    "moe_expert_ffn_backward_saved": (ctypes.c_int, [_c_p] * 12 + [ctypes.c_size_t, _c_p]),
+    "moe_expert_ffn_train": (ctypes.c_int, [_c_p] * 8 + [ctypes.c_size_t, _c_p, ctypes.c_size_t,
+                                                          _c_p]),
     "moe_permute_backward": (ctypes.c_int, [_c_p] * 6),
     "moe_combine_backward": (ctypes.c_int, [_c_p] * 8),
     "moe_route_backward": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_int32] + [_c_p] * 5 +
@@ -279,6 +282,26 @@ def moe_dispatch_shard(cfg, rank, world, T_global, records, x, expert_indices, p
         _ptr(counts), _ptr(offsets), _ptr(dest), _ptr(perm_token), _ptr(drop_mask), _ptr(f),
         _ptr(aux_loss), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)),
         "moe_dispatch_shard")
+
+
+def moe_expert_ffn_backward_saved(cfg, x_perm, offsets, W_in, W_up, W_out, dy_perm, dx_perm,
+                                  dW_in, dW_up, dW_out, ws, stream=None) -> None:
+    """moe_expert_ffn_backward with the pre-activations that
+    moe_expert_ffn_train left in `ws`."""
+    _check(load_library().moe_expert_ffn_backward_saved(
+        ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(W_in), _ptr(W_up), _ptr(W_out),
+        _ptr(dy_perm), _ptr(dx_perm), _ptr(dW_in), _ptr(dW_up), _ptr(dW_out), _ptr(ws),
+        ws.numel(), _stream(stream)), "moe_expert_ffn_backward_saved")
+
+
+def moe_expert_ffn_train(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws, bwd_ws,
+                         stream=None) -> None:
+    """moe_expert_ffn that also keeps the pre-activations in bwd_ws (the
+    experts' backward workspace)."""
+    _check(load_library().moe_expert_ffn_train(
+        ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(W_in), _ptr(W_up), _ptr(W_out),
+        _ptr(y_perm), _ptr(ws), ws.numel(), _ptr(bwd_ws), bwd_ws.numel(), _stream(stream)),
+        "moe_expert_ffn_train")
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, W_in, W_up, W_out, y_perm, ws, stream=None) -> None:

@@ -73,11 +73,15 @@ __device__ bool padded_offsets_warp(const int32_t* offsets, int E, int rows_max,
 
 // One warp per padded row: Xp[p] = x_perm[src] (bf16) and dYp[p] =
 // bf16(dy_perm[src]) for the expert's real rows, zeros for its padding.
+// With saved pre-activations (pre != null: the training forward wrote the
+// real rows), a padding row's pre-activations are zeroed too (pre_blocks
+// blocks of kBwdPreBlock floats per row, block b at b * rows_pad rows).
 __global__ void __launch_bounds__(256)
     pack_rows_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __restrict__ dy_perm,
                      const int32_t* __restrict__ offsets, int E, int d, int d_out, int rows_max,
                      int rows_pad, __nv_bfloat16* __restrict__ xp,
-                     __nv_bfloat16* __restrict__ dyp, int32_t* err) {
+                     __nv_bfloat16* __restrict__ dyp, int32_t* err, float* __restrict__ pre,
+                     int pre_blocks) {
   pdl_wait_and_release();
   __shared__ int row_off[257], poff[257];
   if (threadIdx.x < 32) padded_offsets_warp(offsets, E, rows_max, row_off, poff, err);
@@ -109,6 +113,11 @@ __global__ void __launch_bounds__(256)
         yd[v] = make_uint4(0, 0, 0, 0);
       }
     }
+    if (pre != nullptr && !real)
+      for (int b = 0; b < pre_blocks; ++b) {
+        float4* pd = reinterpret_cast<float4*>(pre + ((size_t)b * rows_pad + p) * kBwdPreBlock);
+        for (int v = lane; v < kBwdPreBlock / 4; v += 32) pd[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
   }
 }
 
@@ -225,7 +234,7 @@ cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
                                    const int32_t* offsets, const void* W_in, const void* W_up,
                                    const void* W_out, const float* dy_perm, float* dx_perm,
                                    float* dW_in, float* dW_up, float* dW_out, void* ws,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, bool pre_saved) {
   const ExpertBwdLayout L = expert_backward_layout(c);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* err = reinterpret_cast<int32_t*>(base + L.ctrl);
@@ -250,16 +259,21 @@ cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
   const int rows_pad = expert_backward_pad_rows(rows_max, c.E);
   if (rows_max > 0) {
     const int blocks = std::min(ceil_div(rows_pad, 8), sms * 8);
+    const int pre_blocks = (c.expert_kind == MOE_EXPERT_SWIGLU ? 2 : 1) *
+                           ceil_div(c.d_hidden, kBwdPreBlock);
     cudaError_t e = launch_kernel(pack_rows_kernel, blocks, 256, 0, s, 0,
                                   static_cast<const __nv_bfloat16*>(x_perm), dy_perm, offsets, c.E,
-                                  c.d, c.d_out, rows_max, rows_pad, xp, dyp, err);
+                                  c.d, c.d_out, rows_max, rows_pad, xp, dyp, err,
+                                  pre_saved ? reinterpret_cast<float*>(base + L.pre) : nullptr,
+                                  pre_blocks);
     if (e != cudaSuccess) return e;
   }
   return launch_expert_backward_gemms(
       c, offsets, xp, dyp, static_cast<const __nv_bfloat16*>(W_in),
       static_cast<const __nv_bfloat16*>(W_up), static_cast<const __nv_bfloat16*>(W_out),
       reinterpret_cast<float*>(base + L.pre), reinterpret_cast<__nv_bfloat16*>(base + L.dab),
-      reinterpret_cast<__nv_bfloat16*>(base + L.hid), dx_perm, dW_in, dW_up, dW_out, err, s);
+      reinterpret_cast<__nv_bfloat16*>(base + L.hid), dx_perm, dW_in, dW_up, dW_out, err, s,
+      pre_saved);
 }
 
 cudaError_t launch_permute_backward(const moe_config_t& c, const float* dx_perm,

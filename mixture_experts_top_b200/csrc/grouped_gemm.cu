@@ -110,7 +110,49 @@ struct GemmArgs {
   // Pair kernel: [0] the next tile to hand out, [1] CTAs finished; both 0
   // at launch and left at 0 by the last CTA to finish.
   unsigned* sched;
+  // Training forward (kEpiSwiglu / kEpiRelu, else null): every kept row's
+  // fp32 pre-activations A (and B) are also written into the backward's
+  // layout: blocks of kBwdPreBlock hidden units, block (p, u) = pre_Rp rows,
+  // row = the row's padded row (each expert's rows rounded up to
+  // kBwdPadRows, in expert order).
+  float* pre;
+  int pre_Rp, pre_mt;
 };
+
+// Padded row offsets of the backward's layout (each expert's rows rounded
+// up to kBwdPadRows), by one warp: poff[e] for e = 0..E.
+__device__ __forceinline__ void padded_offsets(const int* row_off, int E, bool ok, int lane,
+                                               int* poff) {
+  int carry = 0;
+  for (int base = 0; base < E; base += 32) {
+    const int e = base + lane;
+    const int pr = (ok && e < E) ? (row_off[e + 1] - row_off[e] + kBwdPadRows - 1) / kBwdPadRows *
+                                       kBwdPadRows
+                                 : 0;
+    int incl = pr;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (e < E) poff[e + 1] = carry + incl;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) poff[0] = 0;
+}
+
+// The row's pre-activations for hidden units [h0, h0 + 32) of matrix p (0:
+// A, 1: B) from 32 fp32 accumulator columns.
+__device__ __forceinline__ void store_pre32(const GemmArgs& g, int p, int prow, int h0,
+                                            const uint32_t (&r)[32]) {
+  float* dst = g.pre + ((size_t)(p * g.pre_mt + h0 / kBwdPreBlock) * g.pre_Rp + prow) *
+                           kBwdPreBlock + (h0 % kBwdPreBlock);
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    if (h0 + 4 * v < g.N)
+      *reinterpret_cast<uint4*>(dst + 4 * v) =
+          make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+}
 
 struct TileCoord {
   int e, m0, rows, n_tile;
@@ -143,7 +185,7 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // warp-collective); only rows with `valid` store.
 template <int EPI>
 __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
-                                                const GemmArgs& g) {
+                                                const GemmArgs& g, int prow = -1) {
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   if (EPI == kEpiScatter) {
     // orow_off is the grouped row; its token's output row gets gate * acc,
@@ -182,6 +224,10 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
       tmem_ld_32x32b_x32(tacc + cc, gr);
       tmem_ld_32x32b_x32(tacc + OUT_COLS + cc, ur);
       tmem_ld_wait();
+      if (valid && prow >= 0) {
+        store_pre32(g, 0, prow, n0 + cc, gr);
+        store_pre32(g, 1, prow, n0 + cc, ur);
+      }
       if (valid) {
         uint32_t pk[16];
 #pragma unroll
@@ -223,6 +269,7 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + cc, r);
       tmem_ld_wait();
+      if (valid && prow >= 0) store_pre32(g, 0, prow, n0 + cc, r);
       if (valid) {
         uint32_t pk[16];
 #pragma unroll
@@ -275,6 +322,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
   int* tile_prefix = reinterpret_cast<int*>(tmem_holder + 4);  // MAX_E + 1
   int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
+  int* poff = row_off + (MAX_E + 1);                             // MAX_E + 1 (training forward)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E;
@@ -301,6 +349,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (e < E) tile_prefix[e + 1] = (carry + incl) * g.n_tiles;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (g.pre != nullptr) padded_offsets(row_off, E, ok, lane, poff);
     if (lane == 0) {
       tile_prefix[0] = 0;
       tma_prefetch_map(&tmA);
@@ -464,7 +513,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = row < c.rows;
       const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
                                                  : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
+      const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow);
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[acc]);
       acc ^= 1;
@@ -536,6 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int* tile_q = reinterpret_cast<int*>(tmem_holder + 4);         // kTileQ
   int* tile_prefix = tile_q + kTileQ;                            // MAX_E + 1
   int* row_off = tile_prefix + (MAX_E + 1);                      // MAX_E + 1
+  int* poff = row_off + (MAX_E + 1);                             // MAX_E + 1 (training forward)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E;
@@ -562,6 +613,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (e < E) tile_prefix[e + 1] = (carry + incl) * g.n_tiles;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (g.pre != nullptr) padded_offsets(row_off, E, ok, lane, poff);
     if (lane == 0) {
       tile_prefix[0] = 0;
       tma_prefetch_map(&tmA);
@@ -776,7 +828,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = row < c.rows;
       const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
                                                  : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g);
+      const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
@@ -867,8 +920,9 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
                                 cudaStream_t s, const int32_t* perm, int a_rows,
-                                const ScatterCombine* sc) {
+                                const ScatterCombine* sc, float* pre) {
   if (rows_max == 0) return cudaSuccess;
+  if (pre != nullptr && epi != kEpiSwiglu && epi != kEpiRelu) return cudaErrorInvalidValue;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const bool gather = perm != nullptr;
   if (gather && (epi == kEpiNone || epi == kEpiScatter || a_rows <= 0)) return cudaErrorInvalidValue;
@@ -895,6 +949,9 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   g.dest = sc != nullptr ? sc->dest : nullptr;
   g.T = sc != nullptr ? sc->T : 0;
   g.sched = sched;
+  g.pre = pre;
+  g.pre_Rp = pre != nullptr ? expert_backward_pad_rows(rows_max, E) : 0;
+  g.pre_mt = ceil_div(N, kBwdPreBlock);
   // Expert groups of 1024 rows or more on average: CTA pairs (M = 256 tiles,
   // a third less traffic per CTA); smaller groups: single CTAs (M = 128
   // tiles waste fewer rows at group edges).

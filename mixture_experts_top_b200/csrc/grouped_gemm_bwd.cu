@@ -225,7 +225,18 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int 
 #pragma unroll
       for (int j = 0; j < 32; ++j) base[(size_t)j * PM] = __uint_as_float(r[j]);
     } else if (STAGE == kDH) {
-      if (m < g.DHp) {
+      if (m < g.DHp && m >= g.DH) {
+        // hidden units past DH (the 64-wide padding): zero gradients and H,
+        // whatever the pre-activation blocks hold there
+        const size_t row = (size_t)(prow0 + c0);
+        const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+          g.dab[(row + j) * wide + m] = z;
+          if (g.swiglu) g.dab[(row + j) * wide + g.DHp + m] = z;
+          g.hid[(row + j) * (size_t)g.DHp + m] = z;
+        }
+      } else if (m < g.DHp) {
         const size_t row = (size_t)(prow0 + c0);
         const float* pa = g.pre + ((size_t)(t.m0 / PM) * g.Rp + row) * PM + mrow;
         const float* pb = g.pre + ((size_t)(g.m_tiles + t.m0 / PM) * g.Rp + row) * PM + mrow;
@@ -628,7 +639,7 @@ cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* o
                                          const __nv_bfloat16* W_out, float* pre,
                                          __nv_bfloat16* dab, __nv_bfloat16* hid, float* dx_perm,
                                          float* dW_in, float* dW_up, float* dW_out, int32_t* err,
-                                         cudaStream_t s) {
+                                         cudaStream_t s, bool pre_saved) {
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const int E = c.E, d = c.d, DH = c.d_hidden, d_out = c.d_out;
   const int swiglu = c.expert_kind == MOE_EXPERT_SWIGLU ? 1 : 0;
@@ -655,7 +666,7 @@ cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* o
   CUtensorMap ta, ta1, tb, tb1, to0, to1, to2;
   cudaError_t e;
 
-  if (c.T * c.top_k > 0) {
+  if (c.T * c.top_k > 0 && !pre_saved) {
     // 1. pre^T = [W_in | W_up]^T Xp^T  (A M-major: the weights as stored; B: Xp rows)
     g.K = d;
     g.m_tiles = ceil_div(DH, PM);
@@ -666,6 +677,8 @@ cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* o
     e = run_stage<kPre>(ta, ta1, tb, tb, ta, ta, ta, g, (1L + swiglu) * g.m_tiles * row_tiles_max,
                         s);
     if (e != cudaSuccess) return e;
+  }
+  if (c.T * c.top_k > 0) {
 
     // 2. dH^T = W_out dYp^T; epilogue: dAB and H  (A K-major: W_out[e] rows)
     g.K = d_out;

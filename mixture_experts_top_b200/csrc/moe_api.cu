@@ -93,9 +93,12 @@ int act_bytes(const moe_config_t& c) { return c.act_dtype == MOE_BF16 ? 2 : 4; }
 // Up and down projections (or the linear expert) on grouped rows.
 // perm == nullptr: A is x_perm, the grouped rows.  Otherwise A is x (T, d)
 // and grouped row r is x[perm[r]].
+// pre (bf16 experts, or null): the experts' backward workspace's pre region,
+// into which the up projection also writes the fp32 pre-activations.
 cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* perm,
                         const int32_t* offsets, const void* W_in, const void* W_up,
-                        const void* W_out, void* y_perm, void* ws, cudaStream_t s) {
+                        const void* W_out, void* y_perm, void* ws, cudaStream_t s,
+                        float* pre = nullptr) {
   const WsLayout L = workspace_layout(c);
   int32_t* err = at<int32_t>(ws, L.ctrl);
   const int rows_max = c.T * c.top_k;
@@ -110,7 +113,7 @@ cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* per
       epi, static_cast<const __nv_bfloat16*>(A), rows_max, c.d,
       static_cast<const __nv_bfloat16*>(W_in),
       epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
-      offsets, hidden, err, sched, s, perm, c.T);
+      offsets, hidden, err, sched, s, perm, c.T, nullptr, pre);
   if (e != cudaSuccess) return e;
   return launch_grouped_gemm(kEpiNone, hidden, rows_max, c.d_hidden,
                              static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
@@ -423,13 +426,18 @@ size_t moe_expert_backward_workspace_size(const moe_config_t* cfg) {
   return expert_backward_layout(*cfg).total;
 }
 
-int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
-                            const void* W_in, const void* W_up, const void* W_out,
-                            const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
-                            float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+namespace {
+
+int expert_backward_entry(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                          const void* W_in, const void* W_up, const void* W_out,
+                          const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
+                          float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                          bool pre_saved) {
   int st = check_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config_t& c = *cfg;
+  if (pre_saved && c.expert_kind == MOE_EXPERT_LINEAR)
+    return fail(MOE_ERR_UNSUPPORTED, "linear experts keep no pre-activations");
   const bool swiglu = c.expert_kind == MOE_EXPERT_SWIGLU;
   const bool linear = c.expert_kind == MOE_EXPERT_LINEAR;
   MOE_REQUIRE(offsets);
@@ -466,8 +474,41 @@ int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const i
                                        " bytes (moe_expert_backward_workspace_size)");
   const cudaError_t e = launch_expert_backward(c, x_perm, offsets, W_in, W_up, W_out, dy_perm,
                                                dx_perm, dW_in, dW_up, dW_out, ws,
-                                               reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_backward");
+                                               reinterpret_cast<cudaStream_t>(stream), pre_saved);
+  return e == cudaSuccess ? MOE_OK
+                          : cuda_fail(e, pre_saved ? "moe_expert_ffn_backward_saved"
+                                                   : "moe_expert_ffn_backward");
+}
+
+// The experts' backward workspace given to the training forward.
+int check_bwd_ws(const moe_config_t& c, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return fail(MOE_ERR_WORKSPACE, "backward workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_WORKSPACE, "backward workspace must be 256-byte aligned");
+  const size_t need = expert_backward_layout(c).total;
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "backward workspace too small: need " + std::to_string(need) +
+                                       " bytes (moe_expert_backward_workspace_size)");
+  return MOE_OK;
+}
+
+}  // namespace
+
+int moe_expert_ffn_backward(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                            const void* W_in, const void* W_up, const void* W_out,
+                            const float* dy_perm, float* dx_perm, float* dW_in, float* dW_up,
+                            float* dW_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return expert_backward_entry(cfg, x_perm, offsets, W_in, W_up, W_out, dy_perm, dx_perm, dW_in,
+                               dW_up, dW_out, ws, ws_bytes, stream, false);
+}
+
+int moe_expert_ffn_backward_saved(const moe_config_t* cfg, const void* x_perm,
+                                  const int32_t* offsets, const void* W_in, const void* W_up,
+                                  const void* W_out, const float* dy_perm, float* dx_perm,
+                                  float* dW_in, float* dW_up, float* dW_out, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream) {
+  return expert_backward_entry(cfg, x_perm, offsets, W_in, W_up, W_out, dy_perm, dx_perm, dW_in,
+                               dW_up, dW_out, ws, ws_bytes, stream, true);
 }
 
 int moe_permute_backward(const moe_config_t* cfg, const float* dx_perm, const int32_t* dest,
@@ -639,6 +680,37 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm, const int32_t* o
   const cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws,
                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn");
+}
+
+int moe_expert_ffn_train(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
+                         const void* W_in, const void* W_up, const void* W_out, void* y_perm,
+                         void* ws, size_t ws_bytes, void* bwd_ws, size_t bwd_ws_bytes,
+                         moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.expert_kind == MOE_EXPERT_LINEAR)
+    return fail(MOE_ERR_UNSUPPORTED, "linear experts keep no pre-activations");
+  MOE_REQUIRE(offsets);
+  MOE_REQUIRE(W_in);
+  if (c.expert_kind == MOE_EXPERT_SWIGLU) MOE_REQUIRE(W_up);
+  MOE_REQUIRE(W_out);
+  if (c.T > 0) {
+    MOE_REQUIRE(x_perm);
+    MOE_REQUIRE(y_perm);
+  }
+  MOE_ALIGNED16(W_in);
+  MOE_ALIGNED16(W_up);
+  MOE_ALIGNED16(W_out);
+  MOE_ALIGNED16(x_perm);
+  MOE_ALIGNED16(y_perm);
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = check_bwd_ws(c, bwd_ws, bwd_ws_bytes)) != MOE_OK) return st;
+  float* pre = reinterpret_cast<float*>(static_cast<uint8_t*>(bwd_ws) +
+                                        expert_backward_layout(c).pre);
+  const cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws,
+                                    reinterpret_cast<cudaStream_t>(stream), pre);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_train");
 }
 
 int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t* perm_token,

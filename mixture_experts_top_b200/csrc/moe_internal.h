@@ -196,11 +196,14 @@ struct ScatterCombine {
 // the up projection's operand load).
 // sched: the workspace's tile counter (two unsigned, 0 before the launch and
 // left at 0), used where the CTA-pair kernel runs.
+// pre (kEpiSwiglu / kEpiRelu only, or null): also write every kept row's fp32
+// pre-activations into the experts' backward layout (the `pre` region of its
+// workspace, expert_backward_layout), for moe_expert_ffn_backward_saved.
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
                                 cudaStream_t s, const int32_t* perm = nullptr, int a_rows = 0,
-                                const ScatterCombine* sc = nullptr);
+                                const ScatterCombine* sc = nullptr, float* pre = nullptr);
 
 // Experts' backward (expert_backward.cu, grouped_gemm_bwd.cu).  The bf16
 // GEMMs work on a padded grouped layout: each expert's rows rounded up to a
@@ -217,18 +220,21 @@ struct ExpertBwdLayout {
   size_t ctrl, xp, dyp, pre, dab, hid, total;
 };
 ExpertBwdLayout expert_backward_layout(const moe_config_t& c);
+// pre_saved: the workspace's pre region already holds the pre-activations
+// (written by the training forward); they are not recomputed, and the pack
+// launch zeroes their padding rows.
 cudaError_t launch_expert_backward(const moe_config_t& c, const void* x_perm,
                                    const int32_t* offsets, const void* W_in, const void* W_up,
                                    const void* W_out, const float* dy_perm, float* dx_perm,
                                    float* dW_in, float* dW_up, float* dW_out, void* ws,
-                                   cudaStream_t s);
+                                   cudaStream_t s, bool pre_saved = false);
 cudaError_t launch_expert_backward_gemms(const moe_config_t& c, const int32_t* offsets,
                                          const __nv_bfloat16* xp, const __nv_bfloat16* dyp,
                                          const __nv_bfloat16* W_in, const __nv_bfloat16* W_up,
                                          const __nv_bfloat16* W_out, float* pre,
                                          __nv_bfloat16* dab, __nv_bfloat16* hid, float* dx_perm,
                                          float* dW_in, float* dW_up, float* dW_out, int32_t* err,
-                                         cudaStream_t s);
+                                         cudaStream_t s, bool pre_saved = false);
 // dx (T, d) = dx_add (or 0) + sum over kept slots j of dx_perm[dest[t, j]].
 cudaError_t launch_permute_backward(const moe_config_t& c, const float* dx_perm,
                                     const int32_t* dest, const float* dx_add, float* dx,

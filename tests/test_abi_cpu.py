@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 24
+    assert len(names) == 26
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -231,6 +231,15 @@ def test_expert_backward_argument_checks(moe_lib):
     st = moe_lib.moe_expert_ffn_backward(ctypes.byref(lin), FAKE, FAKE, FAKE, None, None, FAKE,
                                          FAKE, None, None, None, FAKE, n, None)
     assert st == api.MOE_ERR_INVALID_ARG and "dW_in" in moe_lib.moe_last_error_message().decode()
+    # the saved-pre-activation backward: same checks, and linear experts refused
+    st = moe_lib.moe_expert_ffn_backward_saved(ctypes.byref(cfg), *ins, FAKE, FAKE, None, FAKE,
+                                               FAKE, n, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "dW_up" in moe_lib.moe_last_error_message().decode()
+    assert moe_lib.moe_expert_ffn_backward_saved(ctypes.byref(cfg), *ins, *outs, FAKE, n - 256,
+                                                 None) == api.MOE_ERR_WORKSPACE
+    assert moe_lib.moe_expert_ffn_backward_saved(ctypes.byref(lin), FAKE, FAKE, FAKE, None, None,
+                                                 FAKE, FAKE, FAKE, None, None, FAKE, n, None) \
+        == api.MOE_ERR_UNSUPPORTED
     # rows back to tokens
     assert moe_lib.moe_permute_backward(ctypes.byref(cfg), None, FAKE, None, FAKE, None) == \
         api.MOE_ERR_INVALID_ARG
@@ -261,3 +270,24 @@ def test_binding_refuses_missing_library(tmp_path):
             api.load_library(str(tmp_path / "none.so"))
     finally:
         api._lib = saved
+
+
+def test_training_forward_argument_checks(moe_lib):
+    cfg = api.make_config(64, 64, 128, 64, 8, 2, "swiglu", "bf16")
+    ws = moe_lib.moe_workspace_size(ctypes.byref(cfg))
+    bws = moe_lib.moe_expert_backward_workspace_size(ctypes.byref(cfg))
+    args = [FAKE] * 7                          # x_perm, offsets, W_in, W_up, W_out, y_perm, ws
+    ok = lambda *tail: moe_lib.moe_expert_ffn_train(ctypes.byref(cfg), *args, ws, *tail)
+    # the backward workspace: NULL, too small, misaligned
+    assert ok(None, bws, None) == api.MOE_ERR_WORKSPACE
+    assert "backward workspace" in moe_lib.moe_last_error_message().decode()
+    assert ok(FAKE, bws - 256, None) == api.MOE_ERR_WORKSPACE
+    assert ok(FAKE + 16, bws, None) == api.MOE_ERR_WORKSPACE
+    # SwiGLU needs W_up; linear experts keep no pre-activations
+    st = moe_lib.moe_expert_ffn_train(ctypes.byref(cfg), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
+                                      ws, FAKE, bws, None)
+    assert st == api.MOE_ERR_INVALID_ARG and "W_up" in moe_lib.moe_last_error_message().decode()
+    lin = api.make_config(64, 32, 0, 32, 8, 2, "linear", "f32")
+    st = moe_lib.moe_expert_ffn_train(ctypes.byref(lin), FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                                      ws, FAKE, bws, None)
+    assert st == api.MOE_ERR_UNSUPPORTED

@@ -273,3 +273,68 @@ def test_layer_backward_against_oracle(name):
             _check(w, got[key], ref[key], key)
     for key in ("dx", "dW_router", "dbias"):
         _check(w, got[key], ref[key], key, elementwise=False, norm_tol=4e-2)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "fine_grained", "switch_relu", "ragged"])
+def test_training_forward_and_saved_backward(name):
+    """moe_expert_ffn_train writes the same expert rows as moe_expert_ffn
+    (bit for bit) and keeps the pre-activations in the backward workspace;
+    moe_expert_ffn_backward_saved then gives the recomputing backward's
+    gradients up to the order in which the tensor cores summed A and B, and
+    stays within the oracle bounds.  The backward workspace starts filled
+    with NaN, so a pre-activation the forward did not write (a padding row,
+    a padding hidden unit) would show."""
+    w = CASES[name]
+    inp = make_inputs(w, seed=41)
+    cfg = cfg_of(w)
+    ws = api.alloc_workspace(cfg)
+    _, t = _route_dispatch(w, inp, cfg, ws)
+    R = int(host(t["offsets"])[-1])
+    W = {key: dev(inp[key]) for key in ("W_in", "W_up", "W_out")}
+    f32 = dict(dtype=torch.float32, device="cuda")
+    y_plain = torch.full((w.T * w.top_k, w.d_out), 3.0, **f32)
+    y_train = torch.full((w.T * w.top_k, w.d_out), 3.0, **f32)
+    api.moe_expert_ffn(cfg, t["x_perm"], t["offsets"], W["W_in"], W["W_up"], W["W_out"], y_plain,
+                       ws)
+    bws = api.alloc_backward_workspace(cfg)
+    bws[256:].view(torch.uint8).fill_(0xFF)          # NaN everywhere but the error word
+    api.moe_expert_ffn_train(cfg, t["x_perm"], t["offsets"], W["W_in"], W["W_up"], W["W_out"],
+                             y_train, ws, bws)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(ws) == 0
+    assert np.array_equal(host(y_plain), host(y_train))
+
+    rng = np.random.default_rng(42)
+    dy = np.zeros((w.T * w.top_k, w.d_out), np.float32)
+    dy[:R] = rng.standard_normal((R, w.d_out)).astype(np.float32)
+    g_saved, g_rec = _grads(w, w.T), _grads(w, w.T)
+    api.moe_expert_ffn_backward_saved(cfg, t["x_perm"], t["offsets"], W["W_in"], W["W_up"],
+                                      W["W_out"], dev(dy), g_saved["dx_perm"], g_saved["dW_in"],
+                                      g_saved["dW_up"], g_saved["dW_out"], bws)
+    bws2 = api.alloc_backward_workspace(cfg)
+    api.moe_expert_ffn_backward(cfg, t["x_perm"], t["offsets"], W["W_in"], W["W_up"], W["W_out"],
+                                dev(dy), g_rec["dx_perm"], g_rec["dW_in"], g_rec["dW_up"],
+                                g_rec["dW_out"], bws2)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(bws) == 0 and api.moe_device_status(bws2) == 0
+    for key in ("dx_perm", "dW_in", "dW_up", "dW_out"):
+        if g_saved[key] is None:
+            continue
+        a, b = host(g_saved[key]), host(g_rec[key])
+        if key == "dx_perm":
+            a, b = a[:R], b[:R]
+        assert np.isfinite(a).all(), key
+        nb = float(np.linalg.norm(b))
+        assert float(np.linalg.norm(a - b)) <= 2e-3 * max(nb, 1e-30), key
+    # and against the oracle, on the saved path
+    offs = host(t["offsets"])
+    xp = host(t["x_perm"])
+    weights = {key: inp[key] for key in ("W_in", "W_up", "W_out")}
+    dx_ref = np.zeros((R, w.d))
+    for e in range(w.E):
+        lo, hi = int(offs[e]), int(offs[e + 1])
+        if hi > lo:
+            r = O.expert_backward(w.kind, O.widen(xp[lo:hi], w.dtype),
+                                  *O.expert_weights(weights, e, w.dtype), dy[lo:hi])
+            dx_ref[lo:hi] = r["dx"]
+    _check(w, host(g_saved["dx_perm"])[:R], dx_ref, "dx_perm (saved)")
