@@ -147,11 +147,13 @@ __device__ __forceinline__ void store_pre32(const GemmArgs& g, int p, int prow, 
                                             const uint32_t (&r)[32]) {
   float* dst = g.pre + ((size_t)(p * g.pre_mt + h0 / kBwdPreBlock) * g.pre_Rp + prow) *
                            kBwdPreBlock + (h0 % kBwdPreBlock);
+  // read only by the backward, much later: streamed past L2 (evict first)
 #pragma unroll
   for (int v = 0; v < 8; ++v)
     if (h0 + 4 * v < g.N)
-      *reinterpret_cast<uint4*>(dst + 4 * v) =
-          make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+      __stcs(reinterpret_cast<float4*>(dst + 4 * v),
+             make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
 }
 
 struct TileCoord {

@@ -223,7 +223,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int 
       // row, so the pair's warps write (and dH's read) whole runs in order
       float* base = g.pre + ((size_t)(t.p * g.m_tiles + t.m0 / PM) * g.Rp + prow0 + c0) * PM + mrow;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) base[(size_t)j * PM] = __uint_as_float(r[j]);
+      for (int j = 0; j < 32; ++j) __stcs(base + (size_t)j * PM, __uint_as_float(r[j]));
     } else if (STAGE == kDH) {
       if (m < g.DHp && m >= g.DH) {
         // hidden units past DH (the 64-wide padding): zero gradients and H,
@@ -276,7 +276,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int 
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int local = t.n0 + c0 + j;
-          if (local < rows) base[(size_t)local * g.d] = __uint_as_float(r[j]);
+          if (local < rows) __stcs(base + (size_t)local * g.d, __uint_as_float(r[j]));
         }
       }
     }
@@ -312,7 +312,10 @@ __device__ __forceinline__ void epilogue_wgrad(uint32_t tacc, const Tile& t, int
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_3d(out_map, box, t.n0 + c0, t.m0 + rank * BM + q * 32, t.e);
+      // written once, never read here: evict first, so they do not push the
+      // operands that the neighbouring tiles reuse out of L2
+      tma_store_3d(out_map, box, t.n0 + c0, t.m0 + rank * BM + q * 32, t.e,
+                   l2_policy_evict_first());
       bulk_commit_group();
     }
     ++nbox;
