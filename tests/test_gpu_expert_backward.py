@@ -152,8 +152,8 @@ def test_expert_backward_against_oracle(name):
 
 def test_expert_backward_idle_experts_and_repeat():
     """A +30 bias on one expert routes every top-1 slot there: the other
-    experts get exactly zero weight gradients; two calls give identical
-    bits (no atomics)."""
+    experts get exactly zero weight gradients; two calls on one workspace
+    give identical bits (no atomics)."""
     w = CASES["fine_grained"].replace(top_k=1, capacity_factor=0.0, n_hot=0, T=300)
     inp = make_inputs(w, seed=33)
     bias = np.zeros(w.E, np.float32)
@@ -175,6 +175,9 @@ def test_expert_backward_idle_experts_and_repeat():
         torch.cuda.synchronize()
         runs.append({k: host(v) for k, v in g.items() if v is not None})
     assert api.moe_device_status(bws) == 0
+    # nothing but the error word is left in the control block
+    ctrl = host(bws[:256]).view(np.uint32)
+    assert (ctrl[1:] == 0).all(), ctrl[ctrl != 0]
     for key in runs[0]:
         assert np.array_equal(runs[0][key], runs[1][key]), key
         if key != "dx_perm":
