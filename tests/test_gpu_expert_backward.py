@@ -341,3 +341,25 @@ def test_training_forward_and_saved_backward(name):
                                   *O.expert_weights(weights, e, w.dtype), dy[lo:hi])
             dx_ref[lo:hi] = r["dx"]
     _check(w, host(g_saved["dx_perm"])[:R], dx_ref, "dx_perm (saved)")
+
+
+def test_training_forward_and_saved_backward_empty_batch():
+    """T = 0: the training forward writes nothing and the saved backward
+    gives zero weight gradients, like the recomputing one."""
+    w = CASES["mixtral"].replace(T=0)
+    cfg = cfg_of(w)
+    ws = api.alloc_workspace(cfg)
+    bws = api.alloc_backward_workspace(cfg)
+    W = {key: dev(v) for key, v in
+         zip(("W_in", "W_up", "W_out"),
+             (np.zeros((w.E, w.d, w.d_hidden), np.uint16), np.zeros((w.E, w.d, w.d_hidden), np.uint16),
+              np.zeros((w.E, w.d_hidden, w.d_out), np.uint16)))}
+    offsets = torch.zeros(w.E + 1, dtype=torch.int32, device="cuda")
+    api.moe_expert_ffn_train(cfg, None, offsets, W["W_in"], W["W_up"], W["W_out"], None, ws, bws)
+    g = _grads(w, 0)
+    api.moe_expert_ffn_backward_saved(cfg, None, offsets, W["W_in"], W["W_up"], W["W_out"], None,
+                                      None, g["dW_in"], g["dW_up"], g["dW_out"], bws)
+    torch.cuda.synchronize()
+    assert api.moe_device_status(ws) == 0 and api.moe_device_status(bws) == 0
+    for key in ("dW_in", "dW_up", "dW_out"):
+        assert (host(g[key]) == 0).all(), key

@@ -80,3 +80,51 @@ def test_captured_forward_replays_bit_exact(name):
         for k in KEYS:
             assert np.array_equal(ref[k], got[k]), k
     assert not np.array_equal(got1["output"], got2["output"])
+
+
+def test_captured_expert_backward_replays_bit_exact():
+    """The experts' backward (CTA-pair GEMMs, TMA-stored weight gradients)
+    captured and replayed gives the eager call's bits."""
+    from mixture_experts_top_b200 import api
+    w = CASES["mixtral"].replace(T=1024)
+    inp = make_inputs(w, seed=5)
+    cfg = cfg_of(w)
+    E, R = w.E, w.T * w.top_k
+    rng = np.random.default_rng(6)
+    counts = rng.multinomial(R - 40, np.full(E, 1.0 / E))
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32,
+                           device="cuda")
+    x_perm = dev(inp["x"].repeat(w.top_k, axis=0))
+    dy = torch.from_numpy(rng.standard_normal((R, w.d_out)).astype(np.float32)).cuda()
+    W = {key: dev(inp[key]) for key in ("W_in", "W_up", "W_out")}
+    f32 = dict(dtype=torch.float32, device="cuda")
+
+    def grads():
+        return [torch.zeros((R, w.d), **f32), torch.zeros((E, w.d, w.d_hidden), **f32),
+                torch.zeros((E, w.d, w.d_hidden), **f32), torch.zeros((E, w.d_hidden, w.d_out), **f32)]
+
+    def run(out, bws):
+        api.moe_expert_ffn_backward(cfg, x_perm, offsets, W["W_in"], W["W_up"], W["W_out"], dy,
+                                    *out, bws)
+
+    ref, bws0 = grads(), api.alloc_backward_workspace(cfg)
+    run(ref, bws0)
+    torch.cuda.synchronize()
+    got, bws = grads(), api.alloc_backward_workspace(cfg)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(got, bws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for t in got:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(got, bws)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert api.moe_device_status(bws) == 0
+    for a, b in zip(ref, got):
+        assert np.array_equal(host(a), host(b))
