@@ -712,6 +712,8 @@ def run_ours(args, rank, world):
     if w.dtype == "bf16":
         extras["routing_backward"] = routing_backward(w, lb, peaks)
         extras["experts_backward"] = experts_backward(w, lb, peaks)
+        if w.kind != "linear":
+            extras["training_step"] = training_step(w, lb, peaks)
 
     counts = o.counts.cpu().numpy()
     rows = A.kept_rows(counts, w.capacity_factor, T, k)
@@ -771,6 +773,76 @@ def run_ours(args, rank, world):
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def training_step(w, lb, peaks, steps=5, warmup=3):
+    """One training step of the layer through the public calls, timed as a
+    whole: the forward with the experts keeping their pre-activations
+    (moe_route, moe_dispatch, moe_expert_ffn_train, moe_combine), then the
+    backward from a fixed output gradient (moe_combine_backward,
+    moe_route_backward, moe_expert_ffn_backward_saved, moe_permute_backward)."""
+    import torch
+    from mixture_experts_top_b200 import api
+    D, o, cfg, stream = lb.D, lb.layer.out, lb.cfg, lb.stream
+    T, k, E = w.T, w.top_k, w.E
+    f32 = dict(dtype=torch.float32, device="cuda")
+    Lg = torch.empty((T, E), **f32)
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    dy = torch.randn((T, w.d_out), device="cuda", generator=gen).to(o.output.dtype)
+    dyp = torch.empty((T * k, w.d_out), **f32)
+    dg = torch.empty((T, k), **f32)
+    daux = torch.ones(1, **f32)
+    dx_route = torch.empty((T, w.d), **f32)
+    dx_perm = torch.empty((T * k, w.d), **f32)
+    dx = torch.empty((T, w.d), **f32)
+    dWr = torch.empty((w.d, E), **f32)
+    dbias = torch.empty(E, **f32)
+    dWi = torch.empty(tuple(D["W_in"].shape), **f32)
+    dWu = None if D["W_up"] is None else torch.empty(tuple(D["W_up"].shape), **f32)
+    dWo = torch.empty(tuple(D["W_out"].shape), **f32)
+    bws = api.alloc_backward_workspace(cfg)
+    ws = lb.layer.ws
+
+    def once():
+        api.moe_route(cfg, D["x"], D["W_router"], D["logit_bias"], D["noise"], o.expert_indices,
+                      o.gates, lb.P, Lg, ws)
+        api.moe_dispatch(cfg, D["x"], o.expert_indices, lb.P, o.counts, lb.offsets, lb.dest,
+                         lb.perm, o.drop_mask, lb.f, o.aux_loss, lb.x_perm, ws)
+        api.moe_expert_ffn_train(cfg, lb.x_perm, lb.offsets, D["W_in"], D["W_up"], D["W_out"],
+                                 lb.y_perm, ws, bws)
+        api.moe_combine(cfg, lb.y_perm, lb.dest, o.gates, o.output)
+        api.moe_combine_backward(cfg, dy, lb.y_perm, lb.dest, o.gates, dyp, dg)
+        api.moe_route_backward(cfg, D["x"], D["W_router"], Lg, o.expert_indices, o.gates, lb.f,
+                               dg, daux, 0, dx_route, dWr, dbias, None, ws)
+        api.moe_expert_ffn_backward_saved(cfg, lb.x_perm, lb.offsets, D["W_in"], D["W_up"],
+                                          D["W_out"], dyp, dx_perm, dWi, dWu, dWo, bws)
+        api.moe_permute_backward(cfg, dx_perm, lb.dest, dx_route, dx)
+
+    for _ in range(warmup):
+        once()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for _ in range(steps):
+        once()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    if api.moe_device_status(bws) != 0 or lb.device_status() != 0:
+        raise RuntimeError("training step: device error word set")
+    ms = ev[0].elapsed_time(ev[1]) / steps
+    rows = A.kept_rows(o.counts.cpu().numpy(), w.capacity_factor, T, k)
+    fwd = A.expert_gemm_flops(rows, w.d, w.d_hidden, w.d_out, w.kind)
+    flops = 3 * fwd          # forward products, then their dgrad and wgrad
+    ach = flops / (ms / 1e3) / 1e12
+    del dyp, dx_perm, dWi, dWu, dWo, bws
+    torch.cuda.empty_cache()
+    return {"ms": ms, "tokens_per_s": T / (ms / 1e3), "expert_TFLOP/s": ach,
+            "expert_frac_of_burst": ach / peaks["bf16_tflops"], "expert_flops": flops,
+            "steps": steps, "warmup": warmup,
+            "note": "forward (moe_route, moe_dispatch, moe_expert_ffn_train, moe_combine) and "
+                    "backward (moe_combine_backward, moe_route_backward, "
+                    "moe_expert_ffn_backward_saved, moe_permute_backward) from a fixed output "
+                    "gradient, 13+ launches a step; expert FLOPs = 3x the forward's products "
+                    "over the whole step's time"}
 
 
 def routing_backward(w, lb, peaks):
