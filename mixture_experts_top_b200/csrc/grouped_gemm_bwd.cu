@@ -155,7 +155,7 @@ __device__ __forceinline__ float sigmoid_f(float a) { return __fdividef(1.0f, 1.
 
 // Tile order: row stages expert -> M tile -> N tile (an expert's rows, a few
 // MB, stay in L2 while its weight tiles pass over them); kWgrad problem ->
-// expert -> M tile -> N tile.
+// expert -> the weight dimension with more blocks -> the one with fewer.
 template <int STAGE>
 __device__ __forceinline__ Tile decode(int tile, const int* prefix, const int* poff,
                                        const BwdArgs& g) {
@@ -193,8 +193,15 @@ __device__ __forceinline__ Tile decode(int tile, const int* prefix, const int* p
     t.p = p;
     t.e = local / (mt * nt);
     const int rem = local % (mt * nt);
-    t.m0 = (rem / nt) * PM;
-    t.n0 = (rem % nt) * BN;
+    // the dimension with fewer blocks runs innermost: the concurrent tiles
+    // then share a few blocks of the other operand and all of this one's
+    if (nt <= mt) {
+      t.m0 = (rem / nt) * PM;
+      t.n0 = (rem % nt) * BN;
+    } else {
+      t.m0 = (rem % mt) * PM;
+      t.n0 = (rem / mt) * BN;
+    }
     t.n = BN;
     t.kb0 = poff[t.e] / BK;
     t.nkb = (poff[t.e + 1] - poff[t.e]) / BK;
