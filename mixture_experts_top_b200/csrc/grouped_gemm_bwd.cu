@@ -250,8 +250,9 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int 
         float av[32], bv[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          av[j] = pa[(size_t)j * PM];
-          bv[j] = g.swiglu ? pb[(size_t)j * PM] : 0.f;
+          // each read once: streamed (evict first)
+          av[j] = __ldcs(pa + (size_t)j * PM);
+          bv[j] = g.swiglu ? __ldcs(pb + (size_t)j * PM) : 0.f;
         }
         __nv_bfloat16* da = g.dab + row * wide + m;
         __nv_bfloat16* hh = g.hid + row * (size_t)g.DHp + m;
@@ -271,9 +272,9 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, const Tile& t, int 
             dB = 0.0f;
             H = fmaxf(a, 0.0f);
           }
-          da[(size_t)j * wide] = __float2bfloat16_rn(dA);
-          if (g.swiglu) da[(size_t)j * wide + g.DHp] = __float2bfloat16_rn(dB);
-          hh[(size_t)j * g.DHp] = __float2bfloat16_rn(H);
+          __stcs(da + (size_t)j * wide, __float2bfloat16_rn(dA));
+          if (g.swiglu) __stcs(da + (size_t)j * wide + g.DHp, __float2bfloat16_rn(dB));
+          __stcs(hh + (size_t)j * g.DHp, __float2bfloat16_rn(H));
         }
       }
     } else {   // kDX: padded row -> the expert's unpadded grouped row (zero rows skipped)
