@@ -278,7 +278,14 @@ def test_layer_backward_against_oracle(name):
         _check(w, got[key], ref[key], key, elementwise=False, norm_tol=4e-2)
 
 
-@pytest.mark.parametrize("name", ["mixtral", "fine_grained", "switch_relu", "ragged"])
+TRAIN_CASES = dict(CASES)
+# 1024 grouped rows per expert on average: the forward runs on CTA pairs
+TRAIN_CASES["mixtral_pairs"] = WORKLOADS["mixtral"].replace(T=4096, d=256, d_hidden=512,
+                                                            d_out=256)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "fine_grained", "switch_relu", "ragged",
+                                  "mixtral_pairs"])
 def test_training_forward_and_saved_backward(name):
     """moe_expert_ffn_train writes the same expert rows as moe_expert_ffn
     (bit for bit) and keeps the pre-activations in the backward workspace;
@@ -287,7 +294,7 @@ def test_training_forward_and_saved_backward(name):
     stays within the oracle bounds.  The backward workspace starts filled
     with NaN, so a pre-activation the forward did not write (a padding row,
     a padding hidden unit) would show."""
-    w = CASES[name]
+    w = TRAIN_CASES[name]
     inp = make_inputs(w, seed=41)
     cfg = cfg_of(w)
     ws = api.alloc_workspace(cfg)
