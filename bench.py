@@ -125,9 +125,12 @@ def profiled_traffic(kernel_file: str, summary: str):
 
 
 def fused_combine(w) -> bool:
-    """Top-1 with bf16 experts: the combine runs in the down projection's
-    epilogue (moe_expert_ffn_combine), with no combine kernel."""
-    return w.top_k == 1 and w.kind != "linear"
+    """The form moe_forward uses: the combine in the down projection's
+    epilogue (moe_expert_ffn_combine, no combine kernel), or moe_expert_ffn
+    then moe_combine."""
+    from mixture_experts_top_b200 import api as _api
+    return _api.moe_forward_combine_fused(_api.make_config(
+        w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype, w.capacity_factor))
 
 
 def launches_per_step(w, cfg, world: int = 1) -> int:
@@ -137,7 +140,7 @@ def launches_per_step(w, cfg, world: int = 1) -> int:
     E <= 64) or SIMT router + P mean; dispatch = count (its last CTA runs
     the scan) + scatter; experts = up and
     down GEMM (bf16) or the fp32 linear kernel; combine = 1, or 0 where it is
-    fused into the down projection (top-1).  A rank of a split batch adds
+    fused into the down projection.  A rank of a split batch adds
     its exchange record (count + total)."""
     from mixture_experts_top_b200 import api as _api
     if w.T == 0:
@@ -366,7 +369,7 @@ class LayerBench:
                              self.layer.ws)
         mark(2)
         if self.fused_combine:
-            # top-1: the combine is the down projection's epilogue
+            # the combine is the down projection's epilogue
             api.moe_expert_ffn_combine(cfg, self.x_perm, self.offsets, self.perm, self.dest,
                                        o.gates, D["W_in"], D["W_up"], D["W_out"], out,
                                        self.layer.ws)
@@ -528,9 +531,11 @@ def gemm_roofline(w, rows, used, expert_ms, peaks, peak_src, regime):
         tensor_peak = burst = sustained = None
     hbm = peaks["hbm_gbs"]
     elem = 4 if w.kind == "linear" else 2
-    # rows out: fp32 expert rows, or (top-1, combine in the epilogue) every
-    # token's bf16 output row
-    out_bytes = w.T * w.d_out * 2 if fused_combine(w) else rows * w.d_out * 4
+    # rows out: fp32 expert rows (kept for the combine), then with the combine
+    # in the epilogue every token's bf16 output row; at top-1 only the latter
+    out_bytes = rows * w.d_out * 4 if w.top_k > 1 or not fused_combine(w) else 0
+    if fused_combine(w):
+        out_bytes += w.T * w.d_out * 2
     gemm_bytes = (A.expert_weight_bytes(used, w.d, w.d_hidden, w.d_out, w.kind, elem)
                   + rows * w.d * elem + out_bytes
                   + (0 if w.kind == "linear" else 2 * rows * w.d_hidden * 2))

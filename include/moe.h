@@ -111,7 +111,8 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * *code_out (0 = no device-side error since the last clear) and clears it.
  * The word holds the first error recorded: 1 an expert index outside [0, E);
  * 2 offsets that are not a partition of the row buffer; 3 a gathered row
- * index (perm_token) outside [0, T); 4 a sharded dispatch whose exchange
+ * index (perm_token) outside [0, T), or a slot's grouped row (dest) at or
+ * beyond T * top_k in the fused combine; 4 a sharded dispatch whose exchange
  * record for this rank is not its own, or whose records' token counts do
  * not add up to T_global; 20 moe_check_wait_timeout's
  * intended timeout; 16-19 a pipeline wait that ran out of
@@ -344,20 +345,40 @@ int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x, const int32_t*
 
 /* The experts and the combine in one call: output as moe_combine would
  * write it from moe_expert_ffn's rows.  [MLG Algorithm 3; PFD Switch: top-1,
- * a dropped token outputs 0]  With top_k = 1 and bf16 experts the combine
- * is the down projection's epilogue: each kept grouped row r writes
- * gates[t] * row into output row t = perm_token[r] (the same fp32 product
- * and one rounding as moe_combine, so the same bits), tokens whose slot was
- * dropped get a zero row, and neither y_perm nor a combine kernel is used.
- * Otherwise it runs moe_expert_ffn into the workspace's y_perm, then the
- * combine kernel.
+ * a dropped token outputs 0]  With bf16 experts the combine is the down
+ * projection's epilogue and no combine kernel runs:
+ *   top_k = 1: each kept grouped row r writes gates[t] * row into output row
+ *     t = perm_token[r] (the same fp32 product and one rounding as
+ *     moe_combine, so the same bits); no y_perm is written.
+ *   top_k > 1: each kept row is also written, fp32, to the workspace's
+ *     y_perm; after a row has written an output column block it counts
+ *     itself on its token's counter for that block (acquire-release atomic
+ *     add), and the row that completes the token's kept slots sums the
+ *     token's rows for the block in increasing j with moe_combine's fp32
+ *     chain and rounds once: the bits of moe_combine, whatever order the
+ *     tiles finish in.  The up projection zeroes the counters first.
+ * Tokens with every slot dropped get a zero row.  fp32 linear experts run
+ * moe_expert_ffn into the workspace's y_perm, then the combine kernel.
  *   x_perm, offsets, perm_token, dest, gates: moe_dispatch's (and
- *   moe_route's) outputs; W_in, W_up, W_out as in moe_expert_ffn;
+ *   moe_route's) outputs, mutually consistent (dest[t, j] >= 0 is the
+ *   grouped row whose perm_token is t); a perm_token outside [0, T) or a
+ *   dest at or beyond T * top_k is recorded on the error word (code 3) and
+ *   skipped.  W_in, W_up, W_out as in moe_expert_ffn;
  *   output (T, d_out) act_dtype out. */
 int moe_expert_ffn_combine(const moe_config_t* cfg, const void* x_perm, const int32_t* offsets,
                            const int32_t* perm_token, const int32_t* dest, const float* gates,
                            const void* W_in, const void* W_up, const void* W_out, void* output,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Which form moe_forward uses for the experts and the combine: *fused = 1
+ * when it is moe_expert_ffn_combine's combine in the down projection's
+ * epilogue, 0 when it is moe_expert_ffn then moe_combine (fp32 linear
+ * experts always; bf16 top_k > 1 unless the hidden width is at least 4096
+ * and there are at least 1024 * E grouped rows, where the epilogue's extra
+ * reads hide behind long tiles: measured on B200, 0.994x the two-call time
+ * at the Mixtral shape, 1.18x at E = 64, top_k = 6, d_hidden = 1408).
+ * Host-only: no CUDA call.  Returns MOE_OK, or the config check's status. */
+int moe_forward_combine_fused(const moe_config_t* cfg, int32_t* fused);
 
 /* Combine: output[t] = sum over j = 0..top_k-1 with dest[t,j] >= 0 of
  * gates[t,j] * y_perm[dest[t,j]], accumulated in fp32 in increasing j,
@@ -373,7 +394,10 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest
  *   output (T, d_out) act_dtype, expert_indices (T, top_k) int32,
  *   gates (T, top_k) fp32, aux_loss (1) fp32 -- all device pointers;
  *   counts (E) int32 and drop_mask (T, top_k) uint8 are optional (NULL).
- * Inputs as in moe_route and moe_expert_ffn.  Intermediates live in ws. */
+ * Inputs as in moe_route and moe_expert_ffn.  Intermediates live in ws.
+ * The experts and the combine run as moe_expert_ffn_combine, or as
+ * moe_expert_ffn into the workspace's y_perm followed by moe_combine, as
+ * moe_forward_combine_fused reports for cfg; the output bits are the same. */
 int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
                 const float* logit_bias, const float* noise,
                 const void* W_in, const void* W_up, const void* W_out,

@@ -55,6 +55,7 @@ _SIGNATURES = {
     "moe_expert_ffn_gather": (ctypes.c_int, [_c_p] * 9 + [ctypes.c_size_t, _c_p]),
     "moe_combine": (ctypes.c_int, [_c_p] * 6),
     "moe_expert_ffn_combine": (ctypes.c_int, [_c_p] * 11 + [ctypes.c_size_t, _c_p]),
+    "moe_forward_combine_fused": (ctypes.c_int, [_c_p, _c_p]),
     "moe_forward": (ctypes.c_int, [_c_p] * 15 + [ctypes.c_size_t, _c_p]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_error_message": (ctypes.c_char_p, []),
@@ -323,6 +324,16 @@ def moe_expert_ffn_combine(cfg, x_perm, offsets, perm_token, dest, gates, W_in, 
         ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(perm_token), _ptr(dest), _ptr(gates),
         _ptr(W_in), _ptr(W_up), _ptr(W_out), _ptr(output), _ptr(ws), ws.numel(), _stream(stream)),
         "moe_expert_ffn_combine")
+
+
+def moe_forward_combine_fused(cfg) -> bool:
+    """Whether moe_forward runs the combine in the down projection's epilogue
+    (moe_expert_ffn_combine) for cfg, rather than moe_expert_ffn then
+    moe_combine.  Host-only."""
+    out = ctypes.c_int32(0)
+    _check(load_library().moe_forward_combine_fused(ctypes.byref(cfg), ctypes.byref(out)),
+           "moe_forward_combine_fused")
+    return bool(out.value)
 
 
 def moe_combine(cfg, y_perm, dest, gates, output, stream=None) -> None:

@@ -14,6 +14,10 @@
 //            `expert_forward`)
 //   swiglu : out[:, c] = silu(acc_gate[:, c]) * acc_up[:, c]   (the SwiGLU
 //            expert the pages name; silu(z) = z / (1 + exp(-z)))
+//   scatter: the top-1 combine, gate * acc into the token's output row
+//   combine: the top-k combine (Algorithm 3's gate-weighted sum): acc kept in
+//            fp32 as for none, and the last of a token's kept rows to finish
+//            an output column block sums the token's rows into its output
 //
 // B200 design
 //  * One CTA per SM, persistent, 192 threads: warp 0 = TMA producer, warp 1 =
@@ -97,16 +101,24 @@ struct GemmArgs {
   const int32_t* offsets;
   const int32_t* perm;  // gathered A: grouped row r is row perm[r] of the A tensor (else null)
   int a_rows;           // rows of the A tensor (gathered A: tokens)
-  void* out;  // bf16 for kEpiRelu / kEpiSwiglu / kEpiScatter, fp32 for kEpiNone
+  void* out;  // bf16 for kEpiRelu / kEpiSwiglu / kEpiScatter / kEpiCombine, fp32 for kEpiNone
   int32_t* err;
   int E, K, N, rows_max;
   int n_tiles;  // output-column blocks
-  // kEpiScatter (top-1 combine in the epilogue): grouped row r is the only
-  // kept slot of token rows[r]; its output row is gates[token] * acc.
+  // kEpiScatter / kEpiCombine (the combine in the epilogue): grouped row r
+  // is a kept slot of token rows[r].  kEpiScatter (top_k = 1): the output
+  // row is gates[token] * acc.  kEpiCombine: acc goes to row r of yrows, then
+  // arrives on arrive[token * n_tiles + column block]; the last kept row of
+  // the token to arrive writes the output block.
   const int32_t* rows;
-  const float* gates;
-  const int32_t* dest;  // (T) slot of each token, -1 if dropped: that output row is zeroed
-  int T;
+  const float* gates;   // (T, top_k)
+  const int32_t* dest;  // (T, top_k) grouped row of each slot, -1 if dropped
+  int T, top_k;         // a token with no kept slot gets a zero output row
+  float* yrows;
+  unsigned* arrive;
+  // Any kernel: clear_words words set to 0 before the first tile.
+  unsigned* clear;
+  size_t clear_words;
   // Pair kernel: [0] the next tile to hand out, [1] CTAs finished; both 0
   // at launch and left at 0 by the last CTA to finish.
   unsigned* sched;
@@ -185,9 +197,18 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // output columns [n0, n0 + OUT_COLS) of `out` (row offset orow_off), masked to
 // N.  Every lane of the warp executes the tensor-memory loads (they are
 // warp-collective); only rows with `valid` store.
+// kEpiCombine: what a row's arrival left for the combine of its token.
+struct CombineRow {
+  int tok;
+  bool last;    // this row completed its token's kept slots for the block
+  int dj[8];    // the token's slots' grouped rows (-1: dropped or beyond top_k)
+  float gj[8];  // and gates
+};
+
 template <int EPI>
 __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
-                                                const GemmArgs& g, int prow = -1) {
+                                                const GemmArgs& g, int prow = -1,
+                                                CombineRow* cr = nullptr) {
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   if (EPI == kEpiScatter) {
     // orow_off is the grouped row; its token's output row gets gate * acc,
@@ -218,6 +239,65 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
                 make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
+    }
+  } else if (EPI == kEpiCombine) {
+    // orow_off is the grouped row r.  Its fp32 row goes to yrows (the
+    // combine's operand, and the backward's); the row then counts itself on
+    // its token's counter for this column block with release order.  The
+    // arrival that completes the token's kept slots (acquire order: every
+    // other kept row's block is visible) is marked in *cr; combine_last_rows
+    // sums those tokens once the accumulator is released.
+    const int r = (int)orow_off;
+    int tok = 0;
+    if (valid) {
+      tok = g.rows[r];
+      if (tok < 0 || tok >= g.T) {
+        report_error(g.err, kDevBadPerm);
+        valid = false;
+        tok = 0;
+      }
+    }
+    float* yrow = g.yrows + (size_t)r * g.N;
+#pragma unroll 1
+    for (int cc = 0; cc < OUT_COLS; cc += 32) {
+      uint32_t v32[32];
+      tmem_ld_32x32b_x32(tacc + cc, v32);
+      tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int col = n0 + cc + v * 4;
+          if (col < g.N)
+            *reinterpret_cast<uint4*>(yrow + col) =
+                make_uint4(v32[4 * v], v32[4 * v + 1], v32[4 * v + 2], v32[4 * v + 3]);
+        }
+      }
+    }
+    cr->tok = tok;
+    cr->last = false;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cr->dj[j] = -1;
+      cr->gj[j] = 0.f;
+    }
+    if (valid) {
+      int kept = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < g.top_k) {
+          int dd = g.dest[(size_t)tok * g.top_k + j];
+          if (dd >= g.rows_max) {
+            report_error(g.err, kDevBadPerm);
+            dd = -1;
+          }
+          cr->dj[j] = dd;
+          cr->gj[j] = g.gates[(size_t)tok * g.top_k + j];
+          kept += dd >= 0 ? 1 : 0;
+        }
+      }
+      const uint32_t old =
+          atom_add_acq_rel_gpu(g.arrive + (size_t)tok * g.n_tiles + n0 / BN, 1u);
+      cr->last = old + 1u == (uint32_t)kept;
     }
   } else if (EPI == kEpiSwiglu) {
 #pragma unroll 1
@@ -293,17 +373,100 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
   }
 }
 
-// kEpiScatter: the output rows of tokens whose only slot was dropped are
-// zero; the epilogue warps of every CTA write a strided share of them before
-// their first tile (no grouped row maps to such a token, so no tile writes it).
+// kEpiCombine, after the accumulator is released: the warp writes the
+// output block [n0, n0 + BN) of every token one of its lanes completed, two
+// tokens per round.  Each lane owns 8 columns, so every slot row is read as
+// one coalesced 1 KiB segment, all of a round's rows in flight at once; each
+// element is the combine's fp32 chain over the slots in increasing j, then
+// one rounding to bf16.  The rows were written by this warp's lanes (ordered
+// by the warp barrier) or released by other rows' arrivals, which the lane
+// that completed the token acquired.
+__device__ __forceinline__ void combine_last_rows(const GemmArgs& g, const CombineRow& cr, int n0,
+                                                  int lane) {
+  uint32_t m = __ballot_sync(0xffffffffu, cr.last);
+  if (m == 0u) return;
+  __syncwarp();
+  const int col = n0 + 8 * lane;
+  const bool colok = col < g.N;  // N is a multiple of 8: all 8 columns or none
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
+  while (m != 0u) {
+    int src[2];
+    src[0] = __ffs(m) - 1;
+    m &= m - 1u;
+    const bool two = m != 0u;
+    src[1] = two ? __ffs(m) - 1 : src[0];
+    if (two) m &= m - 1u;
+    int tok[2], d[2][8];
+    float gg[2][8];
+    float4 ya[2][8], yb[2][8];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      tok[p] = __shfl_sync(0xffffffffu, cr.tok, src[p]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        d[p][j] = __shfl_sync(0xffffffffu, cr.dj[j], src[p]);
+        gg[p][j] = __shfl_sync(0xffffffffu, cr.gj[j], src[p]);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ya[p][j] = yb[p][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (colok && (p == 0 || two) && d[p][j] >= 0) {
+          const float4* y = reinterpret_cast<const float4*>(g.yrows + (size_t)d[p][j] * g.N + col);
+          ya[p][j] = __ldcg(y);
+          yb[p][j] = __ldcg(y + 1);
+        }
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      if (!colok || (p == 1 && !two)) continue;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (d[p][j] < 0) continue;
+        acc[0] = fmaf(gg[p][j], ya[p][j].x, acc[0]);
+        acc[1] = fmaf(gg[p][j], ya[p][j].y, acc[1]);
+        acc[2] = fmaf(gg[p][j], ya[p][j].z, acc[2]);
+        acc[3] = fmaf(gg[p][j], ya[p][j].w, acc[3]);
+        acc[4] = fmaf(gg[p][j], yb[p][j].x, acc[4]);
+        acc[5] = fmaf(gg[p][j], yb[p][j].y, acc[5]);
+        acc[6] = fmaf(gg[p][j], yb[p][j].z, acc[6]);
+        acc[7] = fmaf(gg[p][j], yb[p][j].w, acc[7]);
+      }
+      *reinterpret_cast<uint4*>(out + (size_t)tok[p] * g.N + col) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+  }
+}
+
+// kEpiScatter / kEpiCombine: the output rows of tokens with every slot
+// dropped are zero; the epilogue warps of every CTA write a strided share of
+// them before their first tile (no grouped row maps to such a token, so no
+// tile writes it).
 __device__ __forceinline__ void zero_dropped_rows(const GemmArgs& g, int warp, int lane) {
   const int w = (int)blockIdx.x * 4 + (warp - 2), nw = (int)gridDim.x * 4;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
   for (int t = w; t < g.T; t += nw) {
-    if (g.dest[t] >= 0) continue;
+    bool kept = false;
+    for (int j = 0; j < g.top_k; ++j) kept = kept || g.dest[(size_t)t * g.top_k + j] >= 0;
+    if (kept) continue;
     uint4* row = reinterpret_cast<uint4*>(out + (size_t)t * g.N);
     for (int v = lane; v < g.N / 8; v += 32) row[v] = make_uint4(0, 0, 0, 0);
   }
+}
+
+// g.clear: the epilogue warps of every CTA zero a strided share of the words
+// before their first tile.
+__device__ __forceinline__ void clear_words(const GemmArgs& g, int warp, int lane) {
+  const size_t i0 = ((size_t)blockIdx.x * 4 + (size_t)(warp - 2)) * 32 + (size_t)lane;
+  const size_t n = (size_t)gridDim.x * 128;
+  for (size_t i = i0; i < g.clear_words; i += n) g.clear[i] = 0u;
 }
 
 template <int EPI, bool GATHER>
@@ -498,7 +661,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp >= 2) {
     // ------------------------------------------------------ epilogue
-    if (EPI == kEpiScatter) zero_dropped_rows(g, warp, lane);
+    if (EPI == kEpiScatter || EPI == kEpiCombine) zero_dropped_rows(g, warp, lane);
+    if (g.clear != nullptr) clear_words(g, warp, lane);
     const int q = warp & 3;               // TMEM lane quarter of this warp
     const int row = q * 32 + lane;        // row inside the tile
     int acc = 0;
@@ -513,12 +677,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
-      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
-                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      const size_t orow_off = (EPI == kEpiScatter || EPI == kEpiCombine)
+                                  ? (size_t)(c.m0 + (valid ? row : 0))
+                                  : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow);
+      CombineRow cr;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr);
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[acc]);
+      if (EPI == kEpiCombine) combine_last_rows(g, cr, n0, lane);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -804,7 +971,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(drain_bar, 0)) report_error(g.err, kDevTimeoutDrain);
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue (both)
-    if (EPI == kEpiScatter) zero_dropped_rows(g, warp, lane);
+    if (EPI == kEpiScatter || EPI == kEpiCombine) zero_dropped_rows(g, warp, lane);
+    if (g.clear != nullptr) clear_words(g, warp, lane);
     const int q = warp & 3;
     const int row = (int)rank * BM + q * 32 + lane;  // row inside the pair tile
     int acc = 0;
@@ -828,13 +996,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after_sync();
       const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const bool valid = row < c.rows;
-      const size_t orow_off = EPI == kEpiScatter ? (size_t)(c.m0 + (valid ? row : 0))
-                                                 : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
+      const size_t orow_off = (EPI == kEpiScatter || EPI == kEpiCombine)
+                                  ? (size_t)(c.m0 + (valid ? row : 0))
+                                  : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow);
+      CombineRow cr;
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
+      if (EPI == kEpiCombine) combine_last_rows(g, cr, n0, lane);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -905,6 +1076,10 @@ cudaError_t run_gemm_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUt
 
 }  // namespace
 
+size_t grouped_gemm_arrive_words(int T, int N) {
+  return (size_t)std::max(T, 0) * (size_t)ceil_div(std::max(N, 1), BN);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
@@ -922,13 +1097,20 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
                                 cudaStream_t s, const int32_t* perm, int a_rows,
-                                const ScatterCombine* sc, float* pre) {
+                                const ScatterCombine* sc, float* pre, unsigned* clear,
+                                size_t clear_words) {
   if (rows_max == 0) return cudaSuccess;
   if (pre != nullptr && epi != kEpiSwiglu && epi != kEpiRelu) return cudaErrorInvalidValue;
   if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
   const bool gather = perm != nullptr;
   if (gather && (epi == kEpiNone || epi == kEpiScatter || a_rows <= 0)) return cudaErrorInvalidValue;
-  if ((epi == kEpiScatter) != (sc != nullptr)) return cudaErrorInvalidValue;
+  const bool combine = epi == kEpiScatter || epi == kEpiCombine;
+  if (combine != (sc != nullptr)) return cudaErrorInvalidValue;
+  if (combine && (sc->top_k < 1 || sc->top_k > 8 || (epi == kEpiScatter && sc->top_k != 1) ||
+                  (epi == kEpiCombine && (sc->y == nullptr || sc->arrive == nullptr))))
+    return cudaErrorInvalidValue;
+  if (gather && epi == kEpiCombine) return cudaErrorInvalidValue;
+  if ((clear == nullptr) != (clear_words == 0)) return cudaErrorInvalidValue;
   CUtensorMap ta, tb0, tb1;
   const bool a_ok = gather ? encode_a(&ta, A, a_rows, K, 1) : encode_a(&ta, A, rows_max, K);
   if (!a_ok || !encode_b(&tb0, B0, E, K, N) ||
@@ -950,6 +1132,11 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
   g.gates = sc != nullptr ? sc->gates : nullptr;
   g.dest = sc != nullptr ? sc->dest : nullptr;
   g.T = sc != nullptr ? sc->T : 0;
+  g.top_k = sc != nullptr ? sc->top_k : 0;
+  g.yrows = sc != nullptr ? sc->y : nullptr;
+  g.arrive = sc != nullptr ? sc->arrive : nullptr;
+  g.clear = clear;
+  g.clear_words = clear_words;
   g.sched = sched;
   g.pre = pre;
   g.pre_Rp = pre != nullptr ? expert_backward_pad_rows(rows_max, E) : 0;
@@ -968,6 +1155,7 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
       case kEpiSwiglu: return run_gemm_pair<kEpiSwiglu, false>(ta, tb0, tb1, g, pairs, s);
       case kEpiRelu: return run_gemm_pair<kEpiRelu, false>(ta, tb0, tb1, g, pairs, s);
       case kEpiScatter: return run_gemm_pair<kEpiScatter, false>(ta, tb0, tb1, g, pairs, s);
+      case kEpiCombine: return run_gemm_pair<kEpiCombine, false>(ta, tb0, tb1, g, pairs, s);
       default: return run_gemm_pair<kEpiNone, false>(ta, tb0, tb1, g, pairs, s);
     }
   }
@@ -980,6 +1168,7 @@ cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, i
     case kEpiSwiglu: return run_gemm<kEpiSwiglu, false>(ta, tb0, tb1, g, grid, s);
     case kEpiRelu: return run_gemm<kEpiRelu, false>(ta, tb0, tb1, g, grid, s);
     case kEpiScatter: return run_gemm<kEpiScatter, false>(ta, tb0, tb1, g, grid, s);
+    case kEpiCombine: return run_gemm<kEpiCombine, false>(ta, tb0, tb1, g, grid, s);
     default: return run_gemm<kEpiNone, false>(ta, tb0, tb1, g, grid, s);
   }
 }

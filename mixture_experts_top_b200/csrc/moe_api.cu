@@ -120,35 +120,55 @@ cudaError_t run_experts(const moe_config_t& c, const void* A, const int32_t* per
                              offsets, y_perm, err, sched, s);
 }
 
-// The experts and the combine: for top_k = 1 with bf16 experts the combine
-// is the down projection's epilogue (gate * row written straight into the
-// token's output row; tokens whose slot was dropped get a zero row), so no
-// y_perm is written and no combine kernel runs; otherwise the experts write
-// y_perm (in the workspace) and the combine kernel sums each token's rows.
+// Whether moe_forward runs the combine in the down projection's epilogue.
+// Top-1 always (no y_perm at all).  Top-k: the epilogue's extra work per
+// tile (write the row, count it, and for the tokens it completes read the
+// other slots' rows back) must hide behind the tile's main loop, which is
+// long only for a large hidden width and several tiles per CTA: on B200 the
+// fused form took 0.994x the time of experts + combine at the Mixtral shape
+// (d_hidden 14336), 1.002x at 64 tokens and 1.18x at E = 64, k = 6,
+// d_hidden 1408.
+bool fuse_combine(const moe_config_t& c) {
+  if (c.expert_kind == MOE_EXPERT_LINEAR) return false;
+  if (c.top_k == 1) return true;
+  return c.d_hidden >= 4096 && (int64_t)c.T * c.top_k >= (int64_t)1024 * c.E;
+}
+
+// The experts and the combine.  fused (bf16 experts only): the combine is
+// the down projection's epilogue.  top_k = 1: gate * row written straight
+// into the token's output row, so no y_perm is written.  top_k > 1: each row
+// also lands in y_perm, and the last of a token's kept rows to finish an
+// output column block sums the token's rows (the up projection zeroes the
+// arrival counters first).  Tokens with every slot dropped get a zero row.
+// Otherwise: y_perm, then the combine kernel.
 cudaError_t run_experts_combine(const moe_config_t& c, const void* x_perm,
                                 const int32_t* offsets, const int32_t* perm_token,
                                 const int32_t* dest, const float* gates, const void* W_in,
                                 const void* W_up, const void* W_out, void* output, void* ws,
-                                cudaStream_t s) {
+                                cudaStream_t s, bool fused) {
   const WsLayout L = workspace_layout(c);
-  if (c.top_k == 1 && c.expert_kind != MOE_EXPERT_LINEAR) {
+  void* y_perm = at<void>(ws, L.y_perm);
+  if (fused && c.expert_kind != MOE_EXPERT_LINEAR) {
     int32_t* err = at<int32_t>(ws, L.ctrl);
-    const int rows_max = c.T;
+    const int rows_max = c.T * c.top_k;
     __nv_bfloat16* hidden = at<__nv_bfloat16>(ws, L.hidden);
     unsigned* sched = at<unsigned>(ws, L.ctrl + kCtrlGemmSched);
+    const bool topk = c.top_k > 1;
+    unsigned* arrive = topk ? at<unsigned>(ws, L.arrive) : nullptr;
+    const size_t arrive_words = topk ? grouped_gemm_arrive_words(c.T, c.d_out) : 0;
     const int epi = c.expert_kind == MOE_EXPERT_SWIGLU ? kEpiSwiglu : kEpiRelu;
     cudaError_t e = launch_grouped_gemm(
         epi, static_cast<const __nv_bfloat16*>(x_perm), rows_max, c.d,
         static_cast<const __nv_bfloat16*>(W_in),
         epi == kEpiSwiglu ? static_cast<const __nv_bfloat16*>(W_up) : nullptr, c.d_hidden, c.E,
-        offsets, hidden, err, sched, s);
+        offsets, hidden, err, sched, s, nullptr, 0, nullptr, nullptr, arrive, arrive_words);
     if (e != cudaSuccess) return e;
-    const ScatterCombine sc{perm_token, gates, dest, c.T};
-    return launch_grouped_gemm(kEpiScatter, hidden, rows_max, c.d_hidden,
+    const ScatterCombine sc{perm_token, gates, dest, c.T, c.top_k,
+                            topk ? static_cast<float*>(y_perm) : nullptr, arrive};
+    return launch_grouped_gemm(topk ? kEpiCombine : kEpiScatter, hidden, rows_max, c.d_hidden,
                                static_cast<const __nv_bfloat16*>(W_out), nullptr, c.d_out, c.E,
                                offsets, output, err, sched, s, nullptr, 0, &sc);
   }
-  void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = run_experts(c, x_perm, nullptr, offsets, W_in, W_up, W_out, y_perm, ws, s);
   if (e != cudaSuccess) return e;
   return launch_combine(c, static_cast<const float*>(y_perm), dest, gates, output, s);
@@ -209,6 +229,9 @@ WsLayout workspace_layout(const moe_config_t& c) {
   L.x_perm = take(Tk * (size_t)c.d * s);
   L.hidden = take(c.expert_kind == MOE_EXPERT_LINEAR ? 0 : Tk * (size_t)c.d_hidden * 2);
   L.y_perm = take(Tk * (size_t)c.d_out * 4);
+  L.arrive = take(c.expert_kind != MOE_EXPERT_LINEAR && c.top_k > 1
+                      ? grouped_gemm_arrive_words(c.T, c.d_out) * 4
+                      : 0);
   const size_t nch = (size_t)route_backward_chunks(c.T, c.E);
   L.dlogits = take((size_t)c.T * E * 4);
   L.dw_part = take(nch * (size_t)c.d * E * 4);
@@ -767,8 +790,16 @@ int moe_expert_ffn_combine(const moe_config_t* cfg, const void* x_perm, const in
   if (c.T == 0) return MOE_OK;
   const cudaError_t e = run_experts_combine(c, x_perm, offsets, perm_token, dest, gates, W_in,
                                             W_up, W_out, output, ws,
-                                            reinterpret_cast<cudaStream_t>(stream));
+                                            reinterpret_cast<cudaStream_t>(stream), true);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_combine");
+}
+
+int moe_forward_combine_fused(const moe_config_t* cfg, int32_t* fused) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(fused);
+  *fused = fuse_combine(*cfg) ? 1 : 0;
+  return MOE_OK;
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* dest,
@@ -837,7 +868,8 @@ int moe_forward(const moe_config_t* cfg, const void* x, const float* W_router,
   // The materialised permute (one copy of each kept row, ~38 us at the
   // Mixtral shape) is far cheaper than gathering A rows inside the GEMM,
   // which re-fetches them for every output column block.
-  e = run_experts_combine(c, x_perm, offs, perm, dest, gates, W_in, W_up, W_out, output, ws, s);
+  e = run_experts_combine(c, x_perm, offs, perm, dest, gates, W_in, W_up, W_out, output, ws, s,
+                          fuse_combine(c));
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward/experts+combine");
   return MOE_OK;
 }

@@ -439,6 +439,20 @@ __device__ __forceinline__ void pdl_wait_and_release() {
 
 // ------------------------------------------------------------- small utils --
 
+// *p += v at GPU scope with acquire-release order: the calling thread's
+// earlier writes become visible to any thread whose later acquire operation
+// on *p reads this add's result (or a later one in the chain of adds), and
+// writes released by the adds this one reads from are visible to the
+// calling thread's later reads.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

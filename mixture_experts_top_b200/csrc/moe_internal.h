@@ -41,6 +41,7 @@ struct WsLayout {
   size_t x_perm;         // (T*k, d) act
   size_t hidden;         // (T*k, d_hidden) bf16
   size_t y_perm;         // (T*k, d_out) fp32
+  size_t arrive;         // (T, d_out / 256) uint32: the top-k combine's arrival counters
   size_t dlogits;        // (T, E) fp32: moe_route_backward's logit gradient
   size_t dw_part;        // (chunks, d, E) fp32: per-chunk partial dW_router
   size_t dbias_part;     // (chunks, E) fp32
@@ -182,14 +183,24 @@ cudaError_t launch_linear_expert(const moe_config_t& c, const float* x_perm,
 // (bf16 output; B0 = gate, B1 = up; each output column pairs one gate and
 // one up column), 3 = the top-1 combine (bf16 output rows of tokens: grouped
 // row r writes gates[t] * acc into row t = rows[r]; tokens with dest[t] < 0
-// get a zero row).
-enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2, kEpiScatter = 3 };
+// get a zero row), 4 = the top-k combine (fp32 rows into y, as epi 0; the
+// last of a token's kept rows to finish a column block sums the token's rows
+// in slot order into its bf16 output row; tokens with every slot dropped get
+// a zero row).
+enum GemmEpilogue { kEpiNone = 0, kEpiRelu = 1, kEpiSwiglu = 2, kEpiScatter = 3, kEpiCombine = 4 };
 struct ScatterCombine {
   const int32_t* rows;   // (rows) token of each grouped row (perm_token)
-  const float* gates;    // (T) the single slot's gate
-  const int32_t* dest;   // (T) the single slot's grouped row, -1 if dropped
+  const float* gates;    // (T, top_k) the slots' gates
+  const int32_t* dest;   // (T, top_k) the slots' grouped rows, -1 if dropped
   int T;
+  int top_k;             // 1 for kEpiScatter
+  float* y;              // kEpiCombine: (rows, N) fp32 expert rows (y_perm)
+  // kEpiCombine: grouped_gemm_arrive_words(T, N) arrival counters, 0 at
+  // launch (the up projection's `clear` zeroes them).
+  unsigned* arrive;
 };
+// Arrival counters kEpiCombine needs for T tokens and N output columns.
+size_t grouped_gemm_arrive_words(int T, int N);
 
 // perm != nullptr (ReLU / SwiGLU only): grouped row r of A is row perm[r] of
 // A, an (a_rows, K) tensor, fetched by TMA row gathers (the permute fused into
@@ -199,11 +210,14 @@ struct ScatterCombine {
 // pre (kEpiSwiglu / kEpiRelu only, or null): also write every kept row's fp32
 // pre-activations into the experts' backward layout (the `pre` region of its
 // workspace, expert_backward_layout), for moe_expert_ffn_backward_saved.
+// clear (or null): clear_words words the epilogue warps set to 0 before
+// their first tile (the next launch's kEpiCombine arrival counters).
 cudaError_t launch_grouped_gemm(int epi, const __nv_bfloat16* A, int rows_max, int K,
                                 const __nv_bfloat16* B0, const __nv_bfloat16* B1, int N, int E,
                                 const int32_t* offsets, void* out, int32_t* err, unsigned* sched,
                                 cudaStream_t s, const int32_t* perm = nullptr, int a_rows = 0,
-                                const ScatterCombine* sc = nullptr, float* pre = nullptr);
+                                const ScatterCombine* sc = nullptr, float* pre = nullptr,
+                                unsigned* clear = nullptr, size_t clear_words = 0);
 
 // Experts' backward (expert_backward.cu, grouped_gemm_bwd.cu).  The bf16
 // GEMMs work on a padded grouped layout: each expert's rows rounded up to a

@@ -74,6 +74,10 @@ class ShardStep:
         self.perm = torch.empty(T * k, **i32)
         self.f = torch.empty(E, dtype=torch.float32, device=dev)
         self.x_perm = torch.empty((T * k, cfg.d), dtype=act, device=dev)
+        # the experts and the combine in the form moe_forward uses for cfg
+        self.fused = api.moe_forward_combine_fused(cfg)
+        self.y_perm = None if self.fused else torch.empty((T * k, cfg.d_out),
+                                                          dtype=torch.float32, device=dev)
         self.out = ForwardOutputs(
             output=torch.empty((T, cfg.d_out), dtype=act, device=dev),
             expert_indices=torch.empty((T, k), **i32),
@@ -101,8 +105,13 @@ class ShardStep:
         api.moe_dispatch_shard(cfg, self.rank, self.world, self.T_global, self.records, x,
                                o.expert_indices, None, o.counts, self.offsets, self.dest,
                                self.perm, o.drop_mask, self.f, o.aux_loss, self.x_perm, self.ws)
-        api.moe_expert_ffn_combine(cfg, self.x_perm, self.offsets, self.perm, self.dest, o.gates,
-                                   W_in, W_up, W_out, o.output, self.ws)
+        if self.fused:
+            api.moe_expert_ffn_combine(cfg, self.x_perm, self.offsets, self.perm, self.dest,
+                                       o.gates, W_in, W_up, W_out, o.output, self.ws)
+        else:
+            api.moe_expert_ffn(cfg, self.x_perm, self.offsets, W_in, W_up, W_out, self.y_perm,
+                               self.ws)
+            api.moe_combine(cfg, self.y_perm, self.dest, o.gates, o.output)
 
     def __call__(self, x, W_router, logit_bias, noise, W_in, W_up, W_out, gather=None):
         self.route(x, W_router, logit_bias, noise)

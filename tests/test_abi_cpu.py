@@ -20,7 +20,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(moe_lib):
     names = declared_functions()
-    assert len(names) == 26
+    assert len(names) == 27
     for n in names:
         assert hasattr(moe_lib, n), n
     assert sorted(api.exported_symbols()) == names
@@ -34,6 +34,23 @@ def _cfg(**kw):
 
 
 FAKE = 0x7F0000000000          # 256-aligned, never dereferenced
+
+
+@pytest.mark.parametrize("name,fused", [("mixtral", True), ("decode", False),
+                                        ("fine_grained", False), ("switch_relu", True),
+                                        ("tiny_linear", False)])
+def test_forward_combine_form(name, fused):
+    """moe_forward's form of the experts and the combine (host-only query):
+    in the down projection's epilogue at top-1 and where long tiles hide the
+    top-k epilogue's reads (Mixtral: d_hidden 14336, 16384 grouped rows), as
+    two calls otherwise (64 tokens; d_hidden 1408; fp32 linear experts)."""
+    from workloads import WORKLOADS
+    w = WORKLOADS[name]
+    cfg = api.make_config(w.T, w.d, w.d_hidden, w.d_out, w.E, w.top_k, w.kind, w.dtype,
+                          w.capacity_factor)
+    assert api.moe_forward_combine_fused(cfg) is fused
+    with pytest.raises(RuntimeError):
+        api.moe_forward_combine_fused(_cfg(top_k=0))
 
 
 @pytest.mark.parametrize("kw,status", [

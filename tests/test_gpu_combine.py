@@ -71,17 +71,27 @@ def test_combine_top1_gate_one_copies_row():
 
 
 @pytest.mark.parametrize("name,k,cf", [("switch_relu", 1, 1.25), ("mixtral", 1, 0.5),
-                                       ("mixtral", 1, 0.0), ("switch_relu", 2, 1.0)])
+                                       ("mixtral", 1, 0.0), ("switch_relu", 2, 1.0),
+                                       ("mixtral", 2, 0.25), ("mixtral", 2, 0.0),
+                                       ("fine_grained", 6, 1.0), ("fine_grained", 8, 0.5),
+                                       ("mixtral_pairs", 2, 0.0), ("mixtral_pairs", 3, 0.5)])
 def test_expert_ffn_combine_equals_ffn_then_combine(name, k, cf):
-    """moe_expert_ffn_combine: at top_k = 1 the combine runs in the down
-    projection's epilogue (no y_perm, dropped tokens zeroed there); it must
-    give the bits of moe_expert_ffn followed by moe_combine, drops included.
-    At top_k = 2 it is those two calls."""
+    """moe_expert_ffn_combine runs the combine in the down projection's
+    epilogue: at top_k = 1 gate * row goes straight to the token's row (no
+    y_perm); at top_k > 1 the last of a token's kept rows to finish a column
+    block sums the token's rows in slot order.  Either way it must give the
+    bits of moe_expert_ffn followed by moe_combine, drops included (tokens
+    with every slot dropped get a zero row), on the single-CTA and the
+    CTA-pair GEMM (mixtral_pairs: 1024 rows per expert or more)."""
     from gpu_util import cfg_of
     from workloads import WORKLOADS, make_inputs
     base = {"switch_relu": WORKLOADS["switch_relu"].replace(T=1500, d=256, d_hidden=512,
                                                             d_out=256),
-            "mixtral": WORKLOADS["mixtral"].replace(T=900, d=256, d_hidden=384, d_out=264)}[name]
+            "mixtral": WORKLOADS["mixtral"].replace(T=900, d=256, d_hidden=384, d_out=264),
+            "fine_grained": WORKLOADS["fine_grained"].replace(T=1100, d=256, d_hidden=352,
+                                                              d_out=520),
+            "mixtral_pairs": WORKLOADS["mixtral"].replace(T=4100, d=256, d_hidden=512,
+                                                          d_out=776)}[name]
     w = base.replace(top_k=k, capacity_factor=cf)
     inp = make_inputs(w, seed=17)
     cfg = cfg_of(w)
@@ -110,7 +120,7 @@ def test_expert_ffn_combine_equals_ffn_then_combine(name, k, cf):
     torch.cuda.synchronize()
     assert api.moe_device_status(ws) == 0
     dropped = host(drop).all(axis=1)
-    if cf > 0 and k == 1:
+    if cf > 0 and (k == 1 or cf <= 0.25):
         assert dropped.any()
     g, r = host(got), host(ref)
     assert np.array_equal(g, r)

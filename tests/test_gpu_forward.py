@@ -23,6 +23,10 @@ REDUCED = {
     "mixtral": WORKLOADS["mixtral"].replace(T=600, d=512, d_hidden=1024, d_out=512),
     "fine_grained": WORKLOADS["fine_grained"].replace(T=1100, d=256, d_hidden=352, d_out=256),
     "decode": WORKLOADS["decode"].replace(d=512, d_hidden=1024, d_out=512),
+    # top-2 with the combine in the down projection's epilogue (hidden width
+    # 4096, 1024 grouped rows per expert), capacity drops included
+    "mixtral_fused_combine": WORKLOADS["mixtral"].replace(T=2048, d=256, d_hidden=4096,
+                                                          d_out=256, E=4, capacity_factor=0.9),
 }
 
 
@@ -77,6 +81,9 @@ def check_rows(w, got_rows, ref_rows, expert_rows):
 @pytest.mark.parametrize("name", list(REDUCED))
 def test_forward_reduced_all_tokens(name):
     w = REDUCED[name]
+    if name == "mixtral_fused_combine":
+        from mixture_experts_top_b200 import api
+        assert api.moe_forward_combine_fused(cfg_of(w))
     inp = make_inputs(w, seed=11)
     g = gpu_forward(w, inp)
     weights = {k: inp[k] for k in ("W_in", "W_up", "W_out")}

@@ -5,8 +5,9 @@ some as thread-block clusters, and the pair GEMM, the router and the
 dispatch keep counters in the workspace that the last CTA of each launch
 puts back to 0; a captured step must therefore replay any number of times
 and give the eager call's bits.  Checked on reduced Mixtral (top-2, pair
-GEMM), Switch (top-1, combine fused in the down projection, noise) and
-fine-grained (E = 64, capacity) shapes: one eager call, then the captured
+GEMM), Switch (top-1, combine fused in the down projection, noise), fine-grained
+(E = 64, capacity) and a top-2 shape whose combine runs in the down
+projection's epilogue: one eager call, then the captured
 call replayed on the same inputs and again on new tokens copied into the
 graph's input buffer, each replay against an eager call on those tokens.
 """
@@ -24,6 +25,10 @@ CASES = {
     "mixtral": WORKLOADS["mixtral"].replace(T=4096, d=512, d_hidden=1024, d_out=512),
     "switch_relu": WORKLOADS["switch_relu"].replace(T=1024, d=256, d_hidden=512, d_out=256),
     "fine_grained": WORKLOADS["fine_grained"].replace(T=1100, d=256, d_hidden=352, d_out=256),
+    # top-2 combine in the down projection's epilogue: its arrival counters,
+    # zeroed by the up projection, must be back at 0 for every replay
+    "mixtral_fused_combine": WORKLOADS["mixtral"].replace(T=2048, d=256, d_hidden=4096,
+                                                          d_out=256, E=4),
 }
 KEYS = ("output", "expert_indices", "gates", "aux_loss", "counts", "drop_mask")
 
