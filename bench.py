@@ -637,6 +637,8 @@ def run_ours(args, rank, world):
     w = WORKLOADS[args.workload]
     if args.tokens:
         w = w.with_tokens(args.tokens)
+    if args.hidden:
+        w = w.replace(d_hidden=args.hidden)
     peaks, peak_src = load_peaks()
 
     # inputs: weights identical on every rank, tokens drawn per rank
@@ -728,7 +730,7 @@ def run_ours(args, rank, world):
     regime = regime_of(elapsed_ms / 1e3)
     gemm = gemm_roofline(w, rows, used, stage_ms[2], peaks, peak_src, regime)
     # DRAM counters exist only for the captured workload (Mixtral shape, T = 8192).
-    captured = w.name == "mixtral" and T == 8192 and w.d == 4096
+    captured = w.name == "mixtral" and T == 8192 and w.d == 4096 and w.d_hidden == 14336
     gemm.update({
         "traffic": profiled_traffic("grouped_gemm.cu", "grouped_gemm_mixtral.md") if captured
                    else None,
@@ -744,7 +746,8 @@ def run_ours(args, rank, world):
 
     # The other configurations, each on this GPU after the main line's
     # timed region (tokens/s, end to end, and each stage against its bound).
-    if world == 1 and not args.no_extras and args.workload == WORKLOAD and not args.tokens:
+    if (world == 1 and not args.no_extras and args.workload == WORKLOAD and not args.tokens
+            and not args.hidden):
         wl = {}
         for name in ("decode", "fine_grained", "switch_relu", "tiny_linear"):
             try:
@@ -1046,6 +1049,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling; not a bench line)")
+    ap.add_argument("--hidden", type=int, default=0,
+                    help="override d_hidden (smaller cases for profiling; not a bench line)")
     ap.add_argument("--cpu-tokens", type=int, default=64,
                     help="tokens in the oracle's timed batch (cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

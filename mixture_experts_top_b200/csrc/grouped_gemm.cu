@@ -72,7 +72,11 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;             // two accumulator buffers
 constexpr int MAX_E = 256;
 constexpr int AUX_BYTES = 4096;               // barriers, tmem address, tile table
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + AUX_BYTES;
+// fp32 row epilogues: per epilogue warp a 32 x 32 staging block (rows padded
+// to 36 floats: conflict-free 16-byte writes by row and reads by column).
+constexpr int EPI_LD = 36;
+constexpr int EPI_BUF_BYTES = 4 * 32 * EPI_LD * 4;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + AUX_BYTES + EPI_BUF_BYTES;
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
 // B bf16 (10-12 = 1), A K-major (bit 15 = 0), B N-major (bit 16 = 1),
@@ -197,6 +201,79 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // output columns [n0, n0 + OUT_COLS) of `out` (row offset orow_off), masked to
 // N.  Every lane of the warp executes the tensor-memory loads (they are
 // warp-collective); only rows with `valid` store.
+// fp32 rows out of the epilogue, coalesced: the warp's 32 rows (lane = row,
+// v32 = its columns [col, col + 32)) go through the warp's staging block and
+// leave as 128-byte row segments, 8 lanes per row and 4 rows per store, rather
+// than as 32 scattered 16-byte pieces per store.  roff[i] / rok[i]: element
+// offset and validity of row 4 i + lane / 8 (from tile_row_slots).
+__device__ __forceinline__ void store_rows_f32(float* wbuf, const uint32_t (&v32)[32], float* base,
+                                               const size_t (&roff)[8], const bool (&rok)[8],
+                                               int col, int N, int lane) {
+  uint4* wrow = reinterpret_cast<uint4*>(wbuf + lane * EPI_LD);
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    wrow[v] = make_uint4(v32[4 * v], v32[4 * v + 1], v32[4 * v + 2], v32[4 * v + 3]);
+  __syncwarp();
+  const int c4 = lane & 7;
+  const bool col_ok = col + 4 * c4 < N;   // N is a multiple of 8: all 4 columns or none
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 val = *reinterpret_cast<const uint4*>(wbuf + (4 * i + (lane >> 3)) * EPI_LD + 4 * c4);
+    if (rok[i] && col_ok) *reinterpret_cast<uint4*>(base + roff[i] + col + 4 * c4) = val;
+  }
+  __syncwarp();
+}
+
+// bf16 rows out of the epilogue, the same way: the warp's 32 rows of 32
+// columns (pk = this lane's row, packed in pairs) leave as 64-byte row
+// segments, 4 lanes per row and 8 rows per store.  Rows of the staging block
+// are 80 bytes apart (conflict-free 16-byte writes by row).  roff[i] /
+// rok[i]: row 8 (i / 2) ... as given by tile_row_slots_bf16.
+constexpr int EPI_LD16 = 40;   // bf16 elements per staging row
+__device__ __forceinline__ void store_rows_bf16(float* wbuf, const uint32_t (&pk)[16],
+                                                __nv_bfloat16* base, const size_t (&roff)[4],
+                                                const bool (&rok)[4], int col, int N, int lane) {
+  __nv_bfloat16* buf = reinterpret_cast<__nv_bfloat16*>(wbuf);
+  uint4* wrow = reinterpret_cast<uint4*>(buf + lane * EPI_LD16);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) wrow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  __syncwarp();
+  const int c8 = lane & 3;
+  const bool col_ok = col + 8 * c8 < N;   // N is a multiple of 8
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 val =
+        *reinterpret_cast<const uint4*>(buf + (8 * i + (lane >> 2)) * EPI_LD16 + 8 * c8);
+    if (rok[i] && col_ok) *reinterpret_cast<uint4*>(base + roff[i] + col + 8 * c8) = val;
+  }
+  __syncwarp();
+}
+
+// Offsets and validity of the rows this lane stores in store_rows_bf16: row
+// 8 i + lane / 4 of the warp's 32.
+__device__ __forceinline__ void tile_row_slots_bf16(size_t off, bool ok, int lane,
+                                                    size_t (&roff)[4], bool (&rok)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int src = 8 * i + (lane >> 2);
+    roff[i] = __shfl_sync(0xffffffffu, (unsigned long long)off, src);
+    rok[i] = __shfl_sync(0xffffffffu, ok ? 1 : 0, src) != 0;
+  }
+}
+
+// Offsets (elements) and validity of the rows this lane stores in
+// store_rows_f32: row 4 i + lane / 8 of the warp's 32, whose own lanes hold
+// `off` and `ok`.
+__device__ __forceinline__ void tile_row_slots(size_t off, bool ok, int lane, size_t (&roff)[8],
+                                               bool (&rok)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int src = 4 * i + (lane >> 3);
+    roff[i] = __shfl_sync(0xffffffffu, (unsigned long long)off, src);
+    rok[i] = __shfl_sync(0xffffffffu, ok ? 1 : 0, src) != 0;
+  }
+}
+
 // kEpiCombine: what a row's arrival left for the combine of its token.
 struct CombineRow {
   int tok;
@@ -208,7 +285,7 @@ struct CombineRow {
 template <int EPI>
 __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
                                                 const GemmArgs& g, int prow = -1,
-                                                CombineRow* cr = nullptr) {
+                                                CombineRow* cr = nullptr, float* wbuf = nullptr) {
   constexpr int OUT_COLS = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   if (EPI == kEpiScatter) {
     // orow_off is the grouped row; its token's output row gets gate * acc,
@@ -220,25 +297,20 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
       valid = tok >= 0 && tok < g.T;
       if (valid) gate = g.gates[tok];
     }
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + (size_t)tok * g.N;
+    size_t roff[4];
+    bool rok[4];
+    tile_row_slots_bf16((size_t)tok * g.N, valid, threadIdx.x & 31, roff, rok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + cc, r);
       tmem_ld_wait();
-      if (valid) {
-        uint32_t pk[16];
+      uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(gate * __uint_as_float(r[2 * i]), gate * __uint_as_float(r[2 * i + 1]));
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int col = n0 + cc + v * 8;
-          if (col < g.N)
-            *reinterpret_cast<uint4*>(orow + col) =
-                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-      }
+      for (int i = 0; i < 16; ++i)
+        pk[i] = pack_bf16x2(gate * __uint_as_float(r[2 * i]), gate * __uint_as_float(r[2 * i + 1]));
+      store_rows_bf16(wbuf, pk, static_cast<__nv_bfloat16*>(g.out), roff, rok, n0 + cc, g.N,
+                      threadIdx.x & 31);
     }
   } else if (EPI == kEpiCombine) {
     // orow_off is the grouped row r.  Its fp32 row goes to yrows (the
@@ -257,21 +329,15 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
         tok = 0;
       }
     }
-    float* yrow = g.yrows + (size_t)r * g.N;
+    size_t roff[8];
+    bool rok[8];
+    tile_row_slots((size_t)r * g.N, valid, threadIdx.x & 31, roff, rok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t v32[32];
       tmem_ld_32x32b_x32(tacc + cc, v32);
       tmem_ld_wait();
-      if (valid) {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int col = n0 + cc + v * 4;
-          if (col < g.N)
-            *reinterpret_cast<uint4*>(yrow + col) =
-                make_uint4(v32[4 * v], v32[4 * v + 1], v32[4 * v + 2], v32[4 * v + 3]);
-        }
-      }
+      store_rows_f32(wbuf, v32, g.yrows, roff, rok, n0 + cc, g.N, threadIdx.x & 31);
     }
     cr->tok = tok;
     cr->last = false;
@@ -300,6 +366,9 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
       cr->last = old + 1u == (uint32_t)kept;
     }
   } else if (EPI == kEpiSwiglu) {
+    size_t roff[4];
+    bool rok[4];
+    tile_row_slots_bf16(orow_off, valid, threadIdx.x & 31, roff, rok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t gr[32], ur[32];
@@ -310,65 +379,47 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
         store_pre32(g, 0, prow, n0 + cc, gr);
         store_pre32(g, 1, prow, n0 + cc, ur);
       }
-      if (valid) {
-        uint32_t pk[16];
+      uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
-          const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
-          pk[i] = pack_bf16x2(h0, h1);
-        }
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int col = n0 + cc + v * 8;
-          if (col < g.N)
-            *reinterpret_cast<uint4*>(orow + col) =
-                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+        const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+        pk[i] = pack_bf16x2(h0, h1);
       }
+      store_rows_bf16(wbuf, pk, static_cast<__nv_bfloat16*>(g.out), roff, rok, n0 + cc, g.N,
+                      threadIdx.x & 31);
     }
   } else if (EPI == kEpiNone) {
+    size_t roff[8];
+    bool rok[8];
+    tile_row_slots(orow_off, valid, threadIdx.x & 31, roff, rok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + cc, r);
       tmem_ld_wait();
-      if (valid) {
-        float* orow = static_cast<float*>(g.out) + orow_off;
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int col = n0 + cc + v * 4;
-          if (col < g.N)
-            *reinterpret_cast<uint4*>(orow + col) =
-                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-        }
-      }
+      store_rows_f32(wbuf, r, static_cast<float*>(g.out), roff, rok, n0 + cc, g.N,
+                     threadIdx.x & 31);
     }
   } else {
+    size_t roff[4];
+    bool rok[4];
+    tile_row_slots_bf16(orow_off, valid, threadIdx.x & 31, roff, rok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + cc, r);
       tmem_ld_wait();
       if (valid && prow >= 0) store_pre32(g, 0, prow, n0 + cc, r);
-      if (valid) {
-        uint32_t pk[16];
+      uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float v0 = fmaxf(__uint_as_float(r[2 * i]), 0.f);
-          const float v1 = fmaxf(__uint_as_float(r[2 * i + 1]), 0.f);
-          pk[i] = pack_bf16x2(v0, v1);
-        }
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(g.out) + orow_off;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int col = n0 + cc + v * 8;
-          if (col < g.N)
-            *reinterpret_cast<uint4*>(orow + col) =
-                make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const float v0 = fmaxf(__uint_as_float(r[2 * i]), 0.f);
+        const float v1 = fmaxf(__uint_as_float(r[2 * i + 1]), 0.f);
+        pk[i] = pack_bf16x2(v0, v1);
       }
+      store_rows_bf16(wbuf, pk, static_cast<__nv_bfloat16*>(g.out), roff, rok, n0 + cc, g.N,
+                      threadIdx.x & 31);
     }
   }
 }
@@ -663,6 +714,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------ epilogue
     if (EPI == kEpiScatter || EPI == kEpiCombine) zero_dropped_rows(g, warp, lane);
     if (g.clear != nullptr) clear_words(g, warp, lane);
+    float* wbuf = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + AUX_BYTES) +
+                  (warp - 2) * 32 * EPI_LD;
     const int q = warp & 3;               // TMEM lane quarter of this warp
     const int row = q * 32 + lane;        // row inside the tile
     int acc = 0;
@@ -682,7 +735,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                   : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
       CombineRow cr;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr);
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr, wbuf);
       tc_fence_before_sync();
       mbar_arrive(&tempty_bar[acc]);
       if (EPI == kEpiCombine) combine_last_rows(g, cr, n0, lane);
@@ -730,7 +783,7 @@ constexpr int kTileQ = 4;                         // tile indices published ahea
 constexpr int kTileQConsumers = 1 + 1 + 4 + 4;
 constexpr int P_STAGES = 6;
 constexpr int P_STAGE_BYTES = A_STAGE + B_STAGE / 2;  // 32 KiB
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + AUX_BYTES + EPI_BUF_BYTES;
 constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
 
@@ -973,6 +1026,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------ epilogue (both)
     if (EPI == kEpiScatter || EPI == kEpiCombine) zero_dropped_rows(g, warp, lane);
     if (g.clear != nullptr) clear_words(g, warp, lane);
+    float* wbuf = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES + AUX_BYTES) +
+                  (warp - 2) * 32 * EPI_LD;
     const int q = warp & 3;
     const int row = (int)rank * BM + q * 32 + lane;  // row inside the pair tile
     int acc = 0;
@@ -1001,7 +1056,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                   : (size_t)(c.m0 + (valid ? row : 0)) * g.N;
       const int prow = g.pre != nullptr ? poff[c.e] + (c.m0 - row_off[c.e]) + row : -1;
       CombineRow cr;
-      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr);
+      store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr, wbuf);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
