@@ -24,7 +24,8 @@
 //             (chunk bases) and the total count; kept, offsets, f and aux = E
 //             * sum f_e P_e (fp64, fixed-order butterfly).
 //   scatter - one warp per token: dest, drop mask, perm_token, and the copy
-//             of x[t] into every kept grouped row with 16-byte vectors
+//             of x[t] into every kept grouped row with 16-byte vectors (the
+//             row's loads issued before the dependent index loads)
 //             (skipped when x_perm is null: the up projection then gathers
 //             the rows through perm_token itself).
 #include "moe_device.cuh"
@@ -80,16 +81,33 @@ __device__ void dispatch_scan_body(const ScanArgs& a) {
   const int rank = a.rank, world = a.world, T_global = a.T_global;
   const int rec = 2 * E + 1;            // ints per exchange record
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nwarps) {
-    int carry = 0;
+  // A warp scans experts e0 + i * nwarps, i < 8, together: the 8 columns of
+  // a 32-chunk block are loaded at once, then scanned one by one.
+  for (int e0 = warp; e0 < E; e0 += 8 * nwarps) {
+    int carry[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) carry[i] = 0;
     for (int c0 = 0; c0 < nchunks; c0 += 32) {
       const int c = c0 + lane;
-      const int v = c < nchunks ? __ldcg(a.chunk_counts + (size_t)c * E + e) : 0;
-      const int incl = warp_inclusive_scan(v);
-      if (c < nchunks) a.chunk_base[(size_t)c * E + e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * nwarps;
+        v[i] = (c < nchunks && e < E) ? __ldcg(a.chunk_counts + (size_t)c * E + e) : 0;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * nwarps;
+        const int incl = warp_inclusive_scan(v[i]);
+        if (c < nchunks && e < E) a.chunk_base[(size_t)c * E + e] = carry[i] + incl - v[i];
+        carry[i] += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
-    if (lane == 0) s_counts[e] = carry;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = e0 + i * nwarps;
+      if (lane == 0 && e < E) s_counts[e] = carry[i];
+    }
   }
   // Sharded batch: this rank's tokens follow those of ranks 0..rank-1 in
   // the batch order, so a slot's position on its expert is offset by their
@@ -179,20 +197,30 @@ __global__ void __launch_bounds__(kCountWarps * 32)
   const int t1 = min(t0 + 32, T);
   const long s_begin = (long)t0 * k, s_end = (long)max(t1, t0) * k;
   const uint32_t lt = lanemask_lt();
-  for (long s0 = s_begin; s0 < s_end; s0 += 32) {
-    const long s = s0 + lane;
-    const bool valid = s < s_end;
-    int e = valid ? idx[s] : -1;
-    if (valid && (e < 0 || e >= E)) {
+  // The warp's 32 k slots, 32 at a time (k <= 8 rounds): every index load is
+  // issued first; each slot's expert and rank stay in registers until the
+  // ranks are final.
+  int ev[8], rv[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const long s = s_begin + 32 * it + lane;
+    ev[it] = (it < k && s < s_end) ? idx[s] : -2;   // -2: no slot
+  }
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    if (it >= k) break;
+    int e = ev[it];
+    if (e != -2 && (e < 0 || e >= E)) {
       report_error(err, kDevBadExpertIndex);
       e = -1;
     }
+    if (e == -2) e = -1;
+    ev[it] = e;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    const int r = (e >= 0) ? whist[warp][e] + __popc(peers & lt) : 0;
+    rv[it] = (e >= 0) ? whist[warp][e] + __popc(peers & lt) : 0;
     __syncwarp();
     if (e >= 0 && (peers & lt) == 0u) whist[warp][e] += __popc(peers);
     __syncwarp();
-    if (valid) local_rank[s] = r;
   }
   __syncthreads();
   // Exclusive scan over warps, per expert; the total is the chunk histogram.
@@ -207,12 +235,11 @@ __global__ void __launch_bounds__(kCountWarps * 32)
     chunk_counts[(size_t)c * E + e] = run;
   }
   __syncthreads();
-  for (long s0 = s_begin; s0 < s_end; s0 += 32) {
-    const long s = s0 + lane;
-    if (s < s_end) {
-      const int e = idx[s];
-      if (e >= 0 && e < E) local_rank[s] += wbase[warp][e];
-    }
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    if (it >= k) break;
+    const long s = s_begin + 32 * it + lane;
+    if (s < s_end) local_rank[s] = rv[it] + (ev[it] >= 0 ? wbase[warp][ev[it]] : 0);
   }
   // With `done`, the last chunk's CTA to finish runs the scan (all chunk
   // histograms are complete and visible by then), and leaves `done` at 0.
@@ -230,7 +257,10 @@ __global__ void __launch_bounds__(kCountWarps * 32)
   }
 }
 
-template <int ELEM>
+// PF: 16-byte vectors per lane loaded ahead, 32 * PF * 16 bytes of the row
+// (the whole row where it fits: a deeper buffer for short rows only costs
+// registers and occupancy).
+template <int ELEM, int PF>
 __global__ void __launch_bounds__(256)
     dispatch_scatter_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ idx,
                             int T, int k, int E, int d, int64_t cap,
@@ -246,6 +276,17 @@ __global__ void __launch_bounds__(256)
   const int nvec = d * ELEM / 16;  // 16-byte vectors per row
   const size_t row_bytes = (size_t)d * ELEM;
   for (int t = gw; t < T; t += nw) {
+    // The row's first 32 * PF vectors are loaded before the index work, so
+    // their latency overlaps the dependent index loads.
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
+    uint4 buf[PF];
+    if (x_perm != nullptr) {
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nvec) buf[i] = __ldg(src + v);
+      }
+    }
     int my_dest = -1;
     if (lane < k) {
       const size_t s = (size_t)t * k + lane;
@@ -263,9 +304,19 @@ __global__ void __launch_bounds__(256)
     int dj[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) dj[j] = __shfl_sync(0xffffffffu, my_dest, j);
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
+#pragma unroll
+    for (int i = 0; i < PF; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nvec) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k && dj[j] >= 0)
+            reinterpret_cast<uint4*>(x_perm + (size_t)dj[j] * row_bytes)[v] = buf[i];
+        }
+      }
+    }
 #pragma unroll 4
-    for (int v = lane; v < nvec; v += 32) {
+    for (int v = lane + 32 * PF; v < nvec; v += 32) {
       const uint4 val = __ldg(src + v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -320,7 +371,11 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
   if (c.T == 0) return cudaSuccess;
   const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
-  return launch_kernel(elem == 2 ? dispatch_scatter_kernel<2> : dispatch_scatter_kernel<4>, blocks,
+  // whole rows ahead up to 4 KiB (8 vectors a lane), else 8 KiB of the row
+  const bool deep = (size_t)c.d * elem > 32 * 8 * 16;
+  auto kern = elem == 2 ? (deep ? dispatch_scatter_kernel<2, 16> : dispatch_scatter_kernel<2, 8>)
+                        : (deep ? dispatch_scatter_kernel<4, 16> : dispatch_scatter_kernel<4, 8>);
+  return launch_kernel(kern, blocks,
                        256, 0, s, 0, static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d,
                        cap, chunk_base, local_rank, offsets, dest, perm_token, drop_mask,
                        static_cast<uint8_t*>(x_perm),
