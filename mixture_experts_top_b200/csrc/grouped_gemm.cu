@@ -737,7 +737,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       CombineRow cr;
       store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr, wbuf);
       tc_fence_before_sync();
-      mbar_arrive(&tempty_bar[acc]);
+      mbar_arrive_relaxed(&tempty_bar[acc]);   // the tile's stores need not drain first
       if (EPI == kEpiCombine) combine_last_rows(g, cr, n0, lane);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -1040,7 +1040,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const int tile = tile_q[slot];
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(cluster_smem_addr(&tq_empty[slot], 0));
+      // relaxed, so that it does not wait for the previous tile's stores; the
+      // condition on `tile` keeps it behind the slot's read
+      if (lane == 0 && tile >= 0) mbar_arrive_cluster_relaxed(cluster_smem_addr(&tq_empty[slot], 0));
       if (tile >= total_tiles) break;
       const TileCoord c = decode_tile<PBM>(tile, tile_prefix, row_off, E, g.n_tiles);
       const int n0 = c.n_tile * OUT_COLS;
@@ -1059,7 +1061,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       store_tile_rows<EPI>(tacc, valid, orow_off, n0, g, prow, &cr, wbuf);
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
+      if (lane == 0) mbar_arrive_leader_relaxed(&tempty_bar[acc]);   // stores need not drain
       if (EPI == kEpiCombine) combine_last_rows(g, cr, n0, lane);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;

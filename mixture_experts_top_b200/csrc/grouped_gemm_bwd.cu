@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(Cfg<STAGE>::THREADS, 1)
                              row_off, g);
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive_leader(&tempty_bar[acc]);
+      if (lane == 0) mbar_arrive_leader_relaxed(&tempty_bar[acc]);   // stores need not drain
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

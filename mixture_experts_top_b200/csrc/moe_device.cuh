@@ -427,6 +427,23 @@ __device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
                : "memory");
 }
 
+// Relaxed arrives: they order none of the thread's earlier memory accesses,
+// so they do not wait for its outstanding global stores.  For barriers that
+// only hand back a resource whose reads are complete, e.g. an accumulator in
+// tensor memory after tcgen05.wait::ld and tcgen05.fence::before_thread_sync,
+// or a queue slot whose value has been read into a register.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_leader_relaxed(uint64_t* bar) {
+  mbar_arrive_cluster_relaxed(leader_smem_addr(bar));
+}
+
 // --------------------------------------------- programmatic dependent launch --
 // Every kernel of the library is launched so that it may be scheduled while
 // the kernel before it in the stream is still draining.  Each kernel first
