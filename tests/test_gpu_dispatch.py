@@ -100,6 +100,17 @@ def test_dispatch_wide_rows():
     check(700, 4096, 8, 2, 0.0, idx, probs, _x(700, 4096, rng))
 
 
+@pytest.mark.parametrize("d,dtype", [(8, "bf16"), (1024, "f32"), (1032, "f32"), (2064, "bf16"),
+                                     (2056, "f32"), (6144, "bf16")])
+def test_dispatch_row_sizes(d, dtype):
+    """Row sizes around the scatter's load-ahead depths (whole rows of up to 4 KiB
+    with 8 vectors a lane, else the first 8 KiB with 16 and the rest after):
+    16 bytes, exactly 4 KiB, just over 4 KiB, just over 8 KiB, 12 KiB."""
+    rng = np.random.default_rng(d)
+    idx, probs = _random_routing(300, 8, 2, rng)
+    check(300, d, 8, 2, 1.0, idx, probs, _x(300, d, rng, dtype), dtype)
+
+
 def test_dispatch_all_on_one_expert_with_capacity():
     """Collapse: every token on expert 3, capacity keeps the first cap tokens."""
     T, E, k = 1000, 8, 1
