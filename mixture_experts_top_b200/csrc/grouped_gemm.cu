@@ -157,21 +157,6 @@ __device__ __forceinline__ void padded_offsets(const int* row_off, int E, bool o
   if (lane == 0) poff[0] = 0;
 }
 
-// The row's pre-activations for hidden units [h0, h0 + 32) of matrix p (0:
-// A, 1: B) from 32 fp32 accumulator columns.
-__device__ __forceinline__ void store_pre32(const GemmArgs& g, int p, int prow, int h0,
-                                            const uint32_t (&r)[32]) {
-  float* dst = g.pre + ((size_t)(p * g.pre_mt + h0 / kBwdPreBlock) * g.pre_Rp + prow) *
-                           kBwdPreBlock + (h0 % kBwdPreBlock);
-  // read only by the backward, much later: streamed past L2 (evict first)
-#pragma unroll
-  for (int v = 0; v < 8; ++v)
-    if (h0 + 4 * v < g.N)
-      __stcs(reinterpret_cast<float4*>(dst + 4 * v),
-             make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
-}
-
 struct TileCoord {
   int e, m0, rows, n_tile;
 };
@@ -206,22 +191,43 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)
 // leave as 128-byte row segments, 8 lanes per row and 4 rows per store, rather
 // than as 32 scattered 16-byte pieces per store.  roff[i] / rok[i]: element
 // offset and validity of row 4 i + lane / 8 (from tile_row_slots).
+// STREAM: evict-first stores (data read much later, e.g. by the backward).
+// The segment of row i lands at base + roff[i] + col; col_n is its column in
+// the matrix of N columns (the guard), equal to col except in blocked layouts.
+template <bool STREAM = false>
 __device__ __forceinline__ void store_rows_f32(float* wbuf, const uint32_t (&v32)[32], float* base,
                                                const size_t (&roff)[8], const bool (&rok)[8],
-                                               int col, int N, int lane) {
+                                               int col, int N, int lane, int col_n = -1) {
   uint4* wrow = reinterpret_cast<uint4*>(wbuf + lane * EPI_LD);
 #pragma unroll
   for (int v = 0; v < 8; ++v)
     wrow[v] = make_uint4(v32[4 * v], v32[4 * v + 1], v32[4 * v + 2], v32[4 * v + 3]);
   __syncwarp();
   const int c4 = lane & 7;
-  const bool col_ok = col + 4 * c4 < N;   // N is a multiple of 8: all 4 columns or none
+  const bool col_ok = (col_n < 0 ? col : col_n) + 4 * c4 < N;   // N is a multiple of 8
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint4 val = *reinterpret_cast<const uint4*>(wbuf + (4 * i + (lane >> 3)) * EPI_LD + 4 * c4);
-    if (rok[i] && col_ok) *reinterpret_cast<uint4*>(base + roff[i] + col + 4 * c4) = val;
+    if (rok[i] && col_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(base + roff[i] + col + 4 * c4);
+      if (STREAM)
+        __stcs(dst, val);
+      else
+        *dst = val;
+    }
   }
   __syncwarp();
+}
+
+// The warp's rows' pre-activations for hidden units [h0, h0 + 32) of matrix
+// p (0: A, 1: B), from 32 fp32 accumulator columns, through the staging
+// block: proff[i] = padded row * kBwdPreBlock of the lane's store rows.  Read
+// only by the backward, much later: streamed past L2 (evict first).
+__device__ __forceinline__ void store_pre32(float* wbuf, const GemmArgs& g, int p, int h0,
+                                            const uint32_t (&r)[32], const size_t (&proff)[8],
+                                            const bool (&prok)[8], int lane) {
+  float* base = g.pre + (size_t)(p * g.pre_mt + h0 / kBwdPreBlock) * g.pre_Rp * kBwdPreBlock;
+  store_rows_f32<true>(wbuf, r, base, proff, prok, h0 % kBwdPreBlock, g.N, lane, h0);
 }
 
 // bf16 rows out of the epilogue, the same way: the warp's 32 rows of 32
@@ -369,15 +375,21 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
     size_t roff[4];
     bool rok[4];
     tile_row_slots_bf16(orow_off, valid, threadIdx.x & 31, roff, rok);
+    const bool save = g.pre != nullptr;   // uniform: the training forward
+    size_t proff[8];
+    bool prok[8];
+    if (save)
+      tile_row_slots((size_t)(prow < 0 ? 0 : prow) * kBwdPreBlock, valid && prow >= 0,
+                     threadIdx.x & 31, proff, prok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t gr[32], ur[32];
       tmem_ld_32x32b_x32(tacc + cc, gr);
       tmem_ld_32x32b_x32(tacc + OUT_COLS + cc, ur);
       tmem_ld_wait();
-      if (valid && prow >= 0) {
-        store_pre32(g, 0, prow, n0 + cc, gr);
-        store_pre32(g, 1, prow, n0 + cc, ur);
+      if (save) {
+        store_pre32(wbuf, g, 0, n0 + cc, gr, proff, prok, threadIdx.x & 31);
+        store_pre32(wbuf, g, 1, n0 + cc, ur, proff, prok, threadIdx.x & 31);
       }
       uint32_t pk[16];
 #pragma unroll
@@ -405,12 +417,18 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
     size_t roff[4];
     bool rok[4];
     tile_row_slots_bf16(orow_off, valid, threadIdx.x & 31, roff, rok);
+    const bool save = g.pre != nullptr;   // uniform: the training forward
+    size_t proff[8];
+    bool prok[8];
+    if (save)
+      tile_row_slots((size_t)(prow < 0 ? 0 : prow) * kBwdPreBlock, valid && prow >= 0,
+                     threadIdx.x & 31, proff, prok);
 #pragma unroll 1
     for (int cc = 0; cc < OUT_COLS; cc += 32) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + cc, r);
       tmem_ld_wait();
-      if (valid && prow >= 0) store_pre32(g, 0, prow, n0 + cc, r);
+      if (save) store_pre32(wbuf, g, 0, n0 + cc, r, proff, prok, threadIdx.x & 31);
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
