@@ -98,8 +98,9 @@ __device__ void dispatch_scan_body(const ScanArgs& a) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int e = e0 + i * nwarps;
+        if (e >= E) break;   // warp-uniform
         const int incl = warp_inclusive_scan(v[i]);
-        if (c < nchunks && e < E) a.chunk_base[(size_t)c * E + e] = carry[i] + incl - v[i];
+        if (c < nchunks) a.chunk_base[(size_t)c * E + e] = carry[i] + incl - v[i];
         carry[i] += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
@@ -259,7 +260,8 @@ __global__ void __launch_bounds__(kCountWarps * 32)
 
 // PF: 16-byte vectors per lane loaded ahead, 32 * PF * 16 bytes of the row
 // (the whole row where it fits: a deeper buffer for short rows only costs
-// registers and occupancy).
+// registers and occupancy); 0 for small batches, where the launch with fewer
+// registers measured faster.
 template <int ELEM, int PF>
 __global__ void __launch_bounds__(256)
     dispatch_scatter_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ idx,
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(256)
     // The row's first 32 * PF vectors are loaded before the index work, so
     // their latency overlaps the dependent index loads.
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
-    uint4 buf[PF];
+    uint4 buf[PF > 0 ? PF : 1];
     if (x_perm != nullptr) {
 #pragma unroll
       for (int i = 0; i < PF; ++i) {
@@ -371,9 +373,13 @@ cudaError_t launch_dispatch(const moe_config_t& c, const void* x, const int32_t*
   if (c.T == 0) return cudaSuccess;
   const int elem = c.act_dtype == MOE_BF16 ? 2 : 4;
   const int blocks = min(ceil_div(c.T, 8), device_sm_count() * 16);
-  // whole rows ahead up to 4 KiB (8 vectors a lane), else 8 KiB of the row
+  // whole rows ahead up to 4 KiB (8 vectors a lane), else 8 KiB of the row;
+  // none below 1024 tokens
   const bool deep = (size_t)c.d * elem > 32 * 8 * 16;
-  auto kern = elem == 2 ? (deep ? dispatch_scatter_kernel<2, 16> : dispatch_scatter_kernel<2, 8>)
+  auto kern = c.T < 1024
+                  ? (elem == 2 ? dispatch_scatter_kernel<2, 0> : dispatch_scatter_kernel<4, 0>)
+                  : elem == 2
+                        ? (deep ? dispatch_scatter_kernel<2, 16> : dispatch_scatter_kernel<2, 8>)
                         : (deep ? dispatch_scatter_kernel<4, 16> : dispatch_scatter_kernel<4, 8>);
   return launch_kernel(kern, blocks,
                        256, 0, s, 0, static_cast<const uint8_t*>(x), idx, c.T, c.top_k, c.E, c.d,

@@ -102,13 +102,15 @@ def test_dispatch_wide_rows():
 
 @pytest.mark.parametrize("d,dtype", [(8, "bf16"), (1024, "f32"), (1032, "f32"), (2064, "bf16"),
                                      (2056, "f32"), (6144, "bf16")])
-def test_dispatch_row_sizes(d, dtype):
-    """Row sizes around the scatter's load-ahead depths (whole rows of up to 4 KiB
-    with 8 vectors a lane, else the first 8 KiB with 16 and the rest after):
-    16 bytes, exactly 4 KiB, just over 4 KiB, just over 8 KiB, 12 KiB."""
-    rng = np.random.default_rng(d)
-    idx, probs = _random_routing(300, 8, 2, rng)
-    check(300, d, 8, 2, 1.0, idx, probs, _x(300, d, rng, dtype), dtype)
+@pytest.mark.parametrize("T", [300, 1100])
+def test_dispatch_row_sizes(d, dtype, T):
+    """Row sizes around the scatter's load-ahead depths (from 1024 tokens: whole
+    rows of up to 4 KiB with 8 vectors a lane, else the first 8 KiB with 16 and
+    the rest after; below, none): 16 bytes, exactly 4 KiB, just over 4 KiB,
+    just over 8 KiB, 12 KiB."""
+    rng = np.random.default_rng(d + T)
+    idx, probs = _random_routing(T, 8, 2, rng)
+    check(T, d, 8, 2, 1.0, idx, probs, _x(T, d, rng, dtype), dtype)
 
 
 def test_dispatch_all_on_one_expert_with_capacity():
