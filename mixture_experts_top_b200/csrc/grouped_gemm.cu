@@ -72,8 +72,9 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;             // two accumulator buffers
 constexpr int MAX_E = 256;
 constexpr int AUX_BYTES = 4096;               // barriers, tmem address, tile table
-// fp32 row epilogues: per epilogue warp a 32 x 32 staging block (rows padded
-// to 36 floats: conflict-free 16-byte writes by row and reads by column).
+// Row epilogues: per epilogue warp a 32 x 32 staging block (fp32 rows padded
+// to 36 floats: conflict-free 16-byte writes by row and reads by column; bf16
+// rows use it at 40 elements a row).
 constexpr int EPI_LD = 36;
 constexpr int EPI_BUF_BYTES = 4 * 32 * EPI_LD * 4;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + AUX_BYTES + EPI_BUF_BYTES;
@@ -181,11 +182,6 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* prefix, co
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
-// Epilogue of one accumulator row held by this thread (TMEM lane = tile row):
-// reads the 256 accumulator columns in chunks of 32 and writes the row's
-// output columns [n0, n0 + OUT_COLS) of `out` (row offset orow_off), masked to
-// N.  Every lane of the warp executes the tensor-memory loads (they are
-// warp-collective); only rows with `valid` store.
 // fp32 rows out of the epilogue, coalesced: the warp's 32 rows (lane = row,
 // v32 = its columns [col, col + 32)) go through the warp's staging block and
 // leave as 128-byte row segments, 8 lanes per row and 4 rows per store, rather
@@ -234,7 +230,7 @@ __device__ __forceinline__ void store_pre32(float* wbuf, const GemmArgs& g, int 
 // columns (pk = this lane's row, packed in pairs) leave as 64-byte row
 // segments, 4 lanes per row and 8 rows per store.  Rows of the staging block
 // are 80 bytes apart (conflict-free 16-byte writes by row).  roff[i] /
-// rok[i]: row 8 (i / 2) ... as given by tile_row_slots_bf16.
+// rok[i]: row 8 i + lane / 4, from tile_row_slots_bf16.
 constexpr int EPI_LD16 = 40;   // bf16 elements per staging row
 __device__ __forceinline__ void store_rows_bf16(float* wbuf, const uint32_t (&pk)[16],
                                                 __nv_bfloat16* base, const size_t (&roff)[4],
@@ -288,6 +284,11 @@ struct CombineRow {
   float gj[8];  // and gates
 };
 
+// Epilogue of one accumulator row held by this thread (TMEM lane = tile row):
+// reads the 256 accumulator columns in chunks of 32 and writes the row's
+// output columns [n0, n0 + OUT_COLS) of `out` (row offset orow_off), masked to
+// N.  Every lane of the warp executes the tensor-memory loads (they are
+// warp-collective) and the staged stores; only rows with `valid` are written.
 template <int EPI>
 __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_t orow_off, int n0,
                                                 const GemmArgs& g, int prow = -1,
