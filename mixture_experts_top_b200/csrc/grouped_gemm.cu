@@ -325,7 +325,9 @@ __device__ __forceinline__ void store_tile_rows(uint32_t tacc, bool valid, size_
     // its token's counter for this column block with release order.  The
     // arrival that completes the token's kept slots (acquire order: every
     // other kept row's block is visible) is marked in *cr; combine_last_rows
-    // sums those tokens once the accumulator is released.
+    // sums those tokens once the accumulator is released.  The staged store
+    // writes row r's block from other lanes of the warp; the warp barrier
+    // that ends it orders those writes before this lane's releasing add.
     const int r = (int)orow_off;
     int tok = 0;
     if (valid) {
